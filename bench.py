@@ -1,0 +1,346 @@
+"""Benchmark of the SVDQuant NVFP4 W4A4 + low-rank linear (libsvdq) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload qkv]
+
+One step = one forward pass of the layer over one batch of synthetic tokens: K1
+(svdq_quant_act_lora_down: smoothing, NVFP4 activation quantization, low-rank down-projection)
+then K2 (svdq_gemm_w4a4_lora_up: block-scaled FP4 GEMM + low-rank up-projection + bias).
+Default workload: the FLUX-like fused QKV projection, M = 4608 tokens, K = 3072, N = 9216,
+rank 32. Inputs are resident in HBM when the timed region starts; successive steps rotate
+over three buffer sets (inputs, activations, outputs and layer copies, >3x the 126 MB L2) so
+that no step finds its operands in L2.
+
+Metric: layer TFLOPS = (2MNK + 2MNr + 2MKr) / step time, summed over ranks (weak scaling:
+every rank runs its own replica on its own batch, no collective on the data path).
+Rank 0 prints one JSON line. ``--impl reference`` times the fp64 CPU oracle instead (the
+only reference implementation of this method available here) on a bounded row sample.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from synth import CONFIGS, make_inputs  # noqa: E402
+
+METRIC = "W4A4+LoRA linear TFLOPS & fraction of B200 FP4 peak; quant-pass HBM GB/s"
+FP4_OVER_BF16 = 9.0 / 2.25  # nominal dense NVFP4 / BF16 tensor throughput ratio on B200
+L2_BYTES = 126 * 1024 * 1024
+
+
+def layer_flops(M, K, N, r):
+    return 2.0 * M * N * K + 2.0 * M * N * r + 2.0 * M * K * r
+
+
+def k1_bytes(M, K, r):
+    """Algorithmic HBM bytes of K1: read X, inv_lambda, L1; write codes, scales, lora_act."""
+    return 2.0 * M * K + 4.0 * K + 2.0 * K * r + M * K / 2 + M * K / 16 + 2.0 * M * r
+
+
+def k2_flops(M, K, N, r):
+    return 2.0 * M * N * K + 2.0 * M * N * r
+
+
+def read_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling while the timed region runs."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except FileNotFoundError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            out, _ = self.proc.communicate(timeout=10)
+            self.lines = [l for l in out.splitlines() if l.strip()]
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for l in self.lines:
+            f = [x.strip() for x in l.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def cpu_oracle_sample(shape, rows: int, seed: int = 0, budget_s: float = 20.0):
+    """Times the fp64 oracle's forward pass (quantize + down-projection + dequantized GEMM +
+    up-projection) on `rows` tokens of the workload; the SVD prepare is timed apart."""
+    from oracle import svdq_oracle as O
+    from synth import bf16_bits_to_f32
+
+    Xb, W, b, _ = make_inputs(shape, seed=seed)
+    X = bf16_bits_to_f32(Xb).astype(np.float64)
+    t0 = time.perf_counter()
+    layer = O.prepare(W, b, O.calibration_absmax(X), shape.rank)
+    t_prep = time.perf_counter() - t0
+    done, t_fwd, reps = 0, 0.0, 0
+    while t_fwd < budget_s and reps < 64:
+        sl = X[(reps * rows) % shape.M:(reps * rows) % shape.M + rows]
+        t0 = time.perf_counter()
+        O.layer_forward(sl, layer)
+        t_fwd += time.perf_counter() - t0
+        done += sl.shape[0]
+        reps += 1
+    try:
+        from threadpoolctl import threadpool_info
+
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    flops = layer_flops(done, shape.K, shape.N, shape.rank)
+    return {"value": flops / t_fwd / 1e12, "seconds": t_fwd, "tokens": done, "cores": threads,
+            "prepare_s": t_prep, "reps": reps}
+
+
+def run_reference(args, shape, rank, world):
+    if rank != 0:
+        return 0
+    rows = 256
+    res = cpu_oracle_sample(shape, rows, budget_s=max(5.0, min(60.0, 2.0 * args.steps)))
+    ms = res["seconds"] / res["reps"] * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": res["value"], "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": res["reps"], "warmup": 0, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": workload_name(shape), "M": shape.M, "K": shape.K, "N": shape.N, "rank": shape.rank},
+        "cpu_baseline": {"value": res["value"], "unit": "TFLOPS", "cores": res["cores"], "kind": "oracle",
+                         "sample": f"{res['reps']} slices of {rows} tokens ({res['tokens']} tokens) of the workload; "
+                                   f"fp64 numpy oracle forward pass, prepare (SVD) excluded ({res['prepare_s']:.1f} s)"},
+        "e2e": {"value": res["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_name(shape):
+    return f"{shape.name}: SVDQuant NVFP4 W4A4+LoRA linear M={shape.M} K={shape.K} N={shape.N} rank={shape.rank}"
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="qkv", choices=sorted(CONFIGS))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    args = ap.parse_args(argv)
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    shape = CONFIGS[args.workload]
+
+    if args.impl == "reference":
+        return run_reference(args, shape, rank, world)
+
+    import torch
+
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=torch.device("cuda", local))
+
+    from bit_rank_compensated_b200 import build, svdq
+
+    if not os.path.exists(svdq.LIB_PATH):
+        build.build()
+    svdq.load()
+
+    M, K, N, r = shape.M, shape.K, shape.N, shape.rank
+    Xb, W, b, _ = make_inputs(shape, seed=0)
+    dev = torch.device("cuda", local)
+    NB = 3  # rotating buffer sets
+    Xd0 = torch.from_numpy(Xb.view(np.int16)).to(dev).view(torch.bfloat16)
+    Wd = torch.from_numpy(W).to(dev)
+    bd = torch.from_numpy(b).to(dev)
+    ax = svdq.act_absmax(Xd0)
+    layers = [svdq.prepare_weights(Wd, bd, ax, r)]
+    for _ in range(NB - 1):
+        L = svdq.Layer(N, K, r, device=dev)
+        for name in ("wq", "ws", "inv_lambda", "lam", "L1t", "L2t", "bias"):
+            src = getattr(layers[0], name)
+            if src is not None:
+                getattr(L, name).copy_(src)
+        L.s.w_tensor_scale, L.s.x_tensor_scale = layers[0].s.w_tensor_scale, layers[0].s.x_tensor_scale
+        layers.append(L)
+    del Wd
+    Xs = [Xd0] + [Xd0.clone() for _ in range(NB - 1)]
+    bufs = [svdq.alloc_activations(M, layers[0], dev) for _ in range(NB)]
+    Ys = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(NB)]
+    set_bytes = (Xs[0].numel() * 2 + sum(t.numel() * t.element_size() for t in bufs[0] if t is not None)
+                 + Ys[0].numel() * 2 + layers[0].wq.numel() + layers[0].ws.numel())
+    stream = torch.cuda.current_stream()
+
+    def step(i):
+        j = i % NB
+        xq, xs, la = bufs[j]
+        svdq.quant_act_lora_down(Xs[j], layers[j], xq, xs, la, stream)
+        svdq.gemm_w4a4_lora_up(xq, xs, la, M, layers[j], Ys[j], stream)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert svdq.last_device_error() == 0
+
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
+           torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
+        if os.environ.get("CUDA_VISIBLE_DEVICES") else local
+    with ClockSampler(gpu_index) as clk:
+        if dist:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_start = torch.cuda.Event(enable_timing=True)
+        t_end = torch.cuda.Event(enable_timing=True)
+        t_start.record(stream)
+        for i in range(args.steps):
+            j = i % NB
+            xq, xs, la = bufs[j]
+            ev[i][0].record(stream)
+            svdq.quant_act_lora_down(Xs[j], layers[j], xq, xs, la, stream)
+            ev[i][1].record(stream)
+            svdq.gemm_w4a4_lora_up(xq, xs, la, M, layers[j], Ys[j], stream)
+            ev[i][2].record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    k1_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    k2_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    err = svdq.last_device_error()
+
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    # ---------------- end to end through the host-buffer entry point
+    Xh = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).pin_memory()
+    Yh = torch.empty(M, N, dtype=torch.bfloat16).pin_memory()
+    e2e_steps = max(1, args.e2e_steps)
+    for i in range(2):
+        svdq.linear_forward_host(Xh, layers[0], Xs[0], bufs[0], Ys[0], Yh, stream)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(e2e_steps):
+        svdq.linear_forward_host(Xh, layers[i % NB], Xs[i % NB], bufs[i % NB], Ys[i % NB], Yh, stream)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    if dist:
+        t = torch.tensor([e2e_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    flops = layer_flops(M, K, N, r)
+    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
+    e2e_value = world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    hbm_gbs, bf16_tf, peak_kind = read_peaks()
+    fp4_peak = bf16_tf * FP4_OVER_BF16
+    k1_avg = statistics.mean(k1_ms)
+    k2_avg = statistics.mean(k2_ms)
+    k2_tf = k2_flops(M, K, N, r) / (k2_avg * 1e-3) / 1e12
+    k1_gbs = k1_bytes(M, K, r) / (k1_avg * 1e-3) / 1e9
+    traffic = None
+    tr_path = os.path.join(ROOT, "profiles", "k2_traffic.json")
+    if os.path.exists(tr_path):
+        with open(tr_path) as f:
+            tr = json.load(f)
+        if tr.get("workload") == shape.name and tr.get("kernel_rev") == svdq.load().svdq_version():
+            traffic = tr.get("bytes_per_launch")
+    cpu = None
+    if not args.no_cpu_baseline and world == 1:
+        res = cpu_oracle_sample(shape, 256, budget_s=15.0)
+        cpu = {"value": res["value"], "unit": "TFLOPS", "cores": res["cores"], "kind": "oracle",
+               "sample": f"{res['reps']} slices of 256 tokens ({res['tokens']} tokens) of the workload; fp64 numpy "
+                         f"oracle forward pass, prepare (SVD) excluded ({res['prepare_s']:.1f} s)"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "nvfp4", "data": "synthetic",
+        "config": {"workload": workload_name(shape), "M": M, "K": K, "N": N, "rank": r,
+                   "l2": f"{NB} rotating buffer sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2 in total)",
+                   "parallelism": f"replicas x{world}"},
+        "roofline": {"kernel": "svdq_gemm_w4a4_lora_up (K2)", "bound": "tensor", "achieved": k2_tf,
+                     "peak": fp4_peak, "unit": "TFLOP/s", "frac": k2_tf / fp4_peak, "traffic": traffic,
+                     "peak_source": f"{peak_kind} bf16 {bf16_tf:.0f} TF/s x {FP4_OVER_BF16:.0f} (nvfp4/bf16 nominal)",
+                     "achieved_basis": "2MNK + 2MNr per launch / mean CUDA-event duration"},
+        "quant_pass": {"kernel": "svdq_quant_act_lora_down (K1)", "bound": "hbm", "achieved": k1_gbs,
+                       "peak": hbm_gbs, "unit": "GB/s", "frac": k1_gbs / hbm_gbs, "us": k1_avg * 1e3,
+                       "frac_of_8TBs_datasheet": k1_gbs / 8000.0},
+        "k2": {"us": k2_avg * 1e3, "tflops": k2_tf},
+        "tokens_per_s": world * M * args.steps / (total_ms * 1e-3),
+        "cpu_baseline": cpu,
+        "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": int(M * K * 2),
+                "d2h_bytes_per_step": int(M * N * 2), "api": "svdq_linear_forward_host"},
+        "gpu_launches": 2 * args.steps,
+        "clocks": clk.summary(),
+        "device_error": err,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,409 @@
+// C ABI of libsvdq: argument checks, architecture check, TMA tensor-map encoding and kernel
+// launches. Every entry point is declared and documented in include/svdq.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include <mutex>
+
+#include "internal.h"
+#include "svdq.h"
+
+namespace svdq {
+
+__device__ uint32_t g_error_word;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+
+struct DeviceState {
+  std::once_flag once;
+  svdq_status arch = SVDQ_OK;
+  int num_sms = 0;
+  uint32_t *err = nullptr;
+};
+DeviceState g_dev[kMaxDevices];
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+std::once_flag g_encode_once;
+
+void init_encode() {
+  void *fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+      q == cudaDriverEntryPointSuccess)
+    g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+}
+
+// Checks the current device once: compute capability 10.0 ("دعم الأجهزة": unsupported GPUs
+// get a clear error instead of wrong output) and records the SM count and the error word.
+svdq_status device_check(DeviceState **out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SVDQ_ERR_INTERNAL;
+  DeviceState &d = g_dev[dev];
+  std::call_once(d.once, [&]() {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      d.arch = SVDQ_ERR_CUDA;
+      return;
+    }
+    if (major != 10 || minor != 0) {
+      d.arch = SVDQ_ERR_UNSUPPORTED_ARCH;
+      return;
+    }
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_error_word) != cudaSuccess) {
+      d.arch = SVDQ_ERR_CUDA;
+      return;
+    }
+    d.err = static_cast<uint32_t *>(p);
+  });
+  if (d.arch != SVDQ_OK) return d.arch;
+  *out = &d;
+  return SVDQ_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool rank_ok(int r) { return r == 0 || r == 16 || r == 32 || r == 64 || r == 128; }
+
+svdq_status check_layer(const svdq_layer *L) {
+  if (!L) return SVDQ_ERR_INVALID_ARG;
+  if (L->N <= 0 || L->K <= 0 || (L->K % 64) != 0 || (L->N % 16) != 0 || !rank_ok(L->rank))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!L->wq || !L->ws || !L->inv_lambda) return SVDQ_ERR_INVALID_ARG;
+  if (L->rank > 0 && (!L->L1t || !L->L2t)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(L->wq) || !aligned16(L->ws) || !aligned16(L->inv_lambda) || !aligned16(L->bias) ||
+      !aligned16(L->L1t) || !aligned16(L->L2t))
+    return SVDQ_ERR_MISALIGNED;
+  if (!(L->x_tensor_scale > 0.0f) || !(L->w_tensor_scale > 0.0f)) return SVDQ_ERR_INVALID_ARG;
+  return SVDQ_OK;
+}
+
+bool make_map(CUtensorMap *m, CUtensorMapDataType dt, const void *base, uint64_t inner, uint64_t outer,
+              uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swz) {
+  std::call_once(g_encode_once, init_encode);
+  if (!g_encode) return false;
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return g_encode(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, swz,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+CUtensorMapSwizzle swizzle_for_row_bytes(uint32_t b) {
+  return b >= 128 ? CU_TENSOR_MAP_SWIZZLE_128B : (b == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+}
+
+float alpha_of(const svdq_layer *L) { return L->x_tensor_scale * L->w_tensor_scale; }
+
+// Number of CTAs along K per 128-row tile for K1 (cluster size): enough CTAs to give every SM
+// two, at most 8 (the portable cluster limit), and every CTA at least one 64-column chunk.
+int pick_splits(int M, int K, int num_sms, int rank) {
+  const int tiles = (M + 127) / 128;
+  const int nch = K / 64;
+  int s = 1;
+  while (s < 8 && tiles * s < 2 * num_sms && nch >= 2 * s) s *= 2;
+  while (s > 1) {
+    const int cps = (nch + s - 1) / s;
+    if ((s - 1) * cps < nch) break;
+    s /= 2;
+  }
+  (void)rank;
+  return s;
+}
+
+svdq_status run_quant(const uint16_t *X, int M, const svdq_layer *L, uint8_t *xq, uint8_t *xs, uint16_t *la,
+                      bool quantize, bool lora, void *stream) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  st = check_layer(L);
+  if (st != SVDQ_OK) return st;
+  if (!X || M <= 0) return SVDQ_ERR_INVALID_ARG;
+  if (quantize && (!xq || !xs)) return SVDQ_ERR_INVALID_ARG;
+  if (lora && L->rank > 0 && !la) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(xq) || !aligned16(xs) || !aligned16(la)) return SVDQ_ERR_MISALIGNED;
+  if (!quantize && (!lora || L->rank == 0)) return SVDQ_OK;
+  QuantLaunch q;
+  memset(&q, 0, sizeof(q));
+  const int K = L->K, r = lora ? L->rank : 0;
+  if (!make_map(&q.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, static_cast<uint64_t>(K) * 2, 64, 128,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ERR_CUDA;
+  if (r > 0) {
+    if (!make_map(&q.tm_l1, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L1t, K, r, static_cast<uint64_t>(K) * 2, 64, r,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+      return SVDQ_ERR_CUDA;
+  } else {
+    q.tm_l1 = q.tm_x;
+  }
+  q.inv_lambda = L->inv_lambda;
+  q.xq = xq;
+  q.xs = xs;
+  q.lora_act = la;
+  q.M = M;
+  q.K = K;
+  q.rank = L->rank;
+  q.s_x = L->x_tensor_scale;
+  q.d_x = 6.0f * L->x_tensor_scale;
+  q.inv_alpha = 1.0f / alpha_of(L);
+  q.splits = r > 0 ? pick_splits(M, K, d->num_sms, r) : pick_splits(M, K, d->num_sms, 0);
+  q.chunks_per_split = (K / 64 + q.splits - 1) / q.splits;
+  q.quantize = quantize;
+  q.lora = lora;
+  q.err = d->err;
+  q.stream = static_cast<cudaStream_t>(stream);
+  return launch_quant_act(q) == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+svdq_status run_gemm(const uint8_t *xq, const uint8_t *xs, const uint16_t *la, int M, const svdq_layer *L,
+                     uint16_t *Y, bool fp4, bool add_y, bool lora, void *stream) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  st = check_layer(L);
+  if (st != SVDQ_OK) return st;
+  if (M <= 0 || !Y) return SVDQ_ERR_INVALID_ARG;
+  if (fp4 && (!xq || !xs)) return SVDQ_ERR_INVALID_ARG;
+  const int r = lora ? L->rank : 0;
+  if (r > 0 && !la) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(xq) || !aligned16(xs) || !aligned16(la) || !aligned16(Y)) return SVDQ_ERR_MISALIGNED;
+  if (!fp4 && r == 0) return SVDQ_OK;
+  GemmLaunch g;
+  memset(&g, 0, sizeof(g));
+  const int K = L->K, N = L->N;
+  if (fp4) {
+    if (!make_map(&g.tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K / 2, M, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&g.tm_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wq, K / 2, N, K / 2, 128, 256, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SVDQ_ERR_CUDA;
+  }
+  if (r > 0) {
+    const uint32_t kc = r < 64 ? r : 64;
+    const CUtensorMapSwizzle sw = swizzle_for_row_bytes(kc * 2);
+    if (!make_map(&g.tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, la, r, M, static_cast<uint64_t>(r) * 2, kc, 128, sw) ||
+        !make_map(&g.tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L2t, r, N, static_cast<uint64_t>(r) * 2, kc, 256, sw))
+      return SVDQ_ERR_CUDA;
+  }
+  if (!fp4) {
+    g.tm_xq = g.tm_la;
+    g.tm_wq = g.tm_l2;
+  }
+  if (r == 0) {
+    g.tm_la = g.tm_xq;
+    g.tm_l2 = g.tm_wq;
+  }
+  g.xs = xs;
+  g.ws = L->ws;
+  g.bias = L->bias;
+  g.Y = Y;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.rank = r;
+  g.alpha = alpha_of(L);
+  g.fp4 = fp4;
+  g.add_y = add_y;
+  g.num_sms = d->num_sms;
+  g.err = d->err;
+  g.stream = static_cast<cudaStream_t>(stream);
+  return launch_gemm(g) == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
+}  // namespace
+}  // namespace svdq
+
+using namespace svdq;
+
+extern "C" {
+
+const char *svdq_status_string(svdq_status s) {
+  switch (s) {
+    case SVDQ_OK: return "ok";
+    case SVDQ_ERR_INVALID_ARG: return "invalid argument";
+    case SVDQ_ERR_UNSUPPORTED_ARCH: return "unsupported GPU: libsvdq needs compute capability 10.0 (B200, sm_100a)";
+    case SVDQ_ERR_MISALIGNED: return "device pointer not 16-byte aligned";
+    case SVDQ_ERR_CUDA: return "CUDA error";
+    case SVDQ_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case SVDQ_ERR_INTERNAL: return "internal error";
+    case SVDQ_ERR_UNAVAILABLE: return "eigen-solver library (libcusolver.so.11) not found";
+  }
+  return "unknown status";
+}
+
+int svdq_version(void) { return 100; }
+
+size_t svdq_weight_scale_bytes(int N, int K) {
+  if (N <= 0 || K <= 0) return 0;
+  return round_up(static_cast<size_t>(N), 256) * static_cast<size_t>(K / 16);
+}
+
+size_t svdq_act_scale_bytes(int M, int K) {
+  if (M <= 0 || K <= 0) return 0;
+  return round_up(static_cast<size_t>(M), 128) * static_cast<size_t>(K / 16);
+}
+
+svdq_status svdq_act_absmax(const uint16_t *X, int M, int K, float *absmax, void *stream) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  if (!X || !absmax || M <= 0 || K <= 0) return SVDQ_ERR_INVALID_ARG;
+  return launch_col_absmax_bf16(X, M, K, absmax, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SVDQ_OK
+                                                                                                   : SVDQ_ERR_CUDA;
+}
+
+size_t svdq_prepare_workspace_bytes(int N, int K, int rank, svdq_status *status) {
+  PrepPlan plan;
+  svdq_status st = SVDQ_OK;
+  if (N <= 0 || K <= 0 || K % 64 || N % 16 || !rank_ok(rank)) st = SVDQ_ERR_INVALID_ARG;
+  if (st == SVDQ_OK) {
+    const PrepStatus ps = prepare_plan(N, K, rank, &plan);
+    if (ps == PREP_NO_SOLVER) st = SVDQ_ERR_UNAVAILABLE;
+    else if (ps != PREP_OK) st = SVDQ_ERR_CUDA;
+  }
+  if (status) *status = st;
+  return st == SVDQ_OK ? plan.bytes : 0;
+}
+
+svdq_status svdq_prepare_weights(const float *W, const float *bias, const float *act_absmax, int N, int K, int rank,
+                                 svdq_layer *layer, void *workspace, size_t workspace_bytes, void *stream) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  if (!W || !act_absmax || !layer || !workspace) return SVDQ_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || K % 64 || N % 16 || !rank_ok(rank)) return SVDQ_ERR_INVALID_ARG;
+  if (layer->N != N || layer->K != K || layer->rank != rank) return SVDQ_ERR_INVALID_ARG;
+  if (!layer->wq || !layer->ws || !layer->inv_lambda || (rank > 0 && (!layer->L1t || !layer->L2t)))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(act_absmax) || !aligned16(workspace) || !aligned16(layer->wq) ||
+      !aligned16(layer->ws) || !aligned16(layer->inv_lambda) || !aligned16(layer->lambda) ||
+      !aligned16(layer->L1t) || !aligned16(layer->L2t) || !aligned16(layer->bias) || !aligned16(bias))
+    return SVDQ_ERR_MISALIGNED;
+  PrepArgs p;
+  const PrepStatus ps = prepare_plan(N, K, rank, &p.plan);
+  if (ps == PREP_NO_SOLVER) return SVDQ_ERR_UNAVAILABLE;
+  if (ps != PREP_OK) return SVDQ_ERR_CUDA;
+  if (workspace_bytes < p.plan.bytes) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  p.W = W;
+  p.act_absmax = act_absmax;
+  p.N = N;
+  p.K = K;
+  p.rank = rank;
+  p.workspace = workspace;
+  p.lambda_out = layer->lambda;
+  p.inv_lambda = layer->inv_lambda;
+  p.L1t = layer->L1t;
+  p.L2t = layer->L2t;
+  p.wq = layer->wq;
+  p.wscales = layer->ws;
+  p.wscale_bytes = svdq_weight_scale_bytes(N, K);
+  float s_w = 0.0f, s_x = 0.0f;
+  p.s_w = &s_w;
+  p.s_x = &s_x;
+  p.stream = s;
+  const PrepStatus rs = prepare_run(p);
+  if (rs == PREP_SOLVER_FAILED) return SVDQ_ERR_INTERNAL;
+  if (rs != PREP_OK) return SVDQ_ERR_CUDA;
+  if (bias && layer->bias && bias != layer->bias) {
+    if (cudaMemcpyAsync(layer->bias, bias, sizeof(float) * N, cudaMemcpyDeviceToDevice, s) != cudaSuccess ||
+        cudaStreamSynchronize(s) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+  }
+  layer->group = 16;
+  layer->w_tensor_scale = s_w;
+  layer->x_tensor_scale = s_x;
+  return SVDQ_OK;
+}
+
+svdq_status svdq_quantize_rows(const float *A, int rows, int K, float s, int row_pad, uint8_t *codes, uint8_t *scales,
+                               void *stream) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  if (!A || !codes || !scales || rows <= 0 || K <= 0 || K % 64 || !(s > 0.0f) || (row_pad != 128 && row_pad != 256))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(codes) || !aligned16(scales)) return SVDQ_ERR_MISALIGNED;
+  cudaStream_t cs = static_cast<cudaStream_t>(stream);
+  const size_t sbytes = round_up(static_cast<size_t>(rows), row_pad) * (K / 16);
+  if (cudaMemsetAsync(scales, 0, sbytes, cs) != cudaSuccess) return SVDQ_ERR_CUDA;
+  return launch_quantize_rows(A, rows, K, s, codes, scales, cs) == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+svdq_status svdq_quant_act_lora_down(const uint16_t *X, int M, const svdq_layer *layer, uint8_t *xq, uint8_t *xs,
+                                     uint16_t *lora_act, void *stream) {
+  return run_quant(X, M, layer, xq, xs, lora_act, true, true, stream);
+}
+
+svdq_status svdq_gemm_w4a4_lora_up(const uint8_t *xq, const uint8_t *xs, const uint16_t *lora_act, int M,
+                                   const svdq_layer *layer, uint16_t *Y, void *stream) {
+  return run_gemm(xq, xs, lora_act, M, layer, Y, true, false, true, stream);
+}
+
+svdq_status svdq_linear_forward(const uint16_t *X, int M, const svdq_layer *layer, uint8_t *xq, uint8_t *xs,
+                                uint16_t *lora_act, uint16_t *Y, void *stream) {
+  svdq_status st = svdq_quant_act_lora_down(X, M, layer, xq, xs, lora_act, stream);
+  if (st != SVDQ_OK) return st;
+  return svdq_gemm_w4a4_lora_up(xq, xs, lora_act, M, layer, Y, stream);
+}
+
+svdq_status svdq_linear_forward_host(const uint16_t *X_host, int M, const svdq_layer *layer, uint16_t *X_dev,
+                                     uint8_t *xq, uint8_t *xs, uint16_t *lora_act, uint16_t *Y_dev, uint16_t *Y_host,
+                                     void *stream) {
+  if (!X_host || !Y_host || !X_dev || !Y_dev || !layer || M <= 0) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t xb = static_cast<size_t>(M) * layer->K * 2, yb = static_cast<size_t>(M) * layer->N * 2;
+  if (cudaMemcpyAsync(X_dev, X_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess) return SVDQ_ERR_CUDA;
+  svdq_status st = svdq_linear_forward(X_dev, M, layer, xq, xs, lora_act, Y_dev, stream);
+  if (st != SVDQ_OK) return st;
+  if (cudaMemcpyAsync(Y_host, Y_dev, yb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return SVDQ_ERR_CUDA;
+  return cudaStreamSynchronize(s) == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+}
+
+svdq_status svdq_baseline_lora_down(const uint16_t *X, int M, const svdq_layer *layer, uint16_t *lora_act,
+                                    void *stream) {
+  return run_quant(X, M, layer, nullptr, nullptr, lora_act, false, true, stream);
+}
+
+svdq_status svdq_baseline_quantize(const uint16_t *X, int M, const svdq_layer *layer, uint8_t *xq, uint8_t *xs,
+                                   void *stream) {
+  return run_quant(X, M, layer, xq, xs, nullptr, true, false, stream);
+}
+
+svdq_status svdq_baseline_gemm_w4a4(const uint8_t *xq, const uint8_t *xs, int M, const svdq_layer *layer, uint16_t *Y,
+                                    void *stream) {
+  return run_gemm(xq, xs, nullptr, M, layer, Y, true, false, false, stream);
+}
+
+svdq_status svdq_baseline_lora_up(const uint16_t *lora_act, int M, const svdq_layer *layer, uint16_t *Y,
+                                  void *stream) {
+  if (layer && layer->rank == 0) return SVDQ_OK;
+  return run_gemm(nullptr, nullptr, lora_act, M, layer, Y, false, true, true, stream);
+}
+
+svdq_status svdq_last_device_error(void *stream, uint32_t *code) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  if (!code) return SVDQ_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SVDQ_ERR_CUDA;
+  uint32_t v = 0;
+  if (cudaMemcpy(&v, d->err, sizeof(v), cudaMemcpyDeviceToHost) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (v && cudaMemset(d->err, 0, sizeof(v)) != cudaSuccess) return SVDQ_ERR_CUDA;
+  *code = v;
+  return v ? SVDQ_ERR_TIMEOUT : SVDQ_OK;
+}
+
+}  // extern "C"

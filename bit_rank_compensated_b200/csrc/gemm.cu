@@ -1,0 +1,303 @@
+// K2: block-scaled NVFP4 tensor-core GEMM whose output stage adds the low-rank up-projection
+// and the bias and writes bf16 once.
+//
+// "Svdq Int4 Flux.1 Canny Dev" model card, "Nunchaku 引擎設計" (a)/(b): the up-projection and
+// the 4-bit GEMM produce the same output, so one kernel serves both and the 16-bit output is
+// written once.
+//
+// Persistent kernel, one CTA per SM, output tiles of 128 x 256 (rows of X x rows of W).
+// Per tile the k-loop is a sequence of pipeline steps through a 4-stage shared-memory ring:
+//   - rank / 64 (at least one) low-rank steps: lora_act tile (128 x kc bf16) and L2t tile
+//     (256 x kc bf16), kc = min(rank, 64); bf16 tcgen05 MMAs (K = 16 each);
+//   - K / 256 4-bit steps: xq tile (128 rows x 128 bytes), wq tile (256 x 128 bytes), both with
+//     128B swizzle, plus their e4m3 scale blocks (512 bytes per 128 rows x 64 elements), copied
+//     into tensor memory with tcgen05.cp; four kind::mxf4nvf4 MMAs (K = 64 each).
+// All steps accumulate into one fp32 accumulator in tensor memory (128 lanes x 256 columns).
+// lora_act arrives pre-divided by alpha = s_x s_w, so the output stage computes
+// Y = bf16(alpha * acc + bias) for every element.
+//
+// Warp roles (192 threads): warp 0 TMA producer; warp 1 tensor-memory owner and MMA issuer;
+// warps 2..5 output stage (warp w reads lanes 32 (w % 4) .. + 31).
+#include "common.cuh"
+#include "internal.h"
+
+namespace svdq {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BN = 256;
+constexpr int STAGES = 4;
+constexpr uint32_t A_BYTES = 128u * 128u;
+constexpr uint32_t B_BYTES = 256u * 128u;
+constexpr uint32_t SFA_BYTES = 2048u;
+constexpr uint32_t SFB_BYTES = 4096u;
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 55296 = 54 KiB
+constexpr uint32_t DATA_BYTES = STAGES * STAGE_BYTES;
+constexpr uint32_t SMEM = DATA_BYTES + 256 + 1024;
+constexpr uint32_t TMEM_COLS = 512;
+constexpr uint32_t SF_COL0 = 256;   // scale columns follow the accumulator
+constexpr uint32_t SF_COLS = 48;    // per stage: 4 k-blocks x (4 SFA + 8 SFB) columns
+constexpr int THREADS = 192;
+
+struct GArgs {
+  const uint8_t *xs;
+  const uint8_t *ws;
+  const float *bias;
+  uint16_t *Y;
+  int M, N, K;
+  int Mt, Nt;
+  float alpha;
+  uint32_t *err;
+};
+
+template <int RANK, bool FP4, bool ADD_Y>
+__global__ void __launch_bounds__(THREADS, 1)
+    k2_gemm_w4a4_lora_up(const __grid_constant__ CUtensorMap tm_xq, const __grid_constant__ CUtensorMap tm_wq,
+                         const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_l2,
+                         GArgs a) {
+  constexpr int KC = RANK == 0 ? 64 : (RANK < 64 ? RANK : 64);
+  constexpr int N_LORA = RANK == 0 ? 0 : RANK / KC;
+  constexpr uint32_t LORA_ROW = KC * 2;  // bytes per row of a low-rank tile
+  constexpr uint32_t LORA_SWZ = LORA_ROW == 128 ? 2u : (LORA_ROW == 64 ? 4u : 6u);
+  constexpr uint32_t LORA_A_BYTES = 128u * LORA_ROW;
+  constexpr uint32_t LORA_B_BYTES = 256u * LORA_ROW;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DATA_BYTES);
+  const uint32_t bar_full = smem_u32(bars);
+  const uint32_t bar_empty = bar_full + 8 * STAGES;
+  const uint32_t bar_accfull = bar_empty + 8 * STAGES;
+  const uint32_t bar_accempty = bar_accfull + 8;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 2);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int kblocks = a.K / 64;
+  const int n_kt = FP4 ? (kblocks + 3) / 4 : 0;
+  const int total = N_LORA + n_kt;
+  const int tiles = a.Mt * a.Nt;
+
+  auto a_tile = [&](int s) { return smem + s * STAGE_BYTES; };
+  auto b_tile = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
+  auto sfa_tile = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B_BYTES; };
+  auto sfb_tile = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B_BYTES + SFA_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 1);
+    }
+    mbar_init(bar_accfull, 1);
+    mbar_init(bar_accempty, 128);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      if (FP4) {
+        tma_prefetch_desc(&tm_xq);
+        tma_prefetch_desc(&tm_wq);
+      }
+      if (RANK) {
+        tma_prefetch_desc(&tm_la);
+        tma_prefetch_desc(&tm_l2);
+      }
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+        const int mt = tile % a.Mt;
+        const int nt = tile / a.Mt;
+        for (int j = 0; j < total; ++j, ++it) {
+          const int s = it % STAGES;
+          if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1, a.err, KID_GEMM, 1)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = bar_full + 8 * s;
+          if (j < N_LORA) {
+            mbar_arrive_expect_tx(fb, LORA_A_BYTES + LORA_B_BYTES);
+            tma_load_2d(smem_u32(a_tile(s)), &tm_la, j * KC, mt * BM, fb);
+            tma_load_2d(smem_u32(b_tile(s)), &tm_l2, j * KC, nt * BN, fb);
+          } else {
+            const int kt = j - N_LORA;
+            const int kbv = min(4, kblocks - 4 * kt);
+            mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES + 3u * 512u * kbv);
+            tma_load_2d(smem_u32(a_tile(s)), &tm_xq, kt * 128, mt * BM, fb);
+            tma_load_2d(smem_u32(b_tile(s)), &tm_wq, kt * 128, nt * BN, fb);
+            bulk_load(smem_u32(sfa_tile(s)), a.xs + (static_cast<size_t>(mt) * kblocks + 4 * kt) * 512, 512u * kbv, fb);
+            bulk_load(smem_u32(sfb_tile(s)), a.ws + (static_cast<size_t>(2 * nt) * kblocks + 4 * kt) * 512,
+                      512u * kbv, fb);
+            bulk_load(smem_u32(sfb_tile(s)) + 2048, a.ws + (static_cast<size_t>(2 * nt + 1) * kblocks + 4 * kt) * 512,
+                      512u * kbv, fb);
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      // kind::mxf4nvf4: A, B e2m1 (bits 7-9, 10-12 = 1), K-major, N = 256 (bits 17-22),
+      // scale type ue4m3 (bit 23 = 0), M = 128 (bits 24-28), scale ids 0, K = 64.
+      const uint32_t idesc_fp4 = (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BM) >> 4) << 24);
+      // kind::f16: D fp32, A, B bf16, N = 256, M = 128.
+      const uint32_t idesc_bf16 =
+          (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BM) >> 4) << 24);
+      uint32_t it = 0;
+      uint32_t tcount = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tcount) {
+        if (tcount > 0 && !mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 2)) break;
+        tc_fence_after();
+        for (int j = 0; j < total; ++j, ++it) {
+          const int s = it % STAGES;
+          if (!mbar_wait(bar_full + 8 * s, (it / STAGES) & 1, a.err, KID_GEMM, 3)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (j < N_LORA) {
+            const uint64_t ad = umma_desc(smem_u32(a_tile(s)), 16, 8 * LORA_ROW, LORA_SWZ);
+            const uint64_t bd = umma_desc(smem_u32(b_tile(s)), 16, 8 * LORA_ROW, LORA_SWZ);
+#pragma unroll
+            for (int k = 0; k < KC / 16; ++k)
+              mma_bf16(tbase, ad + 2u * k, bd + 2u * k, idesc_bf16, (j | k) != 0 ? 1u : 0u);
+          } else {
+            const int kt = j - N_LORA;
+            const int kbv = min(4, kblocks - 4 * kt);
+            const uint32_t tsf = tbase + SF_COL0 + SF_COLS * s;
+            const uint32_t sfa = smem_u32(sfa_tile(s));
+            const uint32_t sfb = smem_u32(sfb_tile(s));
+            for (int kb = 0; kb < kbv; ++kb) {
+              tmem_cp_32x128b_x4(tsf + 4 * kb, umma_desc(sfa + 512 * kb, 0, 128, 0));
+              tmem_cp_32x128b_x4(tsf + 16 + 8 * kb, umma_desc(sfb + 512 * kb, 0, 128, 0));
+              tmem_cp_32x128b_x4(tsf + 16 + 8 * kb + 4, umma_desc(sfb + 2048 + 512 * kb, 0, 128, 0));
+            }
+            const uint64_t ad = umma_desc(smem_u32(a_tile(s)), 16, 1024, 2);
+            const uint64_t bd = umma_desc(smem_u32(b_tile(s)), 16, 1024, 2);
+            for (int kb = 0; kb < kbv; ++kb)
+              mma_nvfp4(tbase, ad + 2u * kb, bd + 2u * kb, idesc_fp4, tsf + 4 * kb, tsf + 16 + 8 * kb,
+                        (j | kb) != 0 ? 1u : 0u);
+          }
+          tc_commit(bar_empty + 8 * s);
+        }
+        if (!ok) break;
+        tc_commit(bar_accfull);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ output stage
+    const int quad = warp & 3;
+    const int row = quad * 32 + lane;
+    uint32_t tcount = 0;
+    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tcount) {
+      const int mt = tile % a.Mt;
+      const int nt = tile / a.Mt;
+      if (!mbar_wait(bar_accfull, tcount & 1, a.err, KID_GEMM, 4)) break;
+      tc_fence_after();
+      const int m = mt * BM + row;
+      for (int c = 0; c < BN / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tbase + (static_cast<uint32_t>(quad * 32) << 16) + c * 32, r);
+        tmem_wait_ld();
+        if (c == BN / 32 - 1) {
+          tc_fence_before();
+          mbar_arrive(bar_accempty);
+        }
+        const int n = nt * BN + c * 32;
+        if (n >= a.N || m >= a.M) continue;
+        uint16_t *yrow = a.Y + static_cast<size_t>(m) * a.N + n;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          if (n + 8 * q >= a.N) break;
+          float v[8];
+          if (ADD_Y) {
+            const uint4 old = *reinterpret_cast<const uint4 *>(yrow + 8 * q);
+            const uint32_t w[4] = {old.x, old.y, old.z, old.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              v[2 * e] = fmaf(a.alpha, __uint_as_float(r[8 * q + 2 * e]), bf16_lo(w[e]));
+              v[2 * e + 1] = fmaf(a.alpha, __uint_as_float(r[8 * q + 2 * e + 1]), bf16_hi(w[e]));
+            }
+          } else {
+            float bsv[8];
+            if (a.bias) {
+              const float4 b0 = __ldg(reinterpret_cast<const float4 *>(a.bias + n + 8 * q));
+              const float4 b1 = __ldg(reinterpret_cast<const float4 *>(a.bias + n + 8 * q + 4));
+              bsv[0] = b0.x; bsv[1] = b0.y; bsv[2] = b0.z; bsv[3] = b0.w;
+              bsv[4] = b1.x; bsv[5] = b1.y; bsv[6] = b1.z; bsv[7] = b1.w;
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) bsv[e] = 0.0f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = fmaf(a.alpha, __uint_as_float(r[8 * q + e]), bsv[e]);
+          }
+          uint4 o;
+          o.x = pack_bf16x2(v[0], v[1]);
+          o.y = pack_bf16x2(v[2], v[3]);
+          o.z = pack_bf16x2(v[4], v[5]);
+          o.w = pack_bf16x2(v[6], v[7]);
+          *reinterpret_cast<uint4 *>(yrow + 8 * q) = o;
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, TMEM_COLS);
+  }
+}
+
+template <int RANK, bool FP4, bool ADD_Y>
+cudaError_t launch_t(const GemmLaunch &g) {
+  auto kern = k2_gemm_w4a4_lora_up<RANK, FP4, ADD_Y>;
+  static int attr_done[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = 1;
+  }
+  GArgs a{g.xs, g.ws, g.bias, g.Y, g.M, g.N, g.K, (g.M + BM - 1) / BM, (g.N + BN - 1) / BN, g.alpha, g.err};
+  const int tiles = a.Mt * a.Nt;
+  const int grid = tiles < g.num_sms ? tiles : g.num_sms;
+  kern<<<grid, THREADS, SMEM, g.stream>>>(g.tm_xq, g.tm_wq, g.tm_la, g.tm_l2, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmLaunch &g) {
+  if (g.fp4 && !g.add_y) {
+    switch (g.rank) {
+      case 0: return launch_t<0, true, false>(g);
+      case 16: return launch_t<16, true, false>(g);
+      case 32: return launch_t<32, true, false>(g);
+      case 64: return launch_t<64, true, false>(g);
+      case 128: return launch_t<128, true, false>(g);
+    }
+  } else if (!g.fp4 && g.add_y) {
+    switch (g.rank) {
+      case 16: return launch_t<16, false, true>(g);
+      case 32: return launch_t<32, false, true>(g);
+      case 64: return launch_t<64, false, true>(g);
+      case 128: return launch_t<128, false, true>(g);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace svdq

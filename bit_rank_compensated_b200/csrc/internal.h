@@ -1,0 +1,85 @@
+// Internal launch interfaces between the C ABI layer (api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace svdq {
+
+// K1 (and the unfused down-projection / quantize baselines).
+struct QuantLaunch {
+  CUtensorMap tm_x;   // X, bf16 [M, K], box 64 x 128, 128B swizzle
+  CUtensorMap tm_l1;  // L1t, bf16 [rank, K], box 64 x rank, 128B swizzle (unused at rank 0)
+  const float *inv_lambda;
+  uint8_t *xq;
+  uint8_t *xs;
+  uint16_t *lora_act;
+  int M, K, rank;
+  float s_x, d_x, inv_alpha;
+  int splits;            // CTAs along K per 128-row tile (cluster size)
+  int chunks_per_split;  // 64-column chunks per CTA
+  bool quantize;         // write xq / xs
+  bool lora;             // compute the down-projection
+  uint32_t *err;
+  cudaStream_t stream;
+};
+cudaError_t launch_quant_act(const QuantLaunch &q);
+
+// K2 (and the unfused 4-bit GEMM / up-projection baselines).
+struct GemmLaunch {
+  CUtensorMap tm_xq;  // xq, u8 [M, K/2], box 128 x 128, 128B swizzle
+  CUtensorMap tm_wq;  // wq, u8 [N, K/2], box 128 x 256, 128B swizzle
+  CUtensorMap tm_la;  // lora_act, bf16 [M, rank], box kc x 128
+  CUtensorMap tm_l2;  // L2t, bf16 [N, rank], box kc x 256
+  const uint8_t *xs;
+  const uint8_t *ws;
+  const float *bias;
+  uint16_t *Y;
+  int M, N, K, rank;
+  float alpha;
+  bool fp4;    // run the block-scaled 4-bit product
+  bool add_y;  // Y = bf16(Y + alpha * acc) instead of bf16(alpha * acc + bias)
+  int num_sms;
+  uint32_t *err;
+  cudaStream_t stream;
+};
+cudaError_t launch_gemm(const GemmLaunch &g);
+
+// Offline preparation pieces (prepare.cu).
+cudaError_t launch_col_absmax_f32(const float *A, int rows, int cols, float *out, cudaStream_t st);
+cudaError_t launch_col_absmax_bf16(const uint16_t *A, int rows, int cols, float *out, cudaStream_t st);
+cudaError_t launch_quantize_rows(const float *A, int rows, int K, float s, uint8_t *codes, uint8_t *scales,
+                                 cudaStream_t st);
+
+}  // namespace svdq
+
+namespace svdq {
+
+enum PrepStatus { PREP_OK = 0, PREP_CUDA, PREP_NO_SOLVER, PREP_SOLVER_FAILED, PREP_INTERNAL };
+
+struct PrepPlan {
+  int n_g = 0, side = 0, lwork = 0;
+  size_t off_G = 0, off_evals = 0, off_V = 0, off_P = 0, off_Q = 0, off_sig = 0, off_R = 0, off_aw = 0, off_lam = 0,
+         off_scal = 0, off_info = 0, off_work = 0, bytes = 0;
+};
+
+struct PrepArgs {
+  const float *W;
+  const float *act_absmax;
+  int N, K, rank;
+  PrepPlan plan;
+  void *workspace;
+  float *lambda_out;  // may be null
+  float *inv_lambda;
+  uint16_t *L1t, *L2t;
+  uint8_t *wq, *wscales;
+  size_t wscale_bytes;
+  float *s_w, *s_x;  // host outputs
+  cudaStream_t stream;
+};
+
+PrepStatus prepare_plan(int N, int K, int rank, PrepPlan *plan);
+PrepStatus prepare_run(const PrepArgs &p);
+
+}  // namespace svdq

@@ -1,0 +1,309 @@
+// K1: smoothing + NVFP4 activation quantization + low-rank down-projection in one read of X.
+//
+// "Svdq Int4 Flux.1 Canny Dev" model card, "Nunchaku 引擎設計" (b): the down-projection and
+// the quantizer consume the same input, so one kernel serves both.
+//
+// Work decomposition: a CTA owns 128 rows and a contiguous range of 64-column chunks of K.
+// The CTAs that share a row tile form a thread-block cluster along K; their fp32 partial
+// down-projections are summed through distributed shared memory in cluster-rank order, so
+// the result is deterministic and nothing goes through global scratch memory.
+//
+// Warp roles (320 threads):
+//   warp 0      TMA producer: X chunk (128 x 64 bf16, 128B swizzle) and L1t chunk (rank x 64).
+//   warp 1      owns the tensor-memory accumulator (128 lanes x rank fp32 columns) and issues
+//               the bf16 tcgen05 MMAs  acc += bf16(X_hat chunk) * L1 chunk.
+//   warps 2..9  quantizers: thread (row, half) handles 32 elements (two 16-groups) of a chunk:
+//               X_hat = fp32(X * inv_lambda), the group scales and codes, and writes bf16(X_hat)
+//               into the MMA operand tile (same swizzle as the X tile).
+#include "common.cuh"
+#include "internal.h"
+#include "nvfp4.cuh"
+
+namespace svdq {
+namespace {
+
+template <int RANK>
+struct QCfg {
+  static constexpr int STAGES = RANK == 0 ? 4 : 3;
+  static constexpr uint32_t X_BYTES = 128u * 128u;
+  static constexpr uint32_t OP_BYTES = RANK ? 128u * 128u : 0u;
+  static constexpr uint32_t L1_BYTES = RANK * 128u;
+  static constexpr uint32_t STAGE_BYTES = X_BYTES + OP_BYTES + L1_BYTES;
+  static constexpr uint32_t RED_BYTES = RANK * 128u * 4u;
+  static constexpr uint32_t DATA_BYTES =
+      (STAGES * STAGE_BYTES > RED_BYTES) ? STAGES * STAGE_BYTES : RED_BYTES;
+  static constexpr uint32_t BAR_BYTES = 256;
+  static constexpr uint32_t SMEM = DATA_BYTES + BAR_BYTES + 1024;  // + alignment slack
+  static constexpr uint32_t TMEM_COLS = RANK <= 32 ? 32u : static_cast<uint32_t>(RANK);
+  static constexpr int THREADS = 320;
+};
+
+struct QArgs {
+  const float *inv_lambda;
+  uint8_t *xq;
+  uint8_t *xs;
+  uint16_t *lora_act;
+  int M, K;
+  float s_x, d_x, inv_alpha;
+  int chunks_per_split;
+  uint32_t *err;
+};
+
+template <int RANK, bool QUANT>
+__global__ void __launch_bounds__(320, 1)
+    k1_quant_act_lora_down(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
+                           QArgs a) {
+  using C = QCfg<RANK>;
+  constexpr int ST = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::DATA_BYTES);
+  // bars: full[ST] | empty[ST] | opfull[ST] | accfull | tmem holder
+  const uint32_t bar_full = smem_u32(bars);
+  const uint32_t bar_empty = bar_full + 8 * ST;
+  const uint32_t bar_opfull = bar_empty + 8 * ST;
+  const uint32_t bar_acc = bar_opfull + 8 * ST;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 3 * ST + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int split = blockIdx.x;
+  const int nsplit = gridDim.x;
+  const int m0 = blockIdx.y * 128;
+  const int nch = a.K / 64;
+  const int c_begin = split * a.chunks_per_split;
+  int n_local = nch - c_begin;
+  if (n_local > a.chunks_per_split) n_local = a.chunks_per_split;
+  if (n_local < 0) n_local = 0;
+
+  auto x_tile = [&](int s) { return smem + s * C::STAGE_BYTES; };
+  auto op_tile = [&](int s) { return smem + s * C::STAGE_BYTES + C::X_BYTES; };
+  auto l1_tile = [&](int s) { return smem + s * C::STAGE_BYTES + C::X_BYTES + C::OP_BYTES; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_empty + 8 * s, 8 + (RANK ? 1 : 0));
+      mbar_init(bar_opfull + 8 * s, 8);
+    }
+    mbar_init(bar_acc, 1);
+    fence_mbar_init();
+  }
+  if (RANK && warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = RANK ? *tmem_holder : 0u;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_x);
+      if (RANK) tma_prefetch_desc(&tm_l1);
+      for (int i = 0; i < n_local; ++i) {
+        const int s = i % ST;
+        if (i >= ST && !mbar_wait(bar_empty + 8 * s, ((i / ST) - 1) & 1, a.err, KID_QUANT, 1)) break;
+        mbar_arrive_expect_tx(bar_full + 8 * s, C::X_BYTES + C::L1_BYTES);
+        const int kx = (c_begin + i) * 64;
+        tma_load_2d(smem_u32(x_tile(s)), &tm_x, kx, m0, bar_full + 8 * s);
+        if (RANK) tma_load_2d(smem_u32(l1_tile(s)), &tm_l1, kx, 0, bar_full + 8 * s);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (RANK && lane == 0) {
+      // kind::f16: D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9, 10-12 = 1), K-major,
+      // N = RANK (bits 17-22 = N >> 3), M = 128 (bits 24-28 = M >> 4).
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(RANK) >> 3) << 17) | ((128u >> 4) << 24);
+      for (int i = 0; i < n_local; ++i) {
+        const int s = i % ST;
+        const uint32_t par = (i / ST) & 1;
+        if (!mbar_wait(bar_opfull + 8 * s, par, a.err, KID_QUANT, 2)) break;
+        if (!mbar_wait(bar_full + 8 * s, par, a.err, KID_QUANT, 3)) break;
+        tc_fence_after();
+        const uint64_t ad = umma_desc(smem_u32(op_tile(s)), 16, 1024, 2);
+        const uint64_t bd = umma_desc(smem_u32(l1_tile(s)), 16, 1024, 2);
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_bf16(tbase, ad + 2u * k, bd + 2u * k, idesc, (i | k) != 0 ? 1u : 0u);
+        tc_commit(bar_empty + 8 * s);
+      }
+      tc_commit(bar_acc);
+    }
+  } else {
+    // ------------------------------------------------------------ quantizers
+    const int t = threadIdx.x - 64;
+    const int row = t & 127;
+    const int half = t >> 7;
+    const int m = m0 + row;
+    const int ng = a.K / 16;
+    for (int i = 0; i < n_local; ++i) {
+      const int s = i % ST;
+      if (!mbar_wait(bar_full + 8 * s, (i / ST) & 1, a.err, KID_QUANT, 4)) break;
+      const uint8_t *xt = x_tile(s) + row * 128;
+      uint4 raw[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c = half * 4 + q;
+        raw[q] = *reinterpret_cast<const uint4 *>(xt + ((c ^ (row & 7)) << 4));
+      }
+      const int kbase = (c_begin + i) * 64 + half * 32;
+      float xh[32];
+      const float4 *il4 = reinterpret_cast<const float4 *>(a.inv_lambda + kbase);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 l0 = __ldg(il4 + 2 * q);
+        const float4 l1 = __ldg(il4 + 2 * q + 1);
+        const uint32_t w[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
+        xh[8 * q + 0] = __fmul_rn(bf16_lo(w[0]), l0.x);
+        xh[8 * q + 1] = __fmul_rn(bf16_hi(w[0]), l0.y);
+        xh[8 * q + 2] = __fmul_rn(bf16_lo(w[1]), l0.z);
+        xh[8 * q + 3] = __fmul_rn(bf16_hi(w[1]), l0.w);
+        xh[8 * q + 4] = __fmul_rn(bf16_lo(w[2]), l1.x);
+        xh[8 * q + 5] = __fmul_rn(bf16_hi(w[2]), l1.y);
+        xh[8 * q + 6] = __fmul_rn(bf16_lo(w[3]), l1.z);
+        xh[8 * q + 7] = __fmul_rn(bf16_hi(w[3]), l1.w);
+      }
+      if (QUANT) {
+        uint4 codes;
+        const uint32_t sc0 = nvfp4_group16(xh, a.s_x, a.d_x, codes.x, codes.y);
+        const uint32_t sc1 = nvfp4_group16(xh + 16, a.s_x, a.d_x, codes.z, codes.w);
+        if (m < a.M) *reinterpret_cast<uint4 *>(a.xq + static_cast<size_t>(m) * (a.K / 2) + kbase / 2) = codes;
+        *reinterpret_cast<uint16_t *>(a.xs + scale_offset(m, kbase / 16, ng)) =
+            static_cast<uint16_t>(sc0 | (sc1 << 8));
+      }
+      if (RANK) {
+        uint8_t *ot = op_tile(s) + row * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint4 v;
+          v.x = pack_bf16x2(xh[8 * q + 0], xh[8 * q + 1]);
+          v.y = pack_bf16x2(xh[8 * q + 2], xh[8 * q + 3]);
+          v.z = pack_bf16x2(xh[8 * q + 4], xh[8 * q + 5]);
+          v.w = pack_bf16x2(xh[8 * q + 6], xh[8 * q + 7]);
+          const int c = half * 4 + q;
+          *reinterpret_cast<uint4 *>(ot + ((c ^ (row & 7)) << 4)) = v;
+        }
+        fence_proxy_async_smem();
+      }
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(bar_empty + 8 * s);
+        if (RANK) mbar_arrive(bar_opfull + 8 * s);
+      }
+    }
+  }
+
+  if constexpr (RANK > 0) {
+    // ------------------------------------------------------------ split-K reduction
+    float *red = reinterpret_cast<float *>(smem);  // [RANK][128] fp32, aliases the stages
+    if (warp >= 2) {
+      const int quad = warp & 3;
+      const int row = quad * 32 + lane;
+      const bool second = warp >= 6;
+      bool ok = mbar_wait(bar_acc, 0, a.err, KID_QUANT, 5);
+      tc_fence_after();
+      if (RANK == 16) {
+        if (!second) {
+          uint32_t r[16];
+          tmem_ld16(tbase + (static_cast<uint32_t>(quad * 32) << 16), r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) red[j * 128 + row] = (ok && n_local) ? __uint_as_float(r[j]) : 0.0f;
+        }
+      } else {
+        const int cbase = second ? RANK / 2 : 0;
+#pragma unroll
+        for (int c0 = 0; c0 < RANK / 2; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld32(tbase + (static_cast<uint32_t>(quad * 32) << 16) + cbase + c0, r);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            red[(cbase + c0 + j) * 128 + row] = (ok && n_local) ? __uint_as_float(r[j]) : 0.0f;
+        }
+      }
+      tc_fence_before();
+    }
+    cluster_sync_all();
+    const int rows_per = 128 / nsplit;
+    const int r0 = split * rows_per;
+    const uint32_t red_addr = smem_u32(red);
+    constexpr int PAIRS = RANK / 2;
+    for (int idx = threadIdx.x; idx < rows_per * PAIRS; idx += C::THREADS) {
+      const int row = r0 + idx / PAIRS;
+      const int c = 2 * (idx % PAIRS);
+      float s0 = 0.0f, s1 = 0.0f;
+      for (int src = 0; src < nsplit; ++src) {
+        s0 += ld_shared_cluster_f32(map_shared_rank(red_addr + (c * 128 + row) * 4, src));
+        s1 += ld_shared_cluster_f32(map_shared_rank(red_addr + ((c + 1) * 128 + row) * 4, src));
+      }
+      if (m0 + row < a.M)
+        *reinterpret_cast<uint32_t *>(a.lora_act + static_cast<size_t>(m0 + row) * RANK + c) =
+            pack_bf16x2(__fmul_rn(s0, a.inv_alpha), __fmul_rn(s1, a.inv_alpha));
+    }
+    cluster_sync_all();
+  }
+
+  __syncthreads();
+  if (RANK && warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+template <int RANK, bool QUANT>
+cudaError_t launch_t(const QuantLaunch &q) {
+  using C = QCfg<RANK>;
+  auto kern = k1_quant_act_lora_down<RANK, QUANT>;
+  static int attr_done[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_done[dev] = 1;
+  }
+  QArgs a{q.inv_lambda, q.xq, q.xs, q.lora_act, q.M, q.K, q.s_x, q.d_x, q.inv_alpha, q.chunks_per_split, q.err};
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(q.splits, (q.M + 127) / 128, 1);
+  cfg.blockDim = dim3(C::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = q.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = q.splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = RANK ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, q.tm_x, q.tm_l1, a);
+}
+
+}  // namespace
+
+cudaError_t launch_quant_act(const QuantLaunch &q) {
+  const int r = q.lora ? q.rank : 0;
+  if (q.quantize) {
+    switch (r) {
+      case 0: return launch_t<0, true>(q);
+      case 16: return launch_t<16, true>(q);
+      case 32: return launch_t<32, true>(q);
+      case 64: return launch_t<64, true>(q);
+      case 128: return launch_t<128, true>(q);
+    }
+  } else {
+    switch (r) {
+      case 16: return launch_t<16, false>(q);
+      case 32: return launch_t<32, false>(q);
+      case 64: return launch_t<64, false>(q);
+      case 128: return launch_t<128, false>(q);
+    }
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace svdq

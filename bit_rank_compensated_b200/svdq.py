@@ -1,0 +1,289 @@
+"""Thin ctypes binding of libsvdq (include/svdq.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA kernels.
+PyTorch provides device memory (tensors) and the current CUDA stream. There is no CPU
+fallback: when libsvdq.so is missing or the GPU is not a B200 the calls raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libsvdq.so")
+
+SVDQ_OK = 0
+STATUS_NAMES = {
+    0: "SVDQ_OK", 1: "SVDQ_ERR_INVALID_ARG", 2: "SVDQ_ERR_UNSUPPORTED_ARCH", 3: "SVDQ_ERR_MISALIGNED",
+    4: "SVDQ_ERR_CUDA", 5: "SVDQ_ERR_TIMEOUT", 6: "SVDQ_ERR_INTERNAL", 7: "SVDQ_ERR_UNAVAILABLE",
+}
+RANKS = (0, 16, 32, 64, 128)
+GROUP = 16
+
+# Every symbol include/svdq.h declares.
+EXPORTED = (
+    "svdq_status_string", "svdq_version", "svdq_weight_scale_bytes", "svdq_act_scale_bytes", "svdq_act_absmax",
+    "svdq_prepare_workspace_bytes", "svdq_prepare_weights", "svdq_quantize_rows", "svdq_quant_act_lora_down",
+    "svdq_gemm_w4a4_lora_up", "svdq_linear_forward", "svdq_linear_forward_host", "svdq_baseline_lora_down",
+    "svdq_baseline_quantize", "svdq_baseline_gemm_w4a4", "svdq_baseline_lora_up", "svdq_last_device_error",
+)
+
+
+class SvdqError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn}: {STATUS_NAMES.get(status, status)} ({msg})")
+        self.status = status
+
+
+class LayerStruct(ctypes.Structure):
+    _fields_ = [
+        ("N", ctypes.c_int32), ("K", ctypes.c_int32), ("rank", ctypes.c_int32), ("group", ctypes.c_int32),
+        ("w_tensor_scale", ctypes.c_float), ("x_tensor_scale", ctypes.c_float),
+        ("wq", ctypes.c_void_p), ("ws", ctypes.c_void_p), ("inv_lambda", ctypes.c_void_p),
+        ("lambda_", ctypes.c_void_p), ("L1t", ctypes.c_void_p), ("L2t", ctypes.c_void_p),
+        ("bias", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Loads libsvdq.so (built in-tree by bit_rank_compensated_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing; build it with `python -m bit_rank_compensated_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    LP = ctypes.POINTER(LayerStruct)
+    sig = {
+        "svdq_status_string": ([I], ctypes.c_char_p),
+        "svdq_version": ([], I),
+        "svdq_weight_scale_bytes": ([I, I], S),
+        "svdq_act_scale_bytes": ([I, I], S),
+        "svdq_act_absmax": ([P, I, I, P, P], I),
+        "svdq_prepare_workspace_bytes": ([I, I, I, ctypes.POINTER(I)], S),
+        "svdq_prepare_weights": ([P, P, P, I, I, I, LP, P, S, P], I),
+        "svdq_quantize_rows": ([P, I, I, F, I, P, P, P], I),
+        "svdq_quant_act_lora_down": ([P, I, LP, P, P, P, P], I),
+        "svdq_gemm_w4a4_lora_up": ([P, P, P, I, LP, P, P], I),
+        "svdq_linear_forward": ([P, I, LP, P, P, P, P, P], I),
+        "svdq_linear_forward_host": ([P, I, LP, P, P, P, P, P, P, P], I),
+        "svdq_baseline_lora_down": ([P, I, LP, P, P], I),
+        "svdq_baseline_quantize": ([P, I, LP, P, P, P], I),
+        "svdq_baseline_gemm_w4a4": ([P, P, I, LP, P, P], I),
+        "svdq_baseline_lora_up": ([P, I, LP, P, P], I),
+        "svdq_last_device_error": ([P, ctypes.POINTER(ctypes.c_uint32)], I),
+    }
+    for name, (args, res) in sig.items():
+        f = getattr(lib, name)
+        f.argtypes = args
+        f.restype = res
+    _lib = lib
+    return lib
+
+
+def _check(fn: str, status: int):
+    if status != SVDQ_OK:
+        raise SvdqError(fn, status, load().svdq_status_string(status).decode())
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def weight_scale_bytes(N: int, K: int) -> int:
+    return load().svdq_weight_scale_bytes(N, K)
+
+
+def act_scale_bytes(M: int, K: int) -> int:
+    return load().svdq_act_scale_bytes(M, K)
+
+
+class Layer:
+    """Device buffers of one prepared layer (tensors) plus the C struct that points at them."""
+
+    def __init__(self, N: int, K: int, rank: int, device="cuda", with_bias: bool = True):
+        if rank not in RANKS:
+            raise ValueError(f"rank must be one of {RANKS}")
+        self.N, self.K, self.rank = N, K, rank
+        u8 = dict(dtype=torch.uint8, device=device)
+        self.wq = torch.empty(N * K // 2, **u8)
+        self.ws = torch.empty(weight_scale_bytes(N, K), **u8)
+        self.inv_lambda = torch.empty(K, dtype=torch.float32, device=device)
+        self.lam = torch.empty(K, dtype=torch.float32, device=device)
+        self.L1t = torch.empty(max(rank, 1) * K, dtype=torch.bfloat16, device=device) if rank else None
+        self.L2t = torch.empty(N * max(rank, 1), dtype=torch.bfloat16, device=device) if rank else None
+        self.bias = torch.zeros(N, dtype=torch.float32, device=device) if with_bias else None
+        self.s = LayerStruct()
+        self.s.N, self.s.K, self.s.rank, self.s.group = N, K, rank, GROUP
+        self.s.w_tensor_scale = 1.0
+        self.s.x_tensor_scale = 1.0
+        self._sync_ptrs()
+
+    def _sync_ptrs(self):
+        self.s.wq = self.wq.data_ptr()
+        self.s.ws = self.ws.data_ptr()
+        self.s.inv_lambda = self.inv_lambda.data_ptr()
+        self.s.lambda_ = self.lam.data_ptr()
+        self.s.L1t = self.L1t.data_ptr() if self.L1t is not None else None
+        self.s.L2t = self.L2t.data_ptr() if self.L2t is not None else None
+        self.s.bias = self.bias.data_ptr() if self.bias is not None else None
+
+    @property
+    def s_w(self) -> float:
+        return float(self.s.w_tensor_scale)
+
+    @property
+    def s_x(self) -> float:
+        return float(self.s.x_tensor_scale)
+
+    @classmethod
+    def from_arrays(cls, *, N, K, rank, wq, ws, inv_lambda, L1t, L2t, bias, s_w, s_x, lam=None, device="cuda"):
+        """Builds a layer from already prepared host arrays (numpy): packed codes, block-layout
+        scales, inv_lambda, L1t / L2t as bf16 bit patterns (uint16), bias (or None)."""
+        import numpy as np
+
+        L = cls(N, K, rank, device=device, with_bias=bias is not None)
+        L.wq.copy_(torch.from_numpy(np.ascontiguousarray(wq, dtype=np.uint8).reshape(-1)))
+        L.ws.copy_(torch.from_numpy(np.ascontiguousarray(ws, dtype=np.uint8).reshape(-1)))
+        L.inv_lambda.copy_(torch.from_numpy(np.ascontiguousarray(inv_lambda, dtype=np.float32)))
+        if lam is not None:
+            L.lam.copy_(torch.from_numpy(np.ascontiguousarray(lam, dtype=np.float32)))
+        if rank:
+            L.L1t.view(torch.int16).copy_(torch.from_numpy(np.ascontiguousarray(L1t, dtype=np.uint16).reshape(-1).view(np.int16)))
+            L.L2t.view(torch.int16).copy_(torch.from_numpy(np.ascontiguousarray(L2t, dtype=np.uint16).reshape(-1).view(np.int16)))
+        if bias is not None:
+            L.bias.copy_(torch.from_numpy(np.ascontiguousarray(bias, dtype=np.float32)))
+        L.s.w_tensor_scale = float(s_w)
+        L.s.x_tensor_scale = float(s_x)
+        return L
+
+
+def act_absmax(X: torch.Tensor, stream=None) -> torch.Tensor:
+    M, K = X.shape
+    out = torch.empty(K, dtype=torch.float32, device=X.device)
+    _check("svdq_act_absmax", load().svdq_act_absmax(_ptr(X), M, K, _ptr(out), _stream(stream)))
+    return out
+
+
+def prepare_workspace_bytes(N: int, K: int, rank: int) -> int:
+    st = ctypes.c_int(0)
+    n = load().svdq_prepare_workspace_bytes(N, K, rank, ctypes.byref(st))
+    _check("svdq_prepare_workspace_bytes", st.value)
+    return n
+
+
+def prepare_weights(W: torch.Tensor, bias: torch.Tensor | None, act_absmax_: torch.Tensor, rank: int,
+                    stream=None) -> Layer:
+    N, K = W.shape
+    L = Layer(N, K, rank, device=W.device, with_bias=bias is not None)
+    ws = torch.empty(prepare_workspace_bytes(N, K, rank), dtype=torch.uint8, device=W.device)
+    _check("svdq_prepare_weights", load().svdq_prepare_weights(
+        _ptr(W), _ptr(bias), _ptr(act_absmax_), N, K, rank, ctypes.byref(L.s), _ptr(ws), ws.numel(),
+        _stream(stream)))
+    del ws
+    return L
+
+
+def quantize_rows(A: torch.Tensor, s: float, row_pad: int = 256, stream=None):
+    rows, K = A.shape
+    codes = torch.empty(rows * K // 2, dtype=torch.uint8, device=A.device)
+    pad = (rows + row_pad - 1) // row_pad * row_pad
+    scales = torch.empty(pad * K // 16, dtype=torch.uint8, device=A.device)
+    _check("svdq_quantize_rows", load().svdq_quantize_rows(
+        _ptr(A), rows, K, float(s), row_pad, _ptr(codes), _ptr(scales), _stream(stream)))
+    return codes, scales
+
+
+def alloc_activations(M: int, layer: Layer, device="cuda"):
+    xq = torch.empty(M * layer.K // 2, dtype=torch.uint8, device=device)
+    xs = torch.empty(act_scale_bytes(M, layer.K), dtype=torch.uint8, device=device)
+    la = torch.empty(M * max(layer.rank, 1), dtype=torch.bfloat16, device=device) if layer.rank else None
+    return xq, xs, la
+
+
+def quant_act_lora_down(X: torch.Tensor, layer: Layer, xq=None, xs=None, lora_act=None, stream=None):
+    M = X.shape[0]
+    if xq is None:
+        xq, xs, lora_act = alloc_activations(M, layer, X.device)
+    _check("svdq_quant_act_lora_down", load().svdq_quant_act_lora_down(
+        _ptr(X), M, ctypes.byref(layer.s), _ptr(xq), _ptr(xs), _ptr(lora_act), _stream(stream)))
+    return xq, xs, lora_act
+
+
+def gemm_w4a4_lora_up(xq, xs, lora_act, M: int, layer: Layer, Y=None, stream=None):
+    if Y is None:
+        Y = torch.empty(M, layer.N, dtype=torch.bfloat16, device=xq.device)
+    _check("svdq_gemm_w4a4_lora_up", load().svdq_gemm_w4a4_lora_up(
+        _ptr(xq), _ptr(xs), _ptr(lora_act), M, ctypes.byref(layer.s), _ptr(Y), _stream(stream)))
+    return Y
+
+
+def linear_forward(X: torch.Tensor, layer: Layer, bufs=None, Y=None, stream=None):
+    M = X.shape[0]
+    xq, xs, la = bufs if bufs is not None else alloc_activations(M, layer, X.device)
+    if Y is None:
+        Y = torch.empty(M, layer.N, dtype=torch.bfloat16, device=X.device)
+    _check("svdq_linear_forward", load().svdq_linear_forward(
+        _ptr(X), M, ctypes.byref(layer.s), _ptr(xq), _ptr(xs), _ptr(la), _ptr(Y), _stream(stream)))
+    return Y
+
+
+def linear_forward_host(X_host: torch.Tensor, layer: Layer, X_dev, bufs, Y_dev, Y_host, stream=None):
+    M = X_host.shape[0]
+    xq, xs, la = bufs
+    _check("svdq_linear_forward_host", load().svdq_linear_forward_host(
+        _ptr(X_host), M, ctypes.byref(layer.s), _ptr(X_dev), _ptr(xq), _ptr(xs), _ptr(la), _ptr(Y_dev),
+        _ptr(Y_host), _stream(stream)))
+    return Y_host
+
+
+def baseline_lora_down(X, layer, lora_act, stream=None):
+    _check("svdq_baseline_lora_down", load().svdq_baseline_lora_down(
+        _ptr(X), X.shape[0], ctypes.byref(layer.s), _ptr(lora_act), _stream(stream)))
+
+
+def baseline_quantize(X, layer, xq, xs, stream=None):
+    _check("svdq_baseline_quantize", load().svdq_baseline_quantize(
+        _ptr(X), X.shape[0], ctypes.byref(layer.s), _ptr(xq), _ptr(xs), _stream(stream)))
+
+
+def baseline_gemm_w4a4(xq, xs, M, layer, Y, stream=None):
+    _check("svdq_baseline_gemm_w4a4", load().svdq_baseline_gemm_w4a4(
+        _ptr(xq), _ptr(xs), M, ctypes.byref(layer.s), _ptr(Y), _stream(stream)))
+
+
+def baseline_lora_up(lora_act, M, layer, Y, stream=None):
+    _check("svdq_baseline_lora_up", load().svdq_baseline_lora_up(
+        _ptr(lora_act), M, ctypes.byref(layer.s), _ptr(Y), _stream(stream)))
+
+
+def unfused_forward(X, layer, bufs, Y, stream=None):
+    """The naive branch of the unfused baseline: four separate kernels."""
+    xq, xs, la = bufs
+    M = X.shape[0]
+    if layer.rank:
+        baseline_lora_down(X, layer, la, stream)
+    baseline_quantize(X, layer, xq, xs, stream)
+    baseline_gemm_w4a4(xq, xs, M, layer, Y, stream)
+    if layer.rank:
+        baseline_lora_up(la, M, layer, Y, stream)
+    return Y
+
+
+def last_device_error(stream=None) -> int:
+    code = ctypes.c_uint32(0)
+    st = load().svdq_last_device_error(_stream(stream), ctypes.byref(code))
+    if st not in (SVDQ_OK, 5):
+        _check("svdq_last_device_error", st)
+    return int(code.value)

@@ -1,0 +1,207 @@
+/*
+ * libsvdq — SVDQuant NVFP4 W4A4 + low-rank linear layer for NVIDIA B200 (sm_100a).
+ *
+ * The layer computes   Y = Q(X_hat) Q(R)^T + (X_hat L1) L2 + b
+ * where X_hat = X diag(lambda)^-1 is the smoothed activation, W_hat = W diag(lambda) the
+ * smoothed weight, W_hat^T ~ L1 L2 its rank-r SVD branch (bf16) and R = W_hat - (L1 L2)^T
+ * the residual; Q() is NVFP4 quantization (e2m1 codes, one e4m3 scale per 16 elements
+ * along K, one fp32 tensor scale).
+ *   - outlier migration and low-rank split: "Svdq Int4 Flux.1 Canny Dev" model card,
+ *     section "SVDQuant 概述", stages 1-3;
+ *   - fusion of the down-projection with the activation quantizer and of the up-projection
+ *     with the 4-bit GEMM: same card, section "Nunchaku 引擎設計", (a) and (b);
+ *   - NVFP4, group size 16, rank 32: "Nunchaku Lite in Diffusers" (blog post), section
+ *     on the quantization_config block ("التحميل الأصلي في الناشرون");
+ *   - refusing unsupported GPUs with a clear error: same post, "دعم الأجهزة".
+ *
+ * Conventions for every entry point:
+ *   - Shapes follow nn.Linear: X is M x K (tokens x in-features), W is N x K, Y is M x N.
+ *     All matrices are row-major and contiguous.
+ *   - "device" pointers are CUDA device (or managed) memory; "host" pointers are host memory.
+ *     All buffers are owned by the caller; the library never allocates or frees them.
+ *   - bf16 values are passed as uint16_t bit patterns.
+ *   - stream is a cudaStream_t passed as void* (NULL = the legacy default stream). Unless a
+ *     function says otherwise it only enqueues work and returns; results are ready when the
+ *     stream reaches that point.
+ *   - Device pointers must be 16-byte aligned.
+ *   - Shape limits: M >= 1; K % 64 == 0; N % 16 == 0; rank in {0, 16, 32, 64, 128}.
+ *     Other values return SVDQ_ERR_INVALID_ARG; misaligned pointers SVDQ_ERR_MISALIGNED.
+ *   - The first call on a device checks for compute capability 10.0 and returns
+ *     SVDQ_ERR_UNSUPPORTED_ARCH on any other GPU. There is no fallback path.
+ *   - Device-side waits are bounded; a kernel that gives up records a code that
+ *     svdq_last_device_error() returns (and the kernel's outputs are then undefined).
+ *
+ * Storage formats:
+ *   - NVFP4 codes: K-major, two e2m1 codes per byte, element 2i in the low nibble;
+ *     a matrix with `rows` rows takes rows * K / 2 bytes.
+ *   - Group scales (e4m3 codes): block layout consumed by the tensor-core GEMM. The scales
+ *     of rows [128 b, 128 b + 128) and groups [4 c, 4 c + 4) (64 elements of K) fill one
+ *     512-byte block at ((b * (K / 64)) + c) * 512; inside it, (row m, group g) sits at
+ *     (m % 32) * 16 + ((m % 128) / 32) * 4 + g % 4. Rows are padded (with zero scales):
+ *     activations to a multiple of 128, weights to a multiple of 256.
+ */
+#ifndef SVDQ_H
+#define SVDQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SVDQ_API __attribute__((visibility("default")))
+#else
+#define SVDQ_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum svdq_status {
+  SVDQ_OK = 0,
+  SVDQ_ERR_INVALID_ARG = 1,      /* a shape, rank or null pointer outside the contract */
+  SVDQ_ERR_UNSUPPORTED_ARCH = 2, /* not a compute capability 10.0 GPU */
+  SVDQ_ERR_MISALIGNED = 3,       /* a device pointer is not 16-byte aligned */
+  SVDQ_ERR_CUDA = 4,             /* a CUDA runtime call or a kernel launch failed */
+  SVDQ_ERR_TIMEOUT = 5,          /* a kernel gave up on a bounded wait */
+  SVDQ_ERR_INTERNAL = 6,         /* an internal consistency check failed */
+  SVDQ_ERR_UNAVAILABLE = 7       /* a runtime dependency (the eigen-solver library) is missing */
+} svdq_status;
+
+/* One prepared layer. Every pointer is a caller-allocated device buffer of the stated size;
+ * svdq_prepare_weights fills them and the two scalar tensor scales. */
+typedef struct svdq_layer {
+  int32_t N, K, rank;
+  int32_t group;            /* always 16 */
+  float w_tensor_scale;     /* s_w = fp32(max|R| / 2688) (1 when R == 0) */
+  float x_tensor_scale;     /* s_x = fp32(max_j fp32(a_x[j] inv_lambda[j]) / 2688), calibrated */
+  uint8_t *wq;              /* N * K / 2 bytes: NVFP4 codes of R (fp32-rounded residual) */
+  uint8_t *ws;              /* svdq_weight_scale_bytes(N, K) bytes: e4m3 group scales of R */
+  float *inv_lambda;        /* K floats: fp32(1 / lambda_j) */
+  float *lambda;            /* K floats: lambda_j (optional; written by prepare when not NULL) */
+  uint16_t *L1t;            /* rank * K bf16: L1 transposed (row j = column j of L1); NULL if rank 0 */
+  uint16_t *L2t;            /* N * rank bf16: L2 transposed (row n = column n of L2); NULL if rank 0 */
+  float *bias;              /* N floats, or NULL for no bias */
+} svdq_layer;
+
+/* Human-readable name of a status code (static string). */
+SVDQ_API const char *svdq_status_string(svdq_status s);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+SVDQ_API int svdq_version(void);
+
+/* Bytes of the weight group-scale buffer (rows padded to a multiple of 256). */
+SVDQ_API size_t svdq_weight_scale_bytes(int N, int K);
+
+/* Bytes of the activation group-scale buffer (rows padded to a multiple of 128). */
+SVDQ_API size_t svdq_act_scale_bytes(int M, int K);
+
+/* Calibration maxima a_x[j] = max_m |X[m, j]| over the rows of X (the activation side of
+ * the smoothing factor; "SVDQuant 概述" stage 2).
+ *   X       device, M x K bf16.
+ *   absmax  device, K floats (overwritten).
+ * Asynchronous on stream. */
+SVDQ_API svdq_status svdq_act_absmax(const uint16_t *X, int M, int K, float *absmax, void *stream);
+
+/* Workspace (device bytes) that svdq_prepare_weights needs for an N x K weight at this rank.
+ * Loads the eigen-solver library on first use (SVDQ_ERR_UNAVAILABLE if it cannot). Returns 0
+ * and sets *status on error when status is not NULL. */
+SVDQ_API size_t svdq_prepare_workspace_bytes(int N, int K, int rank, svdq_status *status);
+
+/* Offline step, once per layer ("SVDQuant 概述" stages 2 and 3; packing for the kernels):
+ *   a_w[j] = max_n |W[n, j]|; lambda_j = fp32(fp32(sqrt a_x[j]) / fp32(sqrt a_w[j])), 1 when
+ *   either is 0; inv_lambda_j = fp32(1 / lambda_j); W_hat = W diag(lambda) (fp64);
+ *   truncated SVD W_hat^T = P S Q^T (fp64, from the eigen-decomposition of the smaller Gram
+ *   matrix), sign fixed so that the largest-magnitude entry of each column of P is positive;
+ *   L1 = bf16(P_r S_r^1/2), L2 = bf16(S_r^1/2 Q_r^T); R = fp32(W_hat - (L1 L2)^T) (fp64 before
+ *   the final rounding); s_w, s_x as in svdq_layer; R quantized to NVFP4 with s_w.
+ *   W           device, N x K fp32.
+ *   bias        device, N fp32, or NULL. Copied into layer->bias when both are non-NULL.
+ *   act_absmax  device, K fp32: calibration maxima a_x (e.g. from svdq_act_absmax).
+ *   layer       in: N, K, rank and the device buffers; out: buffers filled, group = 16,
+ *               w_tensor_scale and x_tensor_scale set.
+ *   workspace   device, at least svdq_prepare_workspace_bytes(N, K, rank) bytes.
+ * Synchronous: returns after the work on stream has finished. */
+SVDQ_API svdq_status svdq_prepare_weights(const float *W, const float *bias, const float *act_absmax,
+                                 int N, int K, int rank, svdq_layer *layer,
+                                 void *workspace, size_t workspace_bytes, void *stream);
+
+/* NVFP4 quantization of the rows of a fp32 matrix A (rows x K) with tensor scale s
+ * ("التحميل الأصلي في الناشرون": nvfp4, group 16). Per 16-element group along K:
+ *   amax = max|a|; scale = e4m3_rn_satfinite(fp32(amax / fp32(6 s)));
+ *   code_i = 0 if scale == 0, else e2m1_rn_satfinite(fp32(a_i / fp32(scale * s)));
+ *   a value that rounds to zero encodes as +0.
+ *   A      device, rows x K fp32.
+ *   codes  device, rows * K / 2 bytes (packed as described above).
+ *   scales device, block layout with rows padded to a multiple of row_pad (128 or 256);
+ *          the padding rows are written as zero scales.
+ * Asynchronous on stream. */
+SVDQ_API svdq_status svdq_quantize_rows(const float *A, int rows, int K, float s, int row_pad,
+                               uint8_t *codes, uint8_t *scales, void *stream);
+
+/* K1 — one pass over X ("Nunchaku 引擎設計" (b): the down-projection and the quantizer read
+ * the same input, so they run as one kernel):
+ *   X_hat[m, k] = fp32(X[m, k] * inv_lambda[k]);
+ *   xq, xs   = NVFP4(X_hat) with tensor scale s_x (same rule as svdq_quantize_rows);
+ *   lora_act = bf16( (sum_k bf16(X_hat[m, k]) L1[k, :]) / alpha ),  alpha = fp32(s_x * s_w),
+ *              accumulated in fp32 on the tensor cores. The 1/alpha pre-scaling lets K2 add
+ *              the branch to the same fp32 accumulator as the 4-bit product.
+ *   X         device, M x K bf16.
+ *   xq        device, M * K / 2 bytes.
+ *   xs        device, svdq_act_scale_bytes(M, K) bytes (padding rows written as zero).
+ *   lora_act  device, M x rank bf16 (unused and may be NULL when rank == 0).
+ * Asynchronous on stream. */
+SVDQ_API svdq_status svdq_quant_act_lora_down(const uint16_t *X, int M, const svdq_layer *layer,
+                                     uint8_t *xq, uint8_t *xs, uint16_t *lora_act, void *stream);
+
+/* K2 — block-scaled FP4 tensor-core GEMM with the up-projection in its output stage
+ * ("Nunchaku 引擎設計" (b): the up-projection and the 4-bit GEMM share one output):
+ *   acc[m, n] = sum_g xs[m,g] ws[n,g] sum_{k in g} e2m1(xq[m,k]) e2m1(wq[n,k])
+ *               + sum_j lora_act[m, j] L2[j, n]                       (fp32, tensor memory)
+ *   Y[m, n]   = bf16(alpha * acc[m, n] + bias[n]),  alpha = fp32(s_x * s_w).
+ *   xq, xs, lora_act  as written by svdq_quant_act_lora_down.
+ *   Y         device, M x N bf16 (written once).
+ * Asynchronous on stream. */
+SVDQ_API svdq_status svdq_gemm_w4a4_lora_up(const uint8_t *xq, const uint8_t *xs, const uint16_t *lora_act,
+                                   int M, const svdq_layer *layer, uint16_t *Y, void *stream);
+
+/* K1 then K2 on the same stream (the layer's forward pass). Buffers as above. */
+SVDQ_API svdq_status svdq_linear_forward(const uint16_t *X, int M, const svdq_layer *layer,
+                                uint8_t *xq, uint8_t *xs, uint16_t *lora_act,
+                                uint16_t *Y, void *stream);
+
+/* The forward pass from and to host memory: copies X_host (M x K bf16) to X_dev, runs
+ * svdq_linear_forward, copies Y_dev (M x N bf16) back to Y_host, all enqueued on stream
+ * (pinned host buffers make the copies asynchronous). Synchronous: returns after the
+ * stream has finished. */
+SVDQ_API svdq_status svdq_linear_forward_host(const uint16_t *X_host, int M, const svdq_layer *layer,
+                                     uint16_t *X_dev, uint8_t *xq, uint8_t *xs,
+                                     uint16_t *lora_act, uint16_t *Y_dev, uint16_t *Y_host,
+                                     void *stream);
+
+/* Unfused baseline: the low-rank branch as separate kernels around the 4-bit GEMM
+ * ("Nunchaku 引擎設計" (a): the branch run naively re-reads the 16-bit input in the
+ * down-projection and re-writes the 16-bit output in the up-projection).
+ *   svdq_baseline_lora_down: lora_act = bf16(sum_k bf16(X_hat) L1 / alpha) (reads X).
+ *   svdq_baseline_quantize:  xq, xs = NVFP4(X_hat) (reads X again).
+ *   svdq_baseline_gemm_w4a4: Y = bf16(alpha * 4-bit product + bias) (no branch).
+ *   svdq_baseline_lora_up:   Y = bf16(Y + alpha * lora_act L2) (reads and rewrites Y).
+ * Same buffers and formats as the fused calls. Asynchronous on stream. */
+SVDQ_API svdq_status svdq_baseline_lora_down(const uint16_t *X, int M, const svdq_layer *layer,
+                                    uint16_t *lora_act, void *stream);
+SVDQ_API svdq_status svdq_baseline_quantize(const uint16_t *X, int M, const svdq_layer *layer,
+                                   uint8_t *xq, uint8_t *xs, void *stream);
+SVDQ_API svdq_status svdq_baseline_gemm_w4a4(const uint8_t *xq, const uint8_t *xs, int M,
+                                    const svdq_layer *layer, uint16_t *Y, void *stream);
+SVDQ_API svdq_status svdq_baseline_lora_up(const uint16_t *lora_act, int M, const svdq_layer *layer,
+                                  uint16_t *Y, void *stream);
+
+/* Reads and clears the device-side error word after synchronizing stream. *code is 0 when
+ * no kernel gave up on a wait; otherwise (kernel id << 16) | (site << 8) | 1.
+ * Returns SVDQ_ERR_TIMEOUT when *code != 0. */
+SVDQ_API svdq_status svdq_last_device_error(void *stream, uint32_t *code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SVDQ_H */
