@@ -188,9 +188,9 @@ svdq_status run_gemm(const uint8_t *xq, const uint8_t *xs, const uint16_t *la, i
       return SVDQ_ERR_CUDA;
   }
   if (r > 0) {
-    const uint32_t kc = r < 64 ? r : 64;
+    const uint32_t kc = r < 32 ? r : 32;
     const CUtensorMapSwizzle sw = swizzle_for_row_bytes(kc * 2);
-    if (!make_map(&g.tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, la, r, M, static_cast<uint64_t>(r) * 2, kc, 128, sw) ||
+    if (!make_map(&g.tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, la, 2 * r, M, static_cast<uint64_t>(r) * 4, kc, 128, sw) ||
         !make_map(&g.tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L2t, r, N, static_cast<uint64_t>(r) * 2, kc, 256, sw))
       return SVDQ_ERR_CUDA;
   }

@@ -7,8 +7,9 @@
 //
 // Persistent kernel, one CTA per SM, output tiles of 128 x 256 (rows of X x rows of W).
 // Per tile the k-loop is a sequence of pipeline steps through a 4-stage shared-memory ring:
-//   - rank / 64 (at least one) low-rank steps: lora_act tile (128 x kc bf16) and L2t tile
-//     (256 x kc bf16), kc = min(rank, 64); bf16 tcgen05 MMAs (K = 16 each);
+//   - rank / kc low-rank steps, kc = min(rank, 32): the hi and lo planes of lora_act
+//     (128 x kc bf16 each) and an L2t tile (256 x kc bf16); bf16 tcgen05 MMAs (K = 16 each),
+//     hi and lo against the same L2t tile;
 //   - K / 256 4-bit steps: xq tile (128 rows x 128 bytes), wq tile (256 x 128 bytes), both with
 //     128B swizzle, plus their e4m3 scale blocks (512 bytes per 128 rows x 64 elements), copied
 //     into tensor memory with tcgen05.cp; four kind::mxf4nvf4 MMAs (K = 64 each).
@@ -55,12 +56,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     k2_gemm_w4a4_lora_up(const __grid_constant__ CUtensorMap tm_xq, const __grid_constant__ CUtensorMap tm_wq,
                          const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_l2,
                          GArgs a) {
-  constexpr int KC = RANK == 0 ? 64 : (RANK < 64 ? RANK : 64);
+  // Low-rank steps: kc columns of lora_act (hi and lo planes) and of L2t per step.
+  constexpr int KC = RANK == 0 ? 32 : (RANK < 32 ? RANK : 32);
   constexpr int N_LORA = RANK == 0 ? 0 : RANK / KC;
   constexpr uint32_t LORA_ROW = KC * 2;  // bytes per row of a low-rank tile
-  constexpr uint32_t LORA_SWZ = LORA_ROW == 128 ? 2u : (LORA_ROW == 64 ? 4u : 6u);
+  constexpr uint32_t LORA_SWZ = LORA_ROW == 64 ? 4u : 6u;
   constexpr uint32_t LORA_A_BYTES = 128u * LORA_ROW;
   constexpr uint32_t LORA_B_BYTES = 256u * LORA_ROW;
+  constexpr uint32_t LORA_LO_OFF = 8192u;  // lo plane inside the A slot
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -125,8 +128,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           const uint32_t fb = bar_full + 8 * s;
           if (j < N_LORA) {
-            mbar_arrive_expect_tx(fb, LORA_A_BYTES + LORA_B_BYTES);
+            mbar_arrive_expect_tx(fb, 2 * LORA_A_BYTES + LORA_B_BYTES);
             tma_load_2d(smem_u32(a_tile(s)), &tm_la, j * KC, mt * BM, fb);
+            tma_load_2d(smem_u32(a_tile(s)) + LORA_LO_OFF, &tm_la, RANK + j * KC, mt * BM, fb);
             tma_load_2d(smem_u32(b_tile(s)), &tm_l2, j * KC, nt * BN, fb);
           } else {
             const int kt = j - N_LORA;
@@ -167,10 +171,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_after();
           if (j < N_LORA) {
             const uint64_t ad = umma_desc(smem_u32(a_tile(s)), 16, 8 * LORA_ROW, LORA_SWZ);
+            const uint64_t ald = umma_desc(smem_u32(a_tile(s)) + LORA_LO_OFF, 16, 8 * LORA_ROW, LORA_SWZ);
             const uint64_t bd = umma_desc(smem_u32(b_tile(s)), 16, 8 * LORA_ROW, LORA_SWZ);
 #pragma unroll
-            for (int k = 0; k < KC / 16; ++k)
+            for (int k = 0; k < KC / 16; ++k) {
               mma_bf16(tbase, ad + 2u * k, bd + 2u * k, idesc_bf16, (j | k) != 0 ? 1u : 0u);
+              mma_bf16(tbase, ald + 2u * k, bd + 2u * k, idesc_bf16, 1u);
+            }
           } else {
             const int kt = j - N_LORA;
             const int kbv = min(4, kblocks - 4 * kt);

@@ -8,6 +8,9 @@
 // down-projections are summed through distributed shared memory in cluster-rank order, so
 // the result is deterministic and nothing goes through global scratch memory.
 //
+// The down-projection is stored pre-divided by alpha = s_x s_w as an unevaluated sum of two
+// bf16 values (hi + lo), so the fp32 result reaches K2 without a 16-bit rounding.
+//
 // Warp roles (320 threads):
 //   warp 0      TMA producer: X chunk (128 x 64 bf16, 128B swizzle) and L1t chunk (rank x 64).
 //   warp 1      owns the tensor-memory accumulator (128 lanes x rank fp32 columns) and issues
@@ -241,9 +244,16 @@ __global__ void __launch_bounds__(320, 1)
         s0 += ld_shared_cluster_f32(map_shared_rank(red_addr + (c * 128 + row) * 4, src));
         s1 += ld_shared_cluster_f32(map_shared_rank(red_addr + ((c + 1) * 128 + row) * 4, src));
       }
-      if (m0 + row < a.M)
-        *reinterpret_cast<uint32_t *>(a.lora_act + static_cast<size_t>(m0 + row) * RANK + c) =
-            pack_bf16x2(__fmul_rn(s0, a.inv_alpha), __fmul_rn(s1, a.inv_alpha));
+      if (m0 + row < a.M) {
+        // lora_act row = [hi(0..RANK-1) | lo(0..RANK-1)], v ~ hi + lo with hi = bf16(v),
+        // lo = bf16(v - hi): the pair carries ~16 significant bits of the fp32 value.
+        const float v0 = __fmul_rn(s0, a.inv_alpha), v1 = __fmul_rn(s1, a.inv_alpha);
+        const uint32_t hi = pack_bf16x2(v0, v1);
+        const uint32_t lo = pack_bf16x2(__fsub_rn(v0, bf16_lo(hi)), __fsub_rn(v1, bf16_hi(hi)));
+        uint16_t *dst = a.lora_act + static_cast<size_t>(m0 + row) * (2 * RANK) + c;
+        *reinterpret_cast<uint32_t *>(dst) = hi;
+        *reinterpret_cast<uint32_t *>(dst + RANK) = lo;
+      }
     }
     cluster_sync_all();
   }

@@ -208,7 +208,8 @@ def quantize_rows(A: torch.Tensor, s: float, row_pad: int = 256, stream=None):
 def alloc_activations(M: int, layer: Layer, device="cuda"):
     xq = torch.empty(M * layer.K // 2, dtype=torch.uint8, device=device)
     xs = torch.empty(act_scale_bytes(M, layer.K), dtype=torch.uint8, device=device)
-    la = torch.empty(M * max(layer.rank, 1), dtype=torch.bfloat16, device=device) if layer.rank else None
+    # lora_act rows hold [hi | lo] bf16 planes of the pre-scaled down-projection
+    la = torch.empty(M * 2 * layer.rank, dtype=torch.bfloat16, device=device) if layer.rank else None
     return xq, xs, la
 
 

@@ -142,13 +142,16 @@ SVDQ_API svdq_status svdq_quantize_rows(const float *A, int rows, int K, float s
  * the same input, so they run as one kernel):
  *   X_hat[m, k] = fp32(X[m, k] * inv_lambda[k]);
  *   xq, xs   = NVFP4(X_hat) with tensor scale s_x (same rule as svdq_quantize_rows);
- *   lora_act = bf16( (sum_k bf16(X_hat[m, k]) L1[k, :]) / alpha ),  alpha = fp32(s_x * s_w),
+ *   v[m, :]  = fp32( (sum_k bf16(X_hat[m, k]) L1[k, :]) / alpha ),  alpha = fp32(s_x * s_w),
  *              accumulated in fp32 on the tensor cores. The 1/alpha pre-scaling lets K2 add
  *              the branch to the same fp32 accumulator as the 4-bit product.
+ *   lora_act row m = [hi | lo] (2 * rank bf16): hi = bf16(v), lo = bf16(v - hi), so hi + lo
+ *              carries v with ~16 significant bits (no 16-bit rounding of the branch's
+ *              intermediate before the up-projection).
  *   X         device, M x K bf16.
  *   xq        device, M * K / 2 bytes.
  *   xs        device, svdq_act_scale_bytes(M, K) bytes (padding rows written as zero).
- *   lora_act  device, M x rank bf16 (unused and may be NULL when rank == 0).
+ *   lora_act  device, M x (2 * rank) bf16 (unused and may be NULL when rank == 0).
  * Asynchronous on stream. */
 SVDQ_API svdq_status svdq_quant_act_lora_down(const uint16_t *X, int M, const svdq_layer *layer,
                                      uint8_t *xq, uint8_t *xs, uint16_t *lora_act, void *stream);
@@ -156,7 +159,7 @@ SVDQ_API svdq_status svdq_quant_act_lora_down(const uint16_t *X, int M, const sv
 /* K2 — block-scaled FP4 tensor-core GEMM with the up-projection in its output stage
  * ("Nunchaku 引擎設計" (b): the up-projection and the 4-bit GEMM share one output):
  *   acc[m, n] = sum_g xs[m,g] ws[n,g] sum_{k in g} e2m1(xq[m,k]) e2m1(wq[n,k])
- *               + sum_j lora_act[m, j] L2[j, n]                       (fp32, tensor memory)
+ *               + sum_j (hi[m, j] + lo[m, j]) L2[j, n]                 (fp32, tensor memory)
  *   Y[m, n]   = bf16(alpha * acc[m, n] + bias[n]),  alpha = fp32(s_x * s_w).
  *   xq, xs, lora_act  as written by svdq_quant_act_lora_down.
  *   Y         device, M x N bf16 (written once).
@@ -181,7 +184,7 @@ SVDQ_API svdq_status svdq_linear_forward_host(const uint16_t *X_host, int M, con
 /* Unfused baseline: the low-rank branch as separate kernels around the 4-bit GEMM
  * ("Nunchaku 引擎設計" (a): the branch run naively re-reads the 16-bit input in the
  * down-projection and re-writes the 16-bit output in the up-projection).
- *   svdq_baseline_lora_down: lora_act = bf16(sum_k bf16(X_hat) L1 / alpha) (reads X).
+ *   svdq_baseline_lora_down: lora_act = hi/lo pair of sum_k bf16(X_hat) L1 / alpha (reads X).
  *   svdq_baseline_quantize:  xq, xs = NVFP4(X_hat) (reads X again).
  *   svdq_baseline_gemm_w4a4: Y = bf16(alpha * 4-bit product + bias) (no branch).
  *   svdq_baseline_lora_up:   Y = bf16(Y + alpha * lora_act L2) (reads and rewrites Y).

@@ -63,3 +63,17 @@ def bf16_tensor_to_np(t):
 
 def alpha32(layer: O.Layer) -> float:
     return float(np.float32(np.float32(layer.s_x) * np.float32(layer.s_w)))
+
+
+def lora_pair_bits(v):
+    """[hi | lo] bf16 planes of fp32 values v (rows x r): hi = bf16(v), lo = bf16(v - hi)."""
+    v32 = np.asarray(v, dtype=np.float32)
+    hi = f32_to_bf16_bits(v32)
+    lo = f32_to_bf16_bits((v32 - bf16_bits_to_f32(hi)).astype(np.float32))
+    return np.concatenate([hi, lo], axis=1)
+
+
+def lora_pair_value(la_tensor, M, r):
+    """hi + lo of a lora_act buffer, fp64 (M x r)."""
+    both = bf16_tensor_to_np(la_tensor).reshape(M, 2 * r)
+    return both[:, :r] + both[:, r:]
