@@ -34,7 +34,7 @@ constexpr uint32_t SFA_BYTES = 2048u;
 constexpr uint32_t SFB_BYTES = 4096u;
 constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 55296 = 54 KiB
 constexpr uint32_t DATA_BYTES = STAGES * STAGE_BYTES;
-constexpr uint32_t SMEM = DATA_BYTES + 256 + 1024;
+constexpr uint32_t SMEM = DATA_BYTES + 256 + BN * 4 + 1024;  // + barriers, bias stage, alignment
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = 256;   // scale columns follow the accumulator
 constexpr uint32_t SF_COLS = 48;    // per stage: 4 k-blocks x (4 SFA + 8 SFB) columns
@@ -203,58 +203,78 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else {
     // ------------------------------------------------------------ output stage
+    // Per tile: stage the tile's 256 bias values in shared memory (while the MMAs run), wait
+    // for the accumulator, drain it in 32-column chunks into packed bf16 registers,
+    // release it to the MMA warp, then store the row (512 bytes per thread).
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
+    const int et = threadIdx.x - 64;  // 0..127
+    float *bias_s = reinterpret_cast<float *>(smem + DATA_BYTES + 256);
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tcount) {
       const int mt = tile % a.Mt;
       const int nt = tile / a.Mt;
+      const int n0 = nt * BN;
+      if (!ADD_Y) {
+        asm volatile("bar.sync 1, 128;" ::: "memory");  // previous tile's bias reads are done
+#pragma unroll
+        for (int e = et; e < BN; e += 128) bias_s[e] = (a.bias && n0 + e < a.N) ? __ldg(a.bias + n0 + e) : 0.0f;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
       if (!mbar_wait(bar_accfull, tcount & 1, a.err, KID_GEMM, 4)) break;
       tc_fence_after();
       const int m = mt * BM + row;
-      for (int c = 0; c < BN / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tbase + (static_cast<uint32_t>(quad * 32) << 16) + c * 32, r);
-        tmem_wait_ld();
-        if (c == BN / 32 - 1) {
-          tc_fence_before();
-          mbar_arrive(bar_accempty);
-        }
-        const int n = nt * BN + c * 32;
-        if (n >= a.N || m >= a.M) continue;
-        uint16_t *yrow = a.Y + static_cast<size_t>(m) * a.N + n;
+      const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16);
+      if constexpr (!ADD_Y) {
+        uint32_t packed[BN / 2];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          if (n + 8 * q >= a.N) break;
-          float v[8];
-          if (ADD_Y) {
+        for (int qc = 0; qc < BN / 16; ++qc) {
+          uint32_t r0[16];
+          tmem_ld16(taddr + qc * 16, r0);
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const int c = qc * 16 + 2 * e;
+            packed[qc * 8 + e] = pack_bf16x2(fmaf(a.alpha, __uint_as_float(r0[2 * e]), bias_s[c]),
+                                             fmaf(a.alpha, __uint_as_float(r0[2 * e + 1]), bias_s[c + 1]));
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(bar_accempty);
+        if (m < a.M) {
+          uint16_t *yrow = a.Y + static_cast<size_t>(m) * a.N + n0;
+#pragma unroll
+          for (int w = 0; w < BN / 8; ++w) {
+            if (n0 + 8 * w >= a.N) break;
+            *reinterpret_cast<uint4 *>(yrow + 8 * w) =
+                make_uint4(packed[4 * w], packed[4 * w + 1], packed[4 * w + 2], packed[4 * w + 3]);
+          }
+        }
+      } else {
+        // Unfused up-projection: Y = bf16(Y + alpha * acc), one 32-column chunk at a time.
+        for (int c = 0; c < BN / 32; ++c) {
+          uint32_t r[32];
+          tmem_ld32(taddr + c * 32, r);
+          tmem_wait_ld();
+          if (c == BN / 32 - 1) {
+            tc_fence_before();
+            mbar_arrive(bar_accempty);
+          }
+          const int n = n0 + c * 32;
+          if (n >= a.N || m >= a.M) continue;
+          uint16_t *yrow = a.Y + static_cast<size_t>(m) * a.N + n;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (n + 8 * q >= a.N) break;
             const uint4 old = *reinterpret_cast<const uint4 *>(yrow + 8 * q);
             const uint32_t w[4] = {old.x, old.y, old.z, old.w};
+            uint32_t o[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              v[2 * e] = fmaf(a.alpha, __uint_as_float(r[8 * q + 2 * e]), bf16_lo(w[e]));
-              v[2 * e + 1] = fmaf(a.alpha, __uint_as_float(r[8 * q + 2 * e + 1]), bf16_hi(w[e]));
-            }
-          } else {
-            float bsv[8];
-            if (a.bias) {
-              const float4 b0 = __ldg(reinterpret_cast<const float4 *>(a.bias + n + 8 * q));
-              const float4 b1 = __ldg(reinterpret_cast<const float4 *>(a.bias + n + 8 * q + 4));
-              bsv[0] = b0.x; bsv[1] = b0.y; bsv[2] = b0.z; bsv[3] = b0.w;
-              bsv[4] = b1.x; bsv[5] = b1.y; bsv[6] = b1.z; bsv[7] = b1.w;
-            } else {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) bsv[e] = 0.0f;
-            }
-#pragma unroll
-            for (int e = 0; e < 8; ++e) v[e] = fmaf(a.alpha, __uint_as_float(r[8 * q + e]), bsv[e]);
+            for (int e = 0; e < 4; ++e)
+              o[e] = pack_bf16x2(fmaf(a.alpha, __uint_as_float(r[8 * q + 2 * e]), bf16_lo(w[e])),
+                                 fmaf(a.alpha, __uint_as_float(r[8 * q + 2 * e + 1]), bf16_hi(w[e])));
+            *reinterpret_cast<uint4 *>(yrow + 8 * q) = make_uint4(o[0], o[1], o[2], o[3]);
           }
-          uint4 o;
-          o.x = pack_bf16x2(v[0], v[1]);
-          o.y = pack_bf16x2(v[2], v[3]);
-          o.z = pack_bf16x2(v[4], v[5]);
-          o.w = pack_bf16x2(v[6], v[7]);
-          *reinterpret_cast<uint4 *>(yrow + 8 * q) = o;
         }
       }
     }

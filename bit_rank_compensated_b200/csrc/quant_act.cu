@@ -53,7 +53,7 @@ struct QArgs {
 };
 
 template <int RANK, bool QUANT>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(320, 2)
     k1_quant_act_lora_down(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
                            QArgs a) {
   using C = QCfg<RANK>;
