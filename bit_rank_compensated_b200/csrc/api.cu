@@ -106,19 +106,18 @@ CUtensorMapSwizzle swizzle_for_row_bytes(uint32_t b) {
 
 float alpha_of(const svdq_layer *L) { return L->x_tensor_scale * L->w_tensor_scale; }
 
-// Number of CTAs along K per 128-row tile for K1 (cluster size): enough CTAs to give every SM
-// two, at most 8 (the portable cluster limit), and every CTA at least one 64-column chunk.
-int pick_splits(int M, int K, int num_sms, int rank) {
+// Number of CTAs along K per 128-row tile for K1 (cluster size): the largest power of two up
+// to 8 (the portable cluster limit) that keeps the whole grid resident in one wave at one CTA
+// per SM, with at least one 64-column chunk per CTA.
+int pick_splits(int M, int K, int num_sms) {
   const int tiles = (M + 127) / 128;
   const int nch = K / 64;
-  int s = 1;
-  while (s < 8 && tiles * s < 2 * num_sms && nch >= 2 * s) s *= 2;
+  int s = 8;
   while (s > 1) {
     const int cps = (nch + s - 1) / s;
-    if ((s - 1) * cps < nch) break;
+    if (tiles * s <= num_sms && (s - 1) * cps < nch) break;
     s /= 2;
   }
-  (void)rank;
   return s;
 }
 
@@ -157,7 +156,7 @@ svdq_status run_quant(const uint16_t *X, int M, const svdq_layer *L, uint8_t *xq
   q.s_x = L->x_tensor_scale;
   q.d_x = 6.0f * L->x_tensor_scale;
   q.inv_alpha = 1.0f / alpha_of(L);
-  q.splits = r > 0 ? pick_splits(M, K, d->num_sms, r) : pick_splits(M, K, d->num_sms, 0);
+  q.splits = pick_splits(M, K, d->num_sms);
   q.chunks_per_split = (K / 64 + q.splits - 1) / q.splits;
   q.quantize = quantize;
   q.lora = lora;

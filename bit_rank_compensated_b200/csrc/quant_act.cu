@@ -4,20 +4,22 @@
 // the quantizer consume the same input, so one kernel serves both.
 //
 // Work decomposition: a CTA owns 128 rows and a contiguous range of 64-column chunks of K.
-// The CTAs that share a row tile form a thread-block cluster along K; their fp32 partial
-// down-projections are summed through distributed shared memory in cluster-rank order, so
-// the result is deterministic and nothing goes through global scratch memory.
+// The CTAs that share a row tile form a thread-block cluster along K (sized so that the grid
+// fits the GPU in one wave); their fp32 partial down-projections are summed through
+// distributed shared memory in cluster-rank order, so the result is deterministic and nothing
+// goes through global scratch memory.
 //
 // The down-projection is stored pre-divided by alpha = s_x s_w as an unevaluated sum of two
 // bf16 values (hi + lo), so the fp32 result reaches K2 without a 16-bit rounding.
 //
-// Warp roles (320 threads):
-//   warp 0      TMA producer: X chunk (128 x 64 bf16, 128B swizzle) and L1t chunk (rank x 64).
-//   warp 1      owns the tensor-memory accumulator (128 lanes x rank fp32 columns) and issues
-//               the bf16 tcgen05 MMAs  acc += bf16(X_hat chunk) * L1 chunk.
-//   warps 2..9  quantizers: thread (row, half) handles 32 elements (two 16-groups) of a chunk:
-//               X_hat = fp32(X * inv_lambda), the group scales and codes, and writes bf16(X_hat)
-//               into the MMA operand tile (same swizzle as the X tile).
+// Warp roles (576 threads):
+//   warp 0       TMA producer: per chunk the X tile (128 x 64 bf16, 128B swizzle), the L1t
+//                tile (rank x 64 bf16, 128B swizzle) and 64 inv_lambda values.
+//   warp 1       owns the tensor-memory accumulator (128 lanes x rank fp32 columns) and issues
+//                the bf16 tcgen05 MMAs  acc += bf16(X_hat chunk) * L1 chunk.
+//   warps 2..17  quantizers: lane l of quantizer warp q handles row 8q + l/4 and the 16-element
+//                group l%4 of the chunk: X_hat = fp32(X * inv_lambda), the group's scale and
+//                codes, and bf16(X_hat) into the MMA operand tile (same swizzle as the X tile).
 #include "common.cuh"
 #include "internal.h"
 #include "nvfp4.cuh"
@@ -27,18 +29,20 @@ namespace {
 
 template <int RANK>
 struct QCfg {
-  static constexpr int STAGES = RANK == 0 ? 4 : 3;
+  static constexpr int STAGES = 4;
+  static constexpr int QWARPS = 16;
+  static constexpr int THREADS = 64 + 32 * QWARPS;
   static constexpr uint32_t X_BYTES = 128u * 128u;
   static constexpr uint32_t OP_BYTES = RANK ? 128u * 128u : 0u;
   static constexpr uint32_t L1_BYTES = RANK * 128u;
-  static constexpr uint32_t STAGE_BYTES = X_BYTES + OP_BYTES + L1_BYTES;
+  static constexpr uint32_t IL_BYTES = 64u * 4u;
+  static constexpr uint32_t STAGE_BYTES = (X_BYTES + OP_BYTES + L1_BYTES + IL_BYTES + 1023u) & ~1023u;
   static constexpr uint32_t RED_BYTES = RANK * 128u * 4u;
   static constexpr uint32_t DATA_BYTES =
       (STAGES * STAGE_BYTES > RED_BYTES) ? STAGES * STAGE_BYTES : RED_BYTES;
   static constexpr uint32_t BAR_BYTES = 256;
   static constexpr uint32_t SMEM = DATA_BYTES + BAR_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = RANK <= 32 ? 32u : static_cast<uint32_t>(RANK);
-  static constexpr int THREADS = 320;
 };
 
 struct QArgs {
@@ -53,7 +57,7 @@ struct QArgs {
 };
 
 template <int RANK, bool QUANT>
-__global__ void __launch_bounds__(320, 2)
+__global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
     k1_quant_act_lora_down(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
                            QArgs a) {
   using C = QCfg<RANK>;
@@ -82,12 +86,13 @@ __global__ void __launch_bounds__(320, 2)
   auto x_tile = [&](int s) { return smem + s * C::STAGE_BYTES; };
   auto op_tile = [&](int s) { return smem + s * C::STAGE_BYTES + C::X_BYTES; };
   auto l1_tile = [&](int s) { return smem + s * C::STAGE_BYTES + C::X_BYTES + C::OP_BYTES; };
+  auto il_tile = [&](int s) { return smem + s * C::STAGE_BYTES + C::X_BYTES + C::OP_BYTES + C::L1_BYTES; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, 8 + (RANK ? 1 : 0));
-      mbar_init(bar_opfull + 8 * s, 8);
+      mbar_init(bar_empty + 8 * s, C::QWARPS + (RANK ? 1 : 0));
+      mbar_init(bar_opfull + 8 * s, C::QWARPS);
     }
     mbar_init(bar_acc, 1);
     fence_mbar_init();
@@ -109,10 +114,11 @@ __global__ void __launch_bounds__(320, 2)
       for (int i = 0; i < n_local; ++i) {
         const int s = i % ST;
         if (i >= ST && !mbar_wait(bar_empty + 8 * s, ((i / ST) - 1) & 1, a.err, KID_QUANT, 1)) break;
-        mbar_arrive_expect_tx(bar_full + 8 * s, C::X_BYTES + C::L1_BYTES);
+        mbar_arrive_expect_tx(bar_full + 8 * s, C::X_BYTES + C::L1_BYTES + C::IL_BYTES);
         const int kx = (c_begin + i) * 64;
         tma_load_2d(smem_u32(x_tile(s)), &tm_x, kx, m0, bar_full + 8 * s);
         if (RANK) tma_load_2d(smem_u32(l1_tile(s)), &tm_l1, kx, 0, bar_full + 8 * s);
+        bulk_load(smem_u32(il_tile(s)), a.inv_lambda + kx, C::IL_BYTES, bar_full + 8 * s);
       }
     }
   } else if (warp == 1) {
@@ -138,58 +144,56 @@ __global__ void __launch_bounds__(320, 2)
     }
   } else {
     // ------------------------------------------------------------ quantizers
-    const int t = threadIdx.x - 64;
-    const int row = t & 127;
-    const int half = t >> 7;
+    const int row = 8 * (warp - 2) + (lane >> 2);
+    const int g = lane & 3;
     const int m = m0 + row;
     const int ng = a.K / 16;
+    const int c0 = (2 * g) ^ (row & 7), c1 = (2 * g + 1) ^ (row & 7);  // swizzled 16-byte chunks
     for (int i = 0; i < n_local; ++i) {
       const int s = i % ST;
       if (!mbar_wait(bar_full + 8 * s, (i / ST) & 1, a.err, KID_QUANT, 4)) break;
       const uint8_t *xt = x_tile(s) + row * 128;
-      uint4 raw[4];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int c = half * 4 + q;
-        raw[q] = *reinterpret_cast<const uint4 *>(xt + ((c ^ (row & 7)) << 4));
-      }
-      const int kbase = (c_begin + i) * 64 + half * 32;
-      float xh[32];
-      const float4 *il4 = reinterpret_cast<const float4 *>(a.inv_lambda + kbase);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 l0 = __ldg(il4 + 2 * q);
-        const float4 l1 = __ldg(il4 + 2 * q + 1);
-        const uint32_t w[4] = {raw[q].x, raw[q].y, raw[q].z, raw[q].w};
-        xh[8 * q + 0] = __fmul_rn(bf16_lo(w[0]), l0.x);
-        xh[8 * q + 1] = __fmul_rn(bf16_hi(w[0]), l0.y);
-        xh[8 * q + 2] = __fmul_rn(bf16_lo(w[1]), l0.z);
-        xh[8 * q + 3] = __fmul_rn(bf16_hi(w[1]), l0.w);
-        xh[8 * q + 4] = __fmul_rn(bf16_lo(w[2]), l1.x);
-        xh[8 * q + 5] = __fmul_rn(bf16_hi(w[2]), l1.y);
-        xh[8 * q + 6] = __fmul_rn(bf16_lo(w[3]), l1.z);
-        xh[8 * q + 7] = __fmul_rn(bf16_hi(w[3]), l1.w);
-      }
+      const uint4 raw0 = *reinterpret_cast<const uint4 *>(xt + (c0 << 4));
+      const uint4 raw1 = *reinterpret_cast<const uint4 *>(xt + (c1 << 4));
+      const float4 *il4 = reinterpret_cast<const float4 *>(il_tile(s) + g * 64);
+      const float4 l0 = il4[0], l1 = il4[1], l2 = il4[2], l3 = il4[3];
+      float xh[16];
+      xh[0] = __fmul_rn(bf16_lo(raw0.x), l0.x);
+      xh[1] = __fmul_rn(bf16_hi(raw0.x), l0.y);
+      xh[2] = __fmul_rn(bf16_lo(raw0.y), l0.z);
+      xh[3] = __fmul_rn(bf16_hi(raw0.y), l0.w);
+      xh[4] = __fmul_rn(bf16_lo(raw0.z), l1.x);
+      xh[5] = __fmul_rn(bf16_hi(raw0.z), l1.y);
+      xh[6] = __fmul_rn(bf16_lo(raw0.w), l1.z);
+      xh[7] = __fmul_rn(bf16_hi(raw0.w), l1.w);
+      xh[8] = __fmul_rn(bf16_lo(raw1.x), l2.x);
+      xh[9] = __fmul_rn(bf16_hi(raw1.x), l2.y);
+      xh[10] = __fmul_rn(bf16_lo(raw1.y), l2.z);
+      xh[11] = __fmul_rn(bf16_hi(raw1.y), l2.w);
+      xh[12] = __fmul_rn(bf16_lo(raw1.z), l3.x);
+      xh[13] = __fmul_rn(bf16_hi(raw1.z), l3.y);
+      xh[14] = __fmul_rn(bf16_lo(raw1.w), l3.z);
+      xh[15] = __fmul_rn(bf16_hi(raw1.w), l3.w);
+      const int kbase = (c_begin + i) * 64 + g * 16;
       if (QUANT) {
-        uint4 codes;
-        const uint32_t sc0 = nvfp4_group16(xh, a.s_x, a.d_x, codes.x, codes.y);
-        const uint32_t sc1 = nvfp4_group16(xh + 16, a.s_x, a.d_x, codes.z, codes.w);
-        if (m < a.M) *reinterpret_cast<uint4 *>(a.xq + static_cast<size_t>(m) * (a.K / 2) + kbase / 2) = codes;
-        *reinterpret_cast<uint16_t *>(a.xs + scale_offset(m, kbase / 16, ng)) =
-            static_cast<uint16_t>(sc0 | (sc1 << 8));
+        uint2 codes;
+        const uint32_t sc = nvfp4_group16(xh, a.s_x, a.d_x, codes.x, codes.y);
+        if (m < a.M) *reinterpret_cast<uint2 *>(a.xq + static_cast<size_t>(m) * (a.K / 2) + kbase / 2) = codes;
+        a.xs[scale_offset(m, kbase / 16, ng)] = static_cast<uint8_t>(sc);
       }
       if (RANK) {
         uint8_t *ot = op_tile(s) + row * 128;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 v;
-          v.x = pack_bf16x2(xh[8 * q + 0], xh[8 * q + 1]);
-          v.y = pack_bf16x2(xh[8 * q + 2], xh[8 * q + 3]);
-          v.z = pack_bf16x2(xh[8 * q + 4], xh[8 * q + 5]);
-          v.w = pack_bf16x2(xh[8 * q + 6], xh[8 * q + 7]);
-          const int c = half * 4 + q;
-          *reinterpret_cast<uint4 *>(ot + ((c ^ (row & 7)) << 4)) = v;
-        }
+        uint4 v0, v1;
+        v0.x = pack_bf16x2(xh[0], xh[1]);
+        v0.y = pack_bf16x2(xh[2], xh[3]);
+        v0.z = pack_bf16x2(xh[4], xh[5]);
+        v0.w = pack_bf16x2(xh[6], xh[7]);
+        v1.x = pack_bf16x2(xh[8], xh[9]);
+        v1.y = pack_bf16x2(xh[10], xh[11]);
+        v1.z = pack_bf16x2(xh[12], xh[13]);
+        v1.w = pack_bf16x2(xh[14], xh[15]);
+        *reinterpret_cast<uint4 *>(ot + (c0 << 4)) = v0;
+        *reinterpret_cast<uint4 *>(ot + (c1 << 4)) = v1;
         fence_proxy_async_smem();
       }
       __syncwarp();
@@ -206,28 +210,28 @@ __global__ void __launch_bounds__(320, 2)
     if (warp >= 2) {
       const int quad = warp & 3;
       const int row = quad * 32 + lane;
-      const bool second = warp >= 6;
-      bool ok = mbar_wait(bar_acc, 0, a.err, KID_QUANT, 5);
+      const int grp = (warp - 2) >> 2;  // 0..3: column group
+      const bool ok = mbar_wait(bar_acc, 0, a.err, KID_QUANT, 5) && n_local > 0;
       tc_fence_after();
-      if (RANK == 16) {
-        if (!second) {
+      const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16);
+      if constexpr (RANK == 16) {
+        if (grp == 0) {
           uint32_t r[16];
-          tmem_ld16(tbase + (static_cast<uint32_t>(quad * 32) << 16), r);
+          tmem_ld16(taddr, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) red[j * 128 + row] = (ok && n_local) ? __uint_as_float(r[j]) : 0.0f;
+          for (int j = 0; j < 16; ++j) red[j * 128 + row] = ok ? __uint_as_float(r[j]) : 0.0f;
         }
       } else {
-        const int cbase = second ? RANK / 2 : 0;
+        constexpr int CPG = RANK / 4;  // columns per group: 8, 16 or 32
+        const int cb = grp * CPG;
+        uint32_t r[CPG];
+        if constexpr (CPG == 8) tmem_ld8(taddr + cb, r);
+        else if constexpr (CPG == 16) tmem_ld16(taddr + cb, r);
+        else tmem_ld32(taddr + cb, r);
+        tmem_wait_ld();
 #pragma unroll
-        for (int c0 = 0; c0 < RANK / 2; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld32(tbase + (static_cast<uint32_t>(quad * 32) << 16) + cbase + c0, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            red[(cbase + c0 + j) * 128 + row] = (ok && n_local) ? __uint_as_float(r[j]) : 0.0f;
-        }
+        for (int j = 0; j < CPG; ++j) red[(cb + j) * 128 + row] = ok ? __uint_as_float(r[j]) : 0.0f;
       }
       tc_fence_before();
     }

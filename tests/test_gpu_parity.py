@@ -194,12 +194,12 @@ def test_unfused_baseline_matches_oracle(lib):
     Y_ref = O.layer_forward(X, layer_o)
     # The unfused branch writes the 4-bit GEMM's output as bf16 and the up-projection reads it
     # back (the extra 16-bit output round trip), so each element carries one more bf16
-    # rounding of the intermediate Y_mid = alpha * (4-bit product) + b: the bound is
-    # 2^-9 (|Y_mid| + |Y|) plus fp32 accumulation noise.
+    # rounding of the intermediate Y_mid = alpha * (4-bit product) + b. With the bf16 unit
+    # roundoff 2^-8 the bound is 2^-8 (|Y_mid| + |Y|) plus fp32 accumulation noise.
     codes, scales, La = O.quant_act_lora_down(X, layer_o)
     Y_mid = O.gemm_w4a4_lora_up(codes, scales, La[:, :0], O.Layer(**{**layer_o.__dict__, "rank": 0}))
     got = bf16_tensor_to_np(Y).reshape(Y_ref.shape)
-    bound = 2.0 ** -9 * (np.abs(Y_mid) + np.abs(Y_ref)) * 1.01 + 1e-4 * np.sqrt(np.mean(Y_ref ** 2))
+    bound = 2.0 ** -8 * (np.abs(Y_mid) + np.abs(Y_ref)) * 1.01 + 1e-4 * np.sqrt(np.mean(Y_ref ** 2))
     assert np.all(np.abs(got - Y_ref) <= bound)
     assert fro_rel(got, Y_ref) <= 5e-3
 
