@@ -106,21 +106,6 @@ CUtensorMapSwizzle swizzle_for_row_bytes(uint32_t b) {
 
 float alpha_of(const svdq_layer *L) { return L->x_tensor_scale * L->w_tensor_scale; }
 
-// Number of CTAs along K per 128-row tile for K1 (cluster size): the largest power of two up
-// to 8 (the portable cluster limit) that keeps the whole grid resident in one wave at one CTA
-// per SM, with at least one 64-column chunk per CTA.
-int pick_splits(int M, int K, int num_sms) {
-  const int tiles = (M + 127) / 128;
-  const int nch = K / 64;
-  int s = 8;
-  while (s > 1) {
-    const int cps = (nch + s - 1) / s;
-    if (tiles * s <= num_sms && (s - 1) * cps < nch) break;
-    s /= 2;
-  }
-  return s;
-}
-
 svdq_status run_quant(const uint16_t *X, int M, const svdq_layer *L, uint8_t *xq, uint8_t *xs, uint16_t *la,
                       bool quantize, bool lora, void *stream) {
   DeviceState *d = nullptr;
@@ -156,7 +141,7 @@ svdq_status run_quant(const uint16_t *X, int M, const svdq_layer *L, uint8_t *xq
   q.s_x = L->x_tensor_scale;
   q.d_x = 6.0f * L->x_tensor_scale;
   q.inv_alpha = 1.0f / alpha_of(L);
-  q.splits = pick_splits(M, K, d->num_sms);
+  q.splits = quant_act_splits(M, K, L->rank, quantize, lora, d->num_sms);
   q.chunks_per_split = (K / 64 + q.splits - 1) / q.splits;
   q.quantize = quantize;
   q.lora = lora;

@@ -25,6 +25,8 @@ struct QuantLaunch {
   cudaStream_t stream;
 };
 cudaError_t launch_quant_act(const QuantLaunch &q);
+// Cluster size (CTAs along K per row tile) for K1 on the current device.
+int quant_act_splits(int M, int K, int rank, bool quantize, bool lora, int num_sms);
 
 // K2 (and the unfused 4-bit GEMM / up-projection baselines).
 struct GemmLaunch {

@@ -6,14 +6,12 @@
 //   code_i = 0 when scale == 0, else e2m1_rn_satfinite(fp32(v_i / fp32(scale * s)))
 // Division means the correctly rounded fp32 quotient.
 //
-// The element quotients are computed as q_i = v_i * rcp(eff) with the hardware's approximate
-// reciprocal (at most 1 ulp off), so |q_i - v_i / eff| < 2^-21.5 |v_i / eff|, and the correctly
-// rounded quotient f_i lies within the same bound. Their e2m1 codes can differ only if an e2m1
-// rounding threshold (0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5) lies between q_i and f_i or equals
-// f_i. Every threshold has at most two leading significand bits set, so it suffices to flag
-// any |q_i| >= 0.2 within 16 ulps (>= 2^-20 relative) of a value whose low 21 significand bits
-// are zero; a flagged group is redone with correctly rounded divisions. Values below 0.2 code
-// as zero either way.
+// Both divisions go through a reciprocal: q = x * r with r = rcp.approx(y) (at most 1 ulp from
+// 1/y) satisfies |q - x/y| < 2^-21.5 |x/y|, and so does the correctly rounded quotient f. The
+// code (e4m3 or e2m1, both monotone in the value) of any number in [q (1 - 2^-20), q (1 + 2^-20)]
+// is therefore the code of f whenever the codes of the two ends agree; when they differ the
+// group is recomputed with correctly rounded divisions (a rare case: the quotient is within
+// 2^-20 of a rounding threshold).
 #pragma once
 
 #include "common.cuh"
@@ -26,11 +24,29 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
-// 1 when |q| may sit within 2^-20 of an e2m1 rounding threshold, else 0.
-__device__ __forceinline__ uint32_t near_e2m1_threshold(float q) {
-  const uint32_t u = __float_as_uint(q) & 0x7FFFFFFFu;
-  return static_cast<uint32_t>(u >= 0x3E4CCCCDu) & static_cast<uint32_t>(((u + 16u) & 0x1FFFFFu) <= 32u);
+// Packed pair of fp32 values in one 64-bit register.
+struct f2 {
+  uint64_t v;
+};
+
+__device__ __forceinline__ f2 mk2(float lo, float hi) {
+  f2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r.v) : "f"(lo), "f"(hi));
+  return r;
 }
+__device__ __forceinline__ void un2(f2 a, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(a.v));
+}
+// Element-wise a * b, each product rounded to nearest (two fp32 multiplies in one instruction).
+__device__ __forceinline__ f2 mul2(f2 a, f2 b) {
+  f2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r.v) : "l"(a.v), "l"(b.v));
+  return r;
+}
+
+// Low and high ends of the bracket around a quotient q: q (1 -/+ 2^-20).
+constexpr float kBracketLo = 1.0f - 9.5367431640625e-07f;  // 1 - 2^-20
+constexpr float kBracketHi = 1.0f + 9.5367431640625e-07f;  // 1 + 2^-20
 
 __device__ __forceinline__ float absmax16(const float *v) {
   float m[8];
@@ -41,12 +57,21 @@ __device__ __forceinline__ float absmax16(const float *v) {
   return fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
 }
 
+// e4m3 code of fp32(amax / d) for amax >= 0, d > 0, with inv_d = rcp.approx(d).
+__device__ __forceinline__ uint32_t scale_code(float amax, float d, float inv_d) {
+  const float q = __fmul_rn(amax, inv_d);
+  uint16_t both;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(both) : "f"(__fmul_rn(q, kBracketHi)), "f"(__fmul_rn(q, kBracketLo)));
+  const uint32_t lo = both & 0xFFu, hi = both >> 8;
+  return lo == hi ? lo : e4m3_code(__fdiv_rn(amax, d));
+}
+
 // Quantizes v[0..15]; writes the 16 codes as two 32-bit words (element i of the group in
 // bits [4(i % 8), 4(i % 8) + 4) of word i / 8) and returns the e4m3 scale code.
-__device__ __forceinline__ uint32_t nvfp4_group16(const float *v, float s, float d, uint32_t &w0,
+__device__ __forceinline__ uint32_t nvfp4_group16(const float *v, float s, float d, float inv_d, uint32_t &w0,
                                                   uint32_t &w1) {
   const float amax = absmax16(v);
-  const uint32_t sc = e4m3_code(__fdiv_rn(amax, d));
+  const uint32_t sc = scale_code(amax, d, inv_d);
   const float sg = e4m3_value(sc);
   if (sg == 0.0f) {
     w0 = 0u;
@@ -55,19 +80,25 @@ __device__ __forceinline__ uint32_t nvfp4_group16(const float *v, float s, float
   }
   const float eff = __fmul_rn(sg, s);
   const float r = rcp_approx(eff);
-  float q[16];
-  uint32_t flag = 0;
+  const f2 r2 = mk2(r, r), blo = mk2(kBracketLo, kBracketLo), bhi = mk2(kBracketHi, kBracketHi);
+  float lo[16], hi[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    q[i] = __fmul_rn(v[i], r);
-    flag |= near_e2m1_threshold(q[i]);
+  for (int i = 0; i < 16; i += 2) {
+    const f2 q = mul2(mk2(v[i], v[i + 1]), r2);
+    un2(mul2(q, blo), lo[i], lo[i + 1]);
+    un2(mul2(q, bhi), hi[i], hi[i + 1]);
   }
-  if (flag) {
+  const uint32_t l0 = e2m1x8(lo), l1 = e2m1x8(lo + 8);
+  const uint32_t h0 = e2m1x8(hi), h1 = e2m1x8(hi + 8);
+  if ((l0 == h0) & (l1 == h1)) {
+    w0 = l0;
+    w1 = l1;
+    return sc;
+  }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(v[i], eff);
-  }
-  w0 = e2m1x8(q);
-  w1 = e2m1x8(q + 8);
+  for (int i = 0; i < 16; ++i) lo[i] = __fdiv_rn(v[i], eff);
+  w0 = e2m1x8(lo);
+  w1 = e2m1x8(lo + 8);
   return sc;
 }
 

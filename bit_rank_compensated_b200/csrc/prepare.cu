@@ -264,7 +264,8 @@ __global__ void k_residual(const float *W, const float *lam, const uint16_t *L1t
 
 // ------------------------------------------------------------------ NVFP4 rows
 // One thread per 16-element group; scales of padding rows are zeroed by the caller.
-__global__ void k_quantize_rows(const float *A, int rows, int K, float s, float d, uint8_t *codes, uint8_t *scales) {
+__global__ void k_quantize_rows(const float *A, int rows, int K, float s, float d, float inv_d, uint8_t *codes,
+                                uint8_t *scales) {
   const int ng = K / 16;
   const size_t gi = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   if (gi >= static_cast<size_t>(rows) * ng) return;
@@ -280,7 +281,7 @@ __global__ void k_quantize_rows(const float *A, int rows, int K, float s, float 
     v[4 * q + 3] = t.w;
   }
   uint2 w;
-  const uint32_t sc = nvfp4_group16(v, s, d, w.x, w.y);
+  const uint32_t sc = nvfp4_group16(v, s, d, inv_d, w.x, w.y);
   *reinterpret_cast<uint2 *>(codes + static_cast<size_t>(row) * (K / 2) + 8 * g) = w;
   scales[scale_offset(row, g, ng)] = static_cast<uint8_t>(sc);
 }
@@ -290,7 +291,7 @@ cudaError_t launch_quantize_rows(const float *A, int rows, int K, float s, uint8
   const float d = 6.0f * s;  // fp32 multiply, round to nearest
   const size_t groups = static_cast<size_t>(rows) * (K / 16);
   const unsigned blocks = static_cast<unsigned>((groups + 255) / 256);
-  k_quantize_rows<<<blocks, 256, 0, st>>>(A, rows, K, s, d, codes, scales);
+  k_quantize_rows<<<blocks, 256, 0, st>>>(A, rows, K, s, d, 1.0f / d, codes, scales);
   return cudaGetLastError();
 }
 

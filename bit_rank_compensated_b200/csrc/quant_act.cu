@@ -51,7 +51,7 @@ struct QArgs {
   uint8_t *xs;
   uint16_t *lora_act;
   int M, K;
-  float s_x, d_x, inv_alpha;
+  float s_x, d_x, inv_d, inv_alpha;
   int chunks_per_split;
   uint32_t *err;
 };
@@ -147,9 +147,11 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
     const int row = 8 * (warp - 2) + (lane >> 2);
     const int g = lane & 3;
     const int m = m0 + row;
-    const int ng = a.K / 16;
     const int c0 = (2 * g) ^ (row & 7), c1 = (2 * g + 1) ^ (row & 7);  // swizzled 16-byte chunks
-    for (int i = 0; i < n_local; ++i) {
+    // per-chunk output addresses advance by 32 code bytes and one 512-byte scale block
+    uint8_t *xq_p = a.xq + static_cast<size_t>(m) * (a.K / 2) + c_begin * 32 + 8 * g;
+    uint8_t *xs_p = a.xs + scale_offset(m, c_begin * 4 + g, a.K / 16);
+    for (int i = 0; i < n_local; ++i, xq_p += 32, xs_p += 512) {
       const int s = i % ST;
       if (!mbar_wait(bar_full + 8 * s, (i / ST) & 1, a.err, KID_QUANT, 4)) break;
       const uint8_t *xt = x_tile(s) + row * 128;
@@ -157,29 +159,18 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
       const uint4 raw1 = *reinterpret_cast<const uint4 *>(xt + (c1 << 4));
       const float4 *il4 = reinterpret_cast<const float4 *>(il_tile(s) + g * 64);
       const float4 l0 = il4[0], l1 = il4[1], l2 = il4[2], l3 = il4[3];
+      const uint32_t w[8] = {raw0.x, raw0.y, raw0.z, raw0.w, raw1.x, raw1.y, raw1.z, raw1.w};
+      const float il[16] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w,
+                            l2.x, l2.y, l2.z, l2.w, l3.x, l3.y, l3.z, l3.w};
       float xh[16];
-      xh[0] = __fmul_rn(bf16_lo(raw0.x), l0.x);
-      xh[1] = __fmul_rn(bf16_hi(raw0.x), l0.y);
-      xh[2] = __fmul_rn(bf16_lo(raw0.y), l0.z);
-      xh[3] = __fmul_rn(bf16_hi(raw0.y), l0.w);
-      xh[4] = __fmul_rn(bf16_lo(raw0.z), l1.x);
-      xh[5] = __fmul_rn(bf16_hi(raw0.z), l1.y);
-      xh[6] = __fmul_rn(bf16_lo(raw0.w), l1.z);
-      xh[7] = __fmul_rn(bf16_hi(raw0.w), l1.w);
-      xh[8] = __fmul_rn(bf16_lo(raw1.x), l2.x);
-      xh[9] = __fmul_rn(bf16_hi(raw1.x), l2.y);
-      xh[10] = __fmul_rn(bf16_lo(raw1.y), l2.z);
-      xh[11] = __fmul_rn(bf16_hi(raw1.y), l2.w);
-      xh[12] = __fmul_rn(bf16_lo(raw1.z), l3.x);
-      xh[13] = __fmul_rn(bf16_hi(raw1.z), l3.y);
-      xh[14] = __fmul_rn(bf16_lo(raw1.w), l3.z);
-      xh[15] = __fmul_rn(bf16_hi(raw1.w), l3.w);
-      const int kbase = (c_begin + i) * 64 + g * 16;
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        un2(mul2(mk2(bf16_lo(w[e]), bf16_hi(w[e])), mk2(il[2 * e], il[2 * e + 1])), xh[2 * e], xh[2 * e + 1]);
       if (QUANT) {
         uint2 codes;
-        const uint32_t sc = nvfp4_group16(xh, a.s_x, a.d_x, codes.x, codes.y);
-        if (m < a.M) *reinterpret_cast<uint2 *>(a.xq + static_cast<size_t>(m) * (a.K / 2) + kbase / 2) = codes;
-        a.xs[scale_offset(m, kbase / 16, ng)] = static_cast<uint8_t>(sc);
+        const uint32_t sc = nvfp4_group16(xh, a.s_x, a.d_x, a.inv_d, codes.x, codes.y);
+        if (m < a.M) *reinterpret_cast<uint2 *>(xq_p) = codes;
+        *xs_p = static_cast<uint8_t>(sc);
       }
       if (RANK) {
         uint8_t *ot = op_tile(s) + row * 128;
@@ -236,11 +227,12 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
       tc_fence_before();
     }
     cluster_sync_all();
-    const int rows_per = 128 / nsplit;
+    const int rows_per = (128 + nsplit - 1) / nsplit;
     const int r0 = split * rows_per;
+    const int r1 = min(128, r0 + rows_per);
     const uint32_t red_addr = smem_u32(red);
     constexpr int PAIRS = RANK / 2;
-    for (int idx = threadIdx.x; idx < rows_per * PAIRS; idx += C::THREADS) {
+    for (int idx = threadIdx.x; idx < (r1 - r0) * PAIRS; idx += C::THREADS) {
       const int row = r0 + idx / PAIRS;
       const int c = 2 * (idx % PAIRS);
       float s0 = 0.0f, s1 = 0.0f;
@@ -270,18 +262,75 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
 }
 
 template <int RANK, bool QUANT>
-cudaError_t launch_t(const QuantLaunch &q) {
-  using C = QCfg<RANK>;
-  auto kern = k1_quant_act_lora_down<RANK, QUANT>;
+cudaError_t set_attrs() {
   static int attr_done[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(k1_quant_act_lora_down<RANK, QUANT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, QCfg<RANK>::SMEM);
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
-  QArgs a{q.inv_lambda, q.xq, q.xs, q.lora_act, q.M, q.K, q.s_x, q.d_x, q.inv_alpha, q.chunks_per_split, q.err};
+  return cudaSuccess;
+}
+
+// Clusters of `splits` CTAs that can be resident at once (one query per device and size).
+template <int RANK, bool QUANT>
+int max_active_clusters(int splits) {
+  static int cache[64][9] = {};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64 || splits < 1 || splits > 8) return 0;
+  if (cache[dev][splits]) return cache[dev][splits];
+  if (set_attrs<RANK, QUANT>() != cudaSuccess) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(splits, 1, 1);
+  cfg.blockDim = dim3(QCfg<RANK>::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = QCfg<RANK>::SMEM;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = splits;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, k1_quant_act_lora_down<RANK, QUANT>, &cfg) != cudaSuccess) n = 0;
+  cache[dev][splits] = n > 0 ? n : -1;
+  return n;
+}
+
+// Cluster size along K: minimises (waves) x (chunks per CTA + 2), the 2 standing for the
+// per-CTA fixed cost (pipeline fill, reduction); every CTA gets at least one chunk.
+template <int RANK, bool QUANT>
+int pick_splits_t(int M, int K) {
+  const int tiles = (M + 127) / 128;
+  const int nch = K / 64;
+  int best = 1;
+  long best_cost = -1;
+  for (int sp = 1; sp <= 8; ++sp) {
+    const int cps = (nch + sp - 1) / sp;
+    if ((sp - 1) * cps >= nch) continue;
+    const int act = RANK ? max_active_clusters<RANK, QUANT>(sp) : 0;
+    long waves = 1;
+    if (act > 0) waves = (tiles + act - 1) / act;
+    const long cost = waves * (cps + 2);
+    if (best_cost < 0 || cost < best_cost) {
+      best_cost = cost;
+      best = sp;
+    }
+  }
+  return best;
+}
+
+template <int RANK, bool QUANT>
+cudaError_t launch_t(const QuantLaunch &q) {
+  using C = QCfg<RANK>;
+  auto kern = k1_quant_act_lora_down<RANK, QUANT>;
+  cudaError_t e0 = set_attrs<RANK, QUANT>();
+  if (e0 != cudaSuccess) return e0;
+  QArgs a{q.inv_lambda, q.xq, q.xs, q.lora_act, q.M, q.K, q.s_x, q.d_x, 1.0f / q.d_x, q.inv_alpha, q.chunks_per_split, q.err};
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(q.splits, (q.M + 127) / 128, 1);
   cfg.blockDim = dim3(C::THREADS, 1, 1);
@@ -298,6 +347,33 @@ cudaError_t launch_t(const QuantLaunch &q) {
 }
 
 }  // namespace
+
+int quant_act_splits(int M, int K, int rank, bool quantize, bool lora, int num_sms) {
+  const int r = lora ? rank : 0;
+  if (r == 0) {
+    // no cross-CTA reduction: enough CTAs for two per SM, at least one chunk each
+    const int tiles = (M + 127) / 128, nch = K / 64;
+    int sp = 1;
+    while (sp < 16 && tiles * sp < 2 * num_sms && nch >= 2 * sp) sp *= 2;
+    return sp;
+  }
+  if (quantize) {
+    switch (r) {
+      case 16: return pick_splits_t<16, true>(M, K);
+      case 32: return pick_splits_t<32, true>(M, K);
+      case 64: return pick_splits_t<64, true>(M, K);
+      case 128: return pick_splits_t<128, true>(M, K);
+    }
+  } else {
+    switch (r) {
+      case 16: return pick_splits_t<16, false>(M, K);
+      case 32: return pick_splits_t<32, false>(M, K);
+      case 64: return pick_splits_t<64, false>(M, K);
+      case 128: return pick_splits_t<128, false>(M, K);
+    }
+  }
+  return 1;
+}
 
 cudaError_t launch_quant_act(const QuantLaunch &q) {
   const int r = q.lora ? q.rank : 0;
