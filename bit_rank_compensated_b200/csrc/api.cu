@@ -178,6 +178,9 @@ svdq_status run_gemm(const uint8_t *xq, const uint8_t *xs, const uint16_t *la, i
         !make_map(&g.tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L2t, r, N, static_cast<uint64_t>(r) * 2, kc, 256, sw))
       return SVDQ_ERR_CUDA;
   }
+  if (!make_map(&g.tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 64, 128,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ERR_CUDA;
   if (!fp4) {
     g.tm_xq = g.tm_la;
     g.tm_wq = g.tm_l2;

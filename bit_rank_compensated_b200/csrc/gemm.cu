@@ -6,19 +6,25 @@
 // written once.
 //
 // Persistent kernel, one CTA per SM, output tiles of 128 x 256 (rows of X x rows of W).
-// Per tile the k-loop is a sequence of pipeline steps through a 4-stage shared-memory ring:
+// Per tile the k-loop is a sequence of pipeline steps through a 3-stage shared-memory ring:
 //   - rank / kc low-rank steps, kc = min(rank, 32): the hi and lo planes of lora_act
 //     (128 x kc bf16 each) and an L2t tile (256 x kc bf16); bf16 tcgen05 MMAs (K = 16 each),
 //     hi and lo against the same L2t tile;
-//   - K / 256 4-bit steps: xq tile (128 rows x 128 bytes), wq tile (256 x 128 bytes), both with
-//     128B swizzle, plus their e4m3 scale blocks (512 bytes per 128 rows x 64 elements), copied
-//     into tensor memory with tcgen05.cp; four kind::mxf4nvf4 MMAs (K = 64 each).
+//   - K / 256 4-bit steps: xq tile (128 rows x 128 bytes) and wq tile (256 x 128 bytes), both
+//     with 128B swizzle; four kind::mxf4nvf4 MMAs (K = 64 each).
 // All steps accumulate into one fp32 accumulator in tensor memory (128 lanes x 256 columns).
 // lora_act arrives pre-divided by alpha = s_x s_w, so the output stage computes
 // Y = bf16(alpha * acc + bias) for every element.
 //
-// Warp roles (192 threads): warp 0 TMA producer; warp 1 tensor-memory owner and MMA issuer;
-// warps 2..5 output stage (warp w reads lanes 32 (w % 4) .. + 31).
+// Scale factors reach tensor memory without the tensor-memory copy unit: four warps (one per
+// 32-lane sub-partition) read each step's 512-byte scale blocks from global memory (L2) and
+// write them with tcgen05.st in the replicated layout the block-scaled MMA reads (lane i of
+// every sub-partition holds rows i, i+32, i+64, i+96 of a block, one 32-bit column each).
+//
+// Warp roles (320 threads): warp 0 TMA producer; warp 1 tensor-memory owner and MMA issuer;
+// warps 2..5 scale-factor writers; warps 6..9 output stage (warp w reaches lanes 32 (w % 4)..).
+// The output stage drains the accumulator into a swizzled bf16 tile in shared memory, releases
+// it to the MMA warp, and writes the tile with TMA stores (which clip the M / N edges).
 #include "common.cuh"
 #include "internal.h"
 
@@ -27,18 +33,19 @@ namespace {
 
 constexpr int BM = 128;
 constexpr int BN = 256;
-constexpr int STAGES = 4;
+constexpr int STAGES = 3;
 constexpr uint32_t A_BYTES = 128u * 128u;
 constexpr uint32_t B_BYTES = 256u * 128u;
-constexpr uint32_t SFA_BYTES = 2048u;
-constexpr uint32_t SFB_BYTES = 4096u;
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SFA_BYTES + SFB_BYTES;  // 55296 = 54 KiB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KiB
 constexpr uint32_t DATA_BYTES = STAGES * STAGE_BYTES;
-constexpr uint32_t SMEM = DATA_BYTES + 256 + BN * 4 + 1024;  // + barriers, bias stage, alignment
+constexpr uint32_t YST_BYTES = BM * BN * 2;          // bf16 output staging (4 boxes of 128 x 64)
+constexpr uint32_t BIAS_BYTES = BN * 4;
+constexpr uint32_t BAR_BYTES = 256;
+constexpr uint32_t SMEM = DATA_BYTES + YST_BYTES + BIAS_BYTES + BAR_BYTES + 1024;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL0 = 256;   // scale columns follow the accumulator
-constexpr uint32_t SF_COLS = 48;    // per stage: 4 k-blocks x (4 SFA + 8 SFB) columns
-constexpr int THREADS = 192;
+constexpr uint32_t SF_COL0 = 256;  // scale columns follow the accumulator
+constexpr uint32_t SF_COLS = 48;   // per stage: 4 k-blocks x (4 SFA + 8 SFB) columns
+constexpr int THREADS = 320;
 
 struct GArgs {
   const uint8_t *xs;
@@ -55,7 +62,7 @@ template <int RANK, bool FP4, bool ADD_Y>
 __global__ void __launch_bounds__(THREADS, 1)
     k2_gemm_w4a4_lora_up(const __grid_constant__ CUtensorMap tm_xq, const __grid_constant__ CUtensorMap tm_wq,
                          const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_l2,
-                         GArgs a) {
+                         const __grid_constant__ CUtensorMap tm_y, GArgs a) {
   // Low-rank steps: kc columns of lora_act (hi and lo planes) and of L2t per step.
   constexpr int KC = RANK == 0 ? 32 : (RANK < 32 ? RANK : 32);
   constexpr int N_LORA = RANK == 0 ? 0 : RANK / KC;
@@ -67,12 +74,15 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DATA_BYTES);
+  uint8_t *ystage = smem + DATA_BYTES;
+  float *bias_s = reinterpret_cast<float *>(smem + DATA_BYTES + YST_BYTES);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DATA_BYTES + YST_BYTES + BIAS_BYTES);
   const uint32_t bar_full = smem_u32(bars);
   const uint32_t bar_empty = bar_full + 8 * STAGES;
-  const uint32_t bar_accfull = bar_empty + 8 * STAGES;
+  const uint32_t bar_sffull = bar_empty + 8 * STAGES;
+  const uint32_t bar_accfull = bar_sffull + 8 * STAGES;
   const uint32_t bar_accempty = bar_accfull + 8;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * STAGES + 2);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -83,13 +93,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   auto a_tile = [&](int s) { return smem + s * STAGE_BYTES; };
   auto b_tile = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES; };
-  auto sfa_tile = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B_BYTES; };
-  auto sfb_tile = [&](int s) { return smem + s * STAGE_BYTES + A_BYTES + B_BYTES + SFA_BYTES; };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
       mbar_init(bar_full + 8 * s, 1);
       mbar_init(bar_empty + 8 * s, 1);
+      mbar_init(bar_sffull + 8 * s, 128);
     }
     mbar_init(bar_accfull, 1);
     mbar_init(bar_accempty, 128);
@@ -134,15 +143,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             tma_load_2d(smem_u32(b_tile(s)), &tm_l2, j * KC, nt * BN, fb);
           } else {
             const int kt = j - N_LORA;
-            const int kbv = min(4, kblocks - 4 * kt);
-            mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES + 3u * 512u * kbv);
+            mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
             tma_load_2d(smem_u32(a_tile(s)), &tm_xq, kt * 128, mt * BM, fb);
             tma_load_2d(smem_u32(b_tile(s)), &tm_wq, kt * 128, nt * BN, fb);
-            bulk_load(smem_u32(sfa_tile(s)), a.xs + (static_cast<size_t>(mt) * kblocks + 4 * kt) * 512, 512u * kbv, fb);
-            bulk_load(smem_u32(sfb_tile(s)), a.ws + (static_cast<size_t>(2 * nt) * kblocks + 4 * kt) * 512,
-                      512u * kbv, fb);
-            bulk_load(smem_u32(sfb_tile(s)) + 2048, a.ws + (static_cast<size_t>(2 * nt + 1) * kblocks + 4 * kt) * 512,
-                      512u * kbv, fb);
           }
         }
       }
@@ -164,12 +167,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         for (int j = 0; j < total; ++j, ++it) {
           const int s = it % STAGES;
-          if (!mbar_wait(bar_full + 8 * s, (it / STAGES) & 1, a.err, KID_GEMM, 3)) {
+          const uint32_t par = (it / STAGES) & 1;
+          if (!mbar_wait(bar_full + 8 * s, par, a.err, KID_GEMM, 3)) {
             ok = false;
             break;
           }
-          tc_fence_after();
           if (j < N_LORA) {
+            tc_fence_after();
             const uint64_t ad = umma_desc(smem_u32(a_tile(s)), 16, 8 * LORA_ROW, LORA_SWZ);
             const uint64_t ald = umma_desc(smem_u32(a_tile(s)) + LORA_LO_OFF, 16, 8 * LORA_ROW, LORA_SWZ);
             const uint64_t bd = umma_desc(smem_u32(b_tile(s)), 16, 8 * LORA_ROW, LORA_SWZ);
@@ -179,16 +183,14 @@ __global__ void __launch_bounds__(THREADS, 1)
               mma_bf16(tbase, ald + 2u * k, bd + 2u * k, idesc_bf16, 1u);
             }
           } else {
+            if (!mbar_wait(bar_sffull + 8 * s, par, a.err, KID_GEMM, 5)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
             const int kt = j - N_LORA;
             const int kbv = min(4, kblocks - 4 * kt);
             const uint32_t tsf = tbase + SF_COL0 + SF_COLS * s;
-            const uint32_t sfa = smem_u32(sfa_tile(s));
-            const uint32_t sfb = smem_u32(sfb_tile(s));
-            for (int kb = 0; kb < kbv; ++kb) {
-              tmem_cp_32x128b_x4(tsf + 4 * kb, umma_desc(sfa + 512 * kb, 0, 128, 0));
-              tmem_cp_32x128b_x4(tsf + 16 + 8 * kb, umma_desc(sfb + 512 * kb, 0, 128, 0));
-              tmem_cp_32x128b_x4(tsf + 16 + 8 * kb + 4, umma_desc(sfb + 2048 + 512 * kb, 0, 128, 0));
-            }
             const uint64_t ad = umma_desc(smem_u32(a_tile(s)), 16, 1024, 2);
             const uint64_t bd = umma_desc(smem_u32(b_tile(s)), 16, 1024, 2);
             for (int kb = 0; kb < kbv; ++kb)
@@ -201,56 +203,105 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_commit(bar_accfull);
       }
     }
+  } else if (warp < 6) {
+    // ------------------------------------------------------------ scale-factor writers
+    // Lane i of the warp for sub-partition q writes TMEM lane 32 q + i: per k-block the 16-byte
+    // line i of the activation block (4 columns) and of the two weight blocks (8 columns).
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
+      const int mt = tile % a.Mt;
+      const int nt = tile / a.Mt;
+      const uint8_t *xs_t = a.xs + static_cast<size_t>(mt) * kblocks * 512 + lane * 16;
+      const uint8_t *ws0 = a.ws + static_cast<size_t>(2 * nt) * kblocks * 512 + lane * 16;
+      const uint8_t *ws1 = ws0 + static_cast<size_t>(kblocks) * 512;
+      for (int j = 0; j < total; ++j, ++it) {
+        const int s = it % STAGES;
+        uint32_t sa[16], sb[32];
+        if (j >= N_LORA) {
+          const int kt = j - N_LORA;
+          const int kbv = min(4, kblocks - 4 * kt);
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            uint4 va = make_uint4(0, 0, 0, 0), v0 = va, v1 = va;
+            if (kb < kbv) {
+              const size_t off = static_cast<size_t>(4 * kt + kb) * 512;
+              va = __ldg(reinterpret_cast<const uint4 *>(xs_t + off));
+              v0 = __ldg(reinterpret_cast<const uint4 *>(ws0 + off));
+              v1 = __ldg(reinterpret_cast<const uint4 *>(ws1 + off));
+            }
+            sa[4 * kb + 0] = va.x; sa[4 * kb + 1] = va.y; sa[4 * kb + 2] = va.z; sa[4 * kb + 3] = va.w;
+            sb[8 * kb + 0] = v0.x; sb[8 * kb + 1] = v0.y; sb[8 * kb + 2] = v0.z; sb[8 * kb + 3] = v0.w;
+            sb[8 * kb + 4] = v1.x; sb[8 * kb + 5] = v1.y; sb[8 * kb + 6] = v1.z; sb[8 * kb + 7] = v1.w;
+          }
+        }
+        if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1, a.err, KID_GEMM, 6)) {
+          ok = false;
+          break;
+        }
+        if (j >= N_LORA) {
+          const uint32_t tsf = tbase + lane_base + SF_COL0 + SF_COLS * s;
+          tmem_st16(tsf, sa);
+          tmem_st32(tsf + 16, sb);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        mbar_arrive(bar_sffull + 8 * s);
+      }
+    }
   } else {
     // ------------------------------------------------------------ output stage
-    // Per tile: stage the tile's 256 bias values in shared memory (while the MMAs run), wait
-    // for the accumulator, drain it in 32-column chunks into packed bf16 registers,
-    // release it to the MMA warp, then store the row (512 bytes per thread).
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const int et = threadIdx.x - 64;  // 0..127
-    float *bias_s = reinterpret_cast<float *>(smem + DATA_BYTES + 256);
+    const int et = threadIdx.x - 192;  // 0..127
     uint32_t tcount = 0;
     for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tcount) {
       const int mt = tile % a.Mt;
       const int nt = tile / a.Mt;
       const int n0 = nt * BN;
-      if (!ADD_Y) {
-        asm volatile("bar.sync 1, 128;" ::: "memory");  // previous tile's bias reads are done
-#pragma unroll
-        for (int e = et; e < BN; e += 128) bias_s[e] = (a.bias && n0 + e < a.N) ? __ldg(a.bias + n0 + e) : 0.0f;
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-      }
-      if (!mbar_wait(bar_accfull, tcount & 1, a.err, KID_GEMM, 4)) break;
-      tc_fence_after();
       const int m = mt * BM + row;
       const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16);
       if constexpr (!ADD_Y) {
-        uint32_t packed[BN / 2];
+        // previous tile: bias reads done (barrier) and its TMA stores finished reading ystage
+        if (et == 0) bulk_wait_read0();
+        named_bar_sync(1, 128);
 #pragma unroll
+        for (int e = et; e < BN; e += 128) bias_s[e] = (a.bias && n0 + e < a.N) ? __ldg(a.bias + n0 + e) : 0.0f;
+        named_bar_sync(1, 128);
+        if (!mbar_wait(bar_accfull, tcount & 1, a.err, KID_GEMM, 4)) break;
+        tc_fence_after();
+        // 4 boxes of 64 columns; row r of a box holds 128 bytes with 16-byte chunk c at c ^ (r % 8)
+#pragma unroll 1
         for (int qc = 0; qc < BN / 16; ++qc) {
-          uint32_t r0[16];
-          tmem_ld16(taddr + qc * 16, r0);
+          uint32_t r[16];
+          tmem_ld16(taddr + qc * 16, r);
           tmem_wait_ld();
+          uint32_t p[8];
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const int c = qc * 16 + 2 * e;
-            packed[qc * 8 + e] = pack_bf16x2(fmaf(a.alpha, __uint_as_float(r0[2 * e]), bias_s[c]),
-                                             fmaf(a.alpha, __uint_as_float(r0[2 * e + 1]), bias_s[c + 1]));
+            p[e] = pack_bf16x2(fmaf(a.alpha, __uint_as_float(r[2 * e]), bias_s[c]),
+                               fmaf(a.alpha, __uint_as_float(r[2 * e + 1]), bias_s[c + 1]));
           }
+          const int box = qc >> 2;           // 64 columns per box
+          const int ch = (qc & 3) * 2;       // first of the two 16-byte chunks of these 16 columns
+          uint8_t *rowp = ystage + box * (BM * 128) + row * 128;
+          *reinterpret_cast<uint4 *>(rowp + (((ch) ^ (row & 7)) << 4)) = make_uint4(p[0], p[1], p[2], p[3]);
+          *reinterpret_cast<uint4 *>(rowp + (((ch + 1) ^ (row & 7)) << 4)) = make_uint4(p[4], p[5], p[6], p[7]);
         }
         tc_fence_before();
         mbar_arrive(bar_accempty);
-        if (m < a.M) {
-          uint16_t *yrow = a.Y + static_cast<size_t>(m) * a.N + n0;
-#pragma unroll
-          for (int w = 0; w < BN / 8; ++w) {
-            if (n0 + 8 * w >= a.N) break;
-            *reinterpret_cast<uint4 *>(yrow + 8 * w) =
-                make_uint4(packed[4 * w], packed[4 * w + 1], packed[4 * w + 2], packed[4 * w + 3]);
-          }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (et == 0) {
+          for (int box = 0; box < BN / 64; ++box)
+            if (n0 + 64 * box < a.N) tma_store_2d(&tm_y, smem_u32(ystage + box * (BM * 128)), n0 + 64 * box, mt * BM);
+          bulk_commit();
         }
       } else {
+        if (!mbar_wait(bar_accfull, tcount & 1, a.err, KID_GEMM, 4)) break;
+        tc_fence_after();
         // Unfused up-projection: Y = bf16(Y + alpha * acc), one 32-column chunk at a time.
         for (int c = 0; c < BN / 32; ++c) {
           uint32_t r[32];
@@ -278,6 +329,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
+    if (!ADD_Y && et == 0) bulk_wait0();  // stores complete before the CTA exits
   }
 
   __syncthreads();
@@ -293,7 +345,7 @@ cudaError_t launch_t(const GemmLaunch &g) {
   static int attr_done[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
-  if (dev < 64 && !attr_done[dev]) {
+  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
@@ -301,7 +353,7 @@ cudaError_t launch_t(const GemmLaunch &g) {
   GArgs a{g.xs, g.ws, g.bias, g.Y, g.M, g.N, g.K, (g.M + BM - 1) / BM, (g.N + BN - 1) / BN, g.alpha, g.err};
   const int tiles = a.Mt * a.Nt;
   const int grid = tiles < g.num_sms ? tiles : g.num_sms;
-  kern<<<grid, THREADS, SMEM, g.stream>>>(g.tm_xq, g.tm_wq, g.tm_la, g.tm_l2, a);
+  kern<<<grid, THREADS, SMEM, g.stream>>>(g.tm_xq, g.tm_wq, g.tm_la, g.tm_l2, g.tm_y, a);
   return cudaGetLastError();
 }
 

@@ -32,8 +32,9 @@ int quant_act_splits(int M, int K, int rank, bool quantize, bool lora, int num_s
 struct GemmLaunch {
   CUtensorMap tm_xq;  // xq, u8 [M, K/2], box 128 x 128, 128B swizzle
   CUtensorMap tm_wq;  // wq, u8 [N, K/2], box 128 x 256, 128B swizzle
-  CUtensorMap tm_la;  // lora_act, bf16 [M, rank], box kc x 128
+  CUtensorMap tm_la;  // lora_act, bf16 [M, 2 rank] (hi | lo planes), box kc x 128
   CUtensorMap tm_l2;  // L2t, bf16 [N, rank], box kc x 256
+  CUtensorMap tm_y;   // Y, bf16 [M, N], box 64 x 128, 128B swizzle (output stores)
   const uint8_t *xs;
   const uint8_t *ws;
   const float *bias;
