@@ -47,8 +47,43 @@ def k1_bytes(M, K, r):
     return 2.0 * M * K + 4.0 * K + 2.0 * K * r + M * K / 2 + M * K / 16 + 2.0 * M * r
 
 
+def aggregate(flops_per_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job TFLOPS: every rank runs `steps` steps of its own replica; the job takes the
+    slowest rank's time (max over ranks)."""
+    return world * flops_per_step * steps / (max_ms * 1e-3) / 1e12
+
+
+def max_over_ranks(value_ms: float, dist, device) -> float:
+    """Max of a per-rank elapsed time over all ranks (identity without a process group)."""
+    if dist is None:
+        return value_ms
+    import torch
+
+    t = torch.tensor([value_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def k2_flops(M, K, N, r):
     return 2.0 * M * N * K + 2.0 * M * N * r
+
+
+def k2_traffic(workload: str):
+    """DRAM bytes per K2 launch from the committed ncu capture, if it was taken on this exact
+    K2 source (the file records the sha1 of gemm.cu) and workload; otherwise None."""
+    import hashlib
+
+    tr_path = os.path.join(ROOT, "profiles", "k2_traffic.json")
+    src = os.path.join(ROOT, "bit_rank_compensated_b200", "csrc", "gemm.cu")
+    if not (os.path.exists(tr_path) and os.path.exists(src)):
+        return None
+    with open(tr_path) as f:
+        tr = json.load(f)
+    with open(src, "rb") as f:
+        sha = hashlib.sha1(f.read()).hexdigest()
+    if tr.get("workload") == workload and tr.get("source_sha1") == sha:
+        return tr.get("bytes_per_launch")
+    return None
 
 
 def read_peaks():
@@ -262,10 +297,7 @@ def main(argv=None):
     k2_ms = [e[1].elapsed_time(e[2]) for e in ev]
     err = svdq.last_device_error()
 
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, dist, dev)
 
     # ---------------- end to end through the host-buffer entry point
     Xh = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -284,31 +316,23 @@ def main(argv=None):
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
+    e2e_ms = max_over_ranks(e2e_ms, dist, dev)
     if dist:
-        t = torch.tensor([e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
         dist.barrier()
         dist.destroy_process_group()
     if rank != 0:
         return 0
 
     flops = layer_flops(M, K, N, r)
-    value = world * flops * args.steps / (total_ms * 1e-3) / 1e12
-    e2e_value = world * flops * e2e_steps / (e2e_ms * 1e-3) / 1e12
+    value = aggregate(flops, args.steps, world, total_ms)
+    e2e_value = aggregate(flops, e2e_steps, world, e2e_ms)
     hbm_gbs, bf16_tf, peak_kind = read_peaks()
     fp4_peak = bf16_tf * FP4_OVER_BF16
     k1_avg = statistics.mean(k1_ms)
     k2_avg = statistics.mean(k2_ms)
     k2_tf = k2_flops(M, K, N, r) / (k2_avg * 1e-3) / 1e12
     k1_gbs = k1_bytes(M, K, r) / (k1_avg * 1e-3) / 1e9
-    traffic = None
-    tr_path = os.path.join(ROOT, "profiles", "k2_traffic.json")
-    if os.path.exists(tr_path):
-        with open(tr_path) as f:
-            tr = json.load(f)
-        if tr.get("workload") == shape.name and tr.get("kernel_rev") == svdq.load().svdq_version():
-            traffic = tr.get("bytes_per_launch")
+    traffic = k2_traffic(shape.name)
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         res = cpu_oracle_sample(shape, 256, budget_s=15.0)
