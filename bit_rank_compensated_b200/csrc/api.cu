@@ -314,6 +314,22 @@ svdq_status svdq_prepare_weights(const float *W, const float *bias, const float 
   return SVDQ_OK;
 }
 
+svdq_status svdq_smoothing_factors_noalloc(const float *W, const float *act_absmax, int N, int K, float *lambda,
+                                           float *inv_lambda, float *x_tensor_scale, void *stream) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  if (!W || !act_absmax || !lambda || !inv_lambda || !x_tensor_scale || N <= 0 || K <= 0 || K % 64 != 0 ||
+      K > noalloc_max_k())
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(act_absmax) || !aligned16(lambda) || !aligned16(inv_lambda))
+    return SVDQ_ERR_MISALIGNED;
+  return smoothing_noalloc(W, act_absmax, N, K, lambda, inv_lambda, x_tensor_scale,
+                           static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SVDQ_OK
+             : SVDQ_ERR_CUDA;
+}
+
 svdq_status svdq_quantize_rows(const float *A, int rows, int K, float s, int row_pad, uint8_t *codes, uint8_t *scales,
                                void *stream) {
   DeviceState *d = nullptr;

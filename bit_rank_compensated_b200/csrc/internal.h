@@ -83,6 +83,11 @@ struct PrepArgs {
 };
 
 PrepStatus prepare_plan(int N, int K, int rank, PrepPlan *plan);
+
+// Smoothing stage with its scratch in a static device array (no allocation); K <= noalloc_max_k().
+int noalloc_max_k();
+cudaError_t smoothing_noalloc(const float *W, const float *act_absmax, int N, int K, float *lambda,
+                              float *inv_lambda, float *x_tensor_scale, cudaStream_t st);
 PrepStatus prepare_run(const PrepArgs &p);
 
 }  // namespace svdq

@@ -295,6 +295,61 @@ cudaError_t launch_quantize_rows(const float *A, int rows, int K, float s, uint8
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ allocation-free smoothing
+// Some callers cannot allocate device memory at the point where they need a layer's smoothing
+// factors (for example code that runs with a fixed, pre-reserved memory budget, or inside a
+// framework that forbids allocation after start-up). This variant of the smoothing stage keeps
+// its scratch (the K column maxima of W and the running maximum behind s_x) in a file-scope
+// device array instead of the caller's workspace. Every GPU that loads the library holds the
+// array until the process exits; all calls share it, so calls that overlap on the GPU race.
+constexpr int kNoAllocMaxK = 65536;
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocMaxK + 64];
+
+// s = fp32(amax / 2688) (6 x 448), 1 when amax is zero.
+__global__ void k_tensor_scale_from_max(const float *amax, float *s_out) {
+  const float m = *amax;
+  *s_out = m > 0.0f ? __fdiv_rn(m, 2688.0f) : 1.0f;
+}
+
+namespace {
+struct NoAllocSlot {
+  std::once_flag once;
+  float *ptr = nullptr;
+  cudaError_t err = cudaSuccess;
+};
+NoAllocSlot g_noalloc_slot[64];
+}  // namespace
+
+int noalloc_max_k() { return kNoAllocMaxK; }
+
+cudaError_t smoothing_noalloc(const float *W, const float *act_absmax, int N, int K, float *lambda,
+                              float *inv_lambda, float *x_tensor_scale, cudaStream_t st) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || K > kNoAllocMaxK) return cudaErrorInvalidValue;
+  NoAllocSlot &slot = g_noalloc_slot[dev];
+  // Once per device, with that device current: the device address of the array (host code
+  // only sees a host-side stand-in for the symbol).
+  std::call_once(slot.once, [&]() {
+    void *p = nullptr;
+    slot.err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    slot.ptr = static_cast<float *>(p);
+  });
+  if (slot.err != cudaSuccess) return slot.err;
+  float *a_w = slot.ptr;                 // K floats (zeroed by launch_col_absmax_f32)
+  float *axh_max = slot.ptr + kNoAllocMaxK;  // one float, zeroed here
+  e = cudaMemsetAsync(axh_max, 0, sizeof(float), st);
+  if (e != cudaSuccess) return e;
+  e = launch_col_absmax_f32(W, N, K, a_w, st);
+  if (e != cudaSuccess) return e;
+  k_smoothing<<<(K + 255) / 256, 256, 0, st>>>(act_absmax, a_w, K, lambda, inv_lambda, axh_max);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_tensor_scale_from_max<<<1, 1, 0, st>>>(axh_max, x_tensor_scale);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ eigen-solver (dlopen)
 namespace {
 using fn_create = cusolverStatus_t (*)(cusolverDnHandle_t *);

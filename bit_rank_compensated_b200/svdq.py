@@ -28,6 +28,7 @@ EXPORTED = (
     "svdq_prepare_workspace_bytes", "svdq_prepare_weights", "svdq_quantize_rows", "svdq_quant_act_lora_down",
     "svdq_gemm_w4a4_lora_up", "svdq_linear_forward", "svdq_linear_forward_host", "svdq_baseline_lora_down",
     "svdq_baseline_quantize", "svdq_baseline_gemm_w4a4", "svdq_baseline_lora_up", "svdq_last_device_error",
+    "svdq_smoothing_factors_noalloc",
 )
 
 
@@ -78,6 +79,7 @@ def load() -> ctypes.CDLL:
         "svdq_baseline_gemm_w4a4": ([P, P, I, LP, P, P], I),
         "svdq_baseline_lora_up": ([P, I, LP, P, P], I),
         "svdq_last_device_error": ([P, ctypes.POINTER(ctypes.c_uint32)], I),
+        "svdq_smoothing_factors_noalloc": ([P, P, I, I, P, P, P, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -193,6 +195,20 @@ def prepare_weights(W: torch.Tensor, bias: torch.Tensor | None, act_absmax_: tor
         _stream(stream)))
     del ws
     return L
+
+
+def smoothing_factors_noalloc(W: torch.Tensor, act_absmax_: torch.Tensor, lam=None, inv_lam=None, s_x=None,
+                              stream=None):
+    """lambda, inv_lambda and the activation tensor scale of a layer, computed without any
+    device allocation inside the library (its scratch is a static device array, K <= 65536).
+    Output tensors may be passed in (the call then allocates nothing at all)."""
+    N, K = W.shape
+    lam = torch.empty(K, dtype=torch.float32, device=W.device) if lam is None else lam
+    inv_lam = torch.empty(K, dtype=torch.float32, device=W.device) if inv_lam is None else inv_lam
+    s_x = torch.empty(1, dtype=torch.float32, device=W.device) if s_x is None else s_x
+    _check("svdq_smoothing_factors_noalloc", load().svdq_smoothing_factors_noalloc(
+        _ptr(W), _ptr(act_absmax_), N, K, _ptr(lam), _ptr(inv_lam), _ptr(s_x), _stream(stream)))
+    return lam, inv_lam, s_x
 
 
 def quantize_rows(A: torch.Tensor, s: float, row_pad: int = 256, stream=None):

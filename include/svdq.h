@@ -198,6 +198,28 @@ SVDQ_API svdq_status svdq_baseline_gemm_w4a4(const uint8_t *xq, const uint8_t *x
 SVDQ_API svdq_status svdq_baseline_lora_up(const uint16_t *lora_act, int M, const svdq_layer *layer,
                                   uint16_t *Y, void *stream);
 
+/* Allocation-free variant of the smoothing stage of svdq_prepare_weights (this entry point has
+ * no counterpart on the method's pages; it exists for callers that cannot allocate device memory
+ * when they need it, e.g. code running under a fixed, pre-reserved memory budget or inside a
+ * framework that forbids allocations after start-up, and so cannot pass a workspace):
+ *   a_w[j] = max_n |W[n, j]|; lambda_j, inv_lambda_j and s_x exactly as svdq_prepare_weights
+ *   computes them (s_x = fp32(max_j fp32(a_x[j] inv_lambda_j) / 2688), 1 when that maximum is 0).
+ *   W                device, N x K fp32.
+ *   act_absmax       device, K fp32 calibration maxima a_x.
+ *   lambda           device, K fp32 (out).
+ *   inv_lambda       device, K fp32 (out).
+ *   x_tensor_scale   device, 1 fp32 (out).
+ * Its scratch (K column maxima and one running maximum) is a static device array inside the
+ * library sized for K <= 65536 (256 KiB, held on every GPU that loads the library until the
+ * process exits); larger K returns SVDQ_ERR_INVALID_ARG. It calls no allocating routine. The
+ * first call on a device looks up the array's device address (once per device), so make that
+ * first call before any stream capture. All calls share the array and the call clears what must
+ * start at zero; calls that overlap on the GPU (other streams, other threads) race on it.
+ * Asynchronous on stream. */
+SVDQ_API svdq_status svdq_smoothing_factors_noalloc(const float *W, const float *act_absmax, int N, int K,
+                                                    float *lambda, float *inv_lambda, float *x_tensor_scale,
+                                                    void *stream);
+
 /* Reads and clears the device-side error word after synchronizing stream. *code is 0 when
  * no kernel gave up on a wait; otherwise (kernel id << 16) | (site << 8) | 1.
  * Returns SVDQ_ERR_TIMEOUT when *code != 0. */
