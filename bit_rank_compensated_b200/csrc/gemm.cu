@@ -207,48 +207,55 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ------------------------------------------------------------ scale-factor writers
     // Lane i of the warp for sub-partition q writes TMEM lane 32 q + i: per k-block the 16-byte
     // line i of the activation block (4 columns) and of the two weight blocks (8 columns).
+    // The loads for step t + 1 are issued before step t is stored (two register sets).
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    uint32_t it = 0;
-    bool ok = true;
-    for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-      const int mt = tile % a.Mt;
-      const int nt = tile / a.Mt;
-      const uint8_t *xs_t = a.xs + static_cast<size_t>(mt) * kblocks * 512 + lane * 16;
-      const uint8_t *ws0 = a.ws + static_cast<size_t>(2 * nt) * kblocks * 512 + lane * 16;
+    const int my_tiles = tiles > static_cast<int>(blockIdx.x) ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int nsteps = my_tiles * total;
+    auto load = [&](int step, uint32_t(&sa)[16], uint32_t(&sb)[32]) {
+      const int j = step % total;
+      if (j < N_LORA) return;
+      const int tile = blockIdx.x + (step / total) * gridDim.x;
+      const int mt = tile % a.Mt, nt = tile / a.Mt;
+      const int kt = j - N_LORA;
+      const int kbv = min(4, kblocks - 4 * kt);
+      const uint8_t *xs_t = a.xs + (static_cast<size_t>(mt) * kblocks + 4 * kt) * 512 + lane * 16;
+      const uint8_t *ws0 = a.ws + (static_cast<size_t>(2 * nt) * kblocks + 4 * kt) * 512 + lane * 16;
       const uint8_t *ws1 = ws0 + static_cast<size_t>(kblocks) * 512;
-      for (int j = 0; j < total; ++j, ++it) {
-        const int s = it % STAGES;
-        uint32_t sa[16], sb[32];
-        if (j >= N_LORA) {
-          const int kt = j - N_LORA;
-          const int kbv = min(4, kblocks - 4 * kt);
 #pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            uint4 va = make_uint4(0, 0, 0, 0), v0 = va, v1 = va;
-            if (kb < kbv) {
-              const size_t off = static_cast<size_t>(4 * kt + kb) * 512;
-              va = __ldg(reinterpret_cast<const uint4 *>(xs_t + off));
-              v0 = __ldg(reinterpret_cast<const uint4 *>(ws0 + off));
-              v1 = __ldg(reinterpret_cast<const uint4 *>(ws1 + off));
-            }
-            sa[4 * kb + 0] = va.x; sa[4 * kb + 1] = va.y; sa[4 * kb + 2] = va.z; sa[4 * kb + 3] = va.w;
-            sb[8 * kb + 0] = v0.x; sb[8 * kb + 1] = v0.y; sb[8 * kb + 2] = v0.z; sb[8 * kb + 3] = v0.w;
-            sb[8 * kb + 4] = v1.x; sb[8 * kb + 5] = v1.y; sb[8 * kb + 6] = v1.z; sb[8 * kb + 7] = v1.w;
-          }
+      for (int kb = 0; kb < 4; ++kb) {
+        uint4 va = make_uint4(0, 0, 0, 0), v0 = va, v1 = va;
+        if (kb < kbv) {
+          va = __ldg(reinterpret_cast<const uint4 *>(xs_t + kb * 512));
+          v0 = __ldg(reinterpret_cast<const uint4 *>(ws0 + kb * 512));
+          v1 = __ldg(reinterpret_cast<const uint4 *>(ws1 + kb * 512));
         }
-        if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1, a.err, KID_GEMM, 6)) {
-          ok = false;
-          break;
-        }
-        if (j >= N_LORA) {
-          const uint32_t tsf = tbase + lane_base + SF_COL0 + SF_COLS * s;
-          tmem_st16(tsf, sa);
-          tmem_st32(tsf + 16, sb);
-          tmem_wait_st();
-        }
-        tc_fence_before();
-        mbar_arrive(bar_sffull + 8 * s);
+        sa[4 * kb + 0] = va.x; sa[4 * kb + 1] = va.y; sa[4 * kb + 2] = va.z; sa[4 * kb + 3] = va.w;
+        sb[8 * kb + 0] = v0.x; sb[8 * kb + 1] = v0.y; sb[8 * kb + 2] = v0.z; sb[8 * kb + 3] = v0.w;
+        sb[8 * kb + 4] = v1.x; sb[8 * kb + 5] = v1.y; sb[8 * kb + 6] = v1.z; sb[8 * kb + 7] = v1.w;
       }
+    };
+    auto put = [&](int step, const uint32_t(&sa)[16], const uint32_t(&sb)[32]) -> bool {
+      const int s = step % STAGES;
+      if (step >= STAGES && !mbar_wait(bar_empty + 8 * s, ((step / STAGES) - 1) & 1, a.err, KID_GEMM, 6))
+        return false;
+      if (step % total >= N_LORA) {
+        const uint32_t tsf = tbase + lane_base + SF_COL0 + SF_COLS * s;
+        tmem_st16(tsf, sa);
+        tmem_st32(tsf + 16, sb);
+        tmem_wait_st();
+      }
+      tc_fence_before();
+      mbar_arrive(bar_sffull + 8 * s);
+      return true;
+    };
+    uint32_t sa0[16], sb0[32], sa1[16], sb1[32];
+    if (nsteps > 0) load(0, sa0, sb0);
+    for (int step = 0; step < nsteps; step += 2) {
+      if (step + 1 < nsteps) load(step + 1, sa1, sb1);
+      if (!put(step, sa0, sb0)) break;
+      if (step + 1 >= nsteps) break;
+      if (step + 2 < nsteps) load(step + 2, sa0, sb0);
+      if (!put(step + 1, sa1, sb1)) break;
     }
   } else {
     // ------------------------------------------------------------ output stage
@@ -273,22 +280,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         tc_fence_after();
         // 4 boxes of 64 columns; row r of a box holds 128 bytes with 16-byte chunk c at c ^ (r % 8)
 #pragma unroll 1
-        for (int qc = 0; qc < BN / 16; ++qc) {
-          uint32_t r[16];
-          tmem_ld16(taddr + qc * 16, r);
+        for (int box = 0; box < BN / 64; ++box) {
+          uint32_t r[64];
+          tmem_ld32(taddr + box * 64, *reinterpret_cast<uint32_t(*)[32]>(r));
+          tmem_ld32(taddr + box * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
           tmem_wait_ld();
-          uint32_t p[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const int c = qc * 16 + 2 * e;
-            p[e] = pack_bf16x2(fmaf(a.alpha, __uint_as_float(r[2 * e]), bias_s[c]),
-                               fmaf(a.alpha, __uint_as_float(r[2 * e + 1]), bias_s[c + 1]));
-          }
-          const int box = qc >> 2;           // 64 columns per box
-          const int ch = (qc & 3) * 2;       // first of the two 16-byte chunks of these 16 columns
           uint8_t *rowp = ystage + box * (BM * 128) + row * 128;
-          *reinterpret_cast<uint4 *>(rowp + (((ch) ^ (row & 7)) << 4)) = make_uint4(p[0], p[1], p[2], p[3]);
-          *reinterpret_cast<uint4 *>(rowp + (((ch + 1) ^ (row & 7)) << 4)) = make_uint4(p[4], p[5], p[6], p[7]);
+#pragma unroll
+          for (int ch = 0; ch < 8; ++ch) {  // 16-byte chunk ch = columns 8 ch .. 8 ch + 7 of the box
+            uint32_t p[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = box * 64 + ch * 8 + 2 * e;
+              p[e] = pack_bf16x2(fmaf(a.alpha, __uint_as_float(r[ch * 8 + 2 * e]), bias_s[c]),
+                                 fmaf(a.alpha, __uint_as_float(r[ch * 8 + 2 * e + 1]), bias_s[c + 1]));
+            }
+            *reinterpret_cast<uint4 *>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(p[0], p[1], p[2], p[3]);
+          }
         }
         tc_fence_before();
         mbar_arrive(bar_accempty);
