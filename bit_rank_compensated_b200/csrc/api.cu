@@ -168,14 +168,14 @@ svdq_status run_gemm(const uint8_t *xq, const uint8_t *xs, const uint16_t *la, i
   const int K = L->K, N = L->N;
   if (fp4) {
     if (!make_map(&g.tm_xq, CU_TENSOR_MAP_DATA_TYPE_UINT8, xq, K / 2, M, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_map(&g.tm_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wq, K / 2, N, K / 2, 128, 256, CU_TENSOR_MAP_SWIZZLE_128B))
+        !make_map(&g.tm_wq, CU_TENSOR_MAP_DATA_TYPE_UINT8, L->wq, K / 2, N, K / 2, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B))
       return SVDQ_ERR_CUDA;
   }
   if (r > 0) {
     const uint32_t kc = r < 32 ? r : 32;
     const CUtensorMapSwizzle sw = swizzle_for_row_bytes(kc * 2);
     if (!make_map(&g.tm_la, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, la, 2 * r, M, static_cast<uint64_t>(r) * 4, kc, 128, sw) ||
-        !make_map(&g.tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L2t, r, N, static_cast<uint64_t>(r) * 2, kc, 256, sw))
+        !make_map(&g.tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L2t, r, N, static_cast<uint64_t>(r) * 2, kc, 128, sw))
       return SVDQ_ERR_CUDA;
   }
   if (!make_map(&g.tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 64, 128,

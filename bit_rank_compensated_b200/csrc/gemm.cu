@@ -5,47 +5,85 @@
 // the 4-bit GEMM produce the same output, so one kernel serves both and the 16-bit output is
 // written once.
 //
-// Persistent kernel, one CTA per SM, output tiles of 128 x 256 (rows of X x rows of W).
-// Per tile the k-loop is a sequence of pipeline steps through a 3-stage shared-memory ring:
-//   - rank / kc low-rank steps, kc = min(rank, 32): the hi and lo planes of lora_act
-//     (128 x kc bf16 each) and an L2t tile (256 x kc bf16); bf16 tcgen05 MMAs (K = 16 each),
+// Persistent kernel of CTA pairs (clusters of two CTAs on two SMs). A pair owns an output tile
+// of 256 x 256 (rows of X x rows of W) and computes it with cta_group::2 tensor-core MMAs of
+// M = 256, N = 256: each CTA stages its own 128 rows of the activation tile and its own 128
+// rows of the weight tile, the even CTA of the pair issues the MMAs for both, and each CTA's
+// tensor memory holds the accumulator of its 128 rows (all 256 columns). Per SM and per 4-bit
+// step this stages 32 KiB of operands for 512 tensor-core cycles; a one-CTA tile of 128 x 256
+// needs 48 KiB.
+//
+// Per tile the k-loop is a sequence of pipeline steps through a 5-stage shared-memory ring:
+//   - rank / kc low-rank steps, kc = min(rank, 32): per CTA the hi and lo planes of lora_act
+//     (128 x kc bf16 each) and half of an L2t tile (128 x kc bf16); bf16 MMAs (K = 16 each),
 //     hi and lo against the same L2t tile;
-//   - K / 256 4-bit steps: xq tile (128 rows x 128 bytes) and wq tile (256 x 128 bytes), both
-//     with 128B swizzle; four kind::mxf4nvf4 MMAs (K = 64 each).
-// All steps accumulate into one fp32 accumulator in tensor memory (128 lanes x 256 columns).
-// lora_act arrives pre-divided by alpha = s_x s_w, so the output stage computes
-// Y = bf16(alpha * acc + bias) for every element.
+//   - K / 256 4-bit steps: per CTA 128 rows of xq and 128 rows of wq (128 bytes each, 128B
+//     swizzle); four kind::mxf4nvf4 MMAs (K = 64 each).
+// All steps accumulate into one fp32 accumulator. lora_act arrives pre-divided by
+// alpha = s_x s_w, so the output stage computes Y = bf16(alpha * acc + bias) for every element.
 //
-// Scale factors reach tensor memory without the tensor-memory copy unit: four warps (one per
-// 32-lane sub-partition) read each step's 512-byte scale blocks from global memory (L2) and
-// write them with tcgen05.st in the replicated layout the block-scaled MMA reads (lane i of
-// every sub-partition holds rows i, i+32, i+64, i+96 of a block, one 32-bit column each).
+// Scale factors reach tensor memory through registers: tcgen05.st moves them several times
+// faster than the tensor-memory copy unit, which has to replicate every 512-byte block four
+// times. Eight warps per CTA, two per 32-lane sub-partition, each own two of a step's four
+// k-blocks: they load the 16-byte lines of the step's scale blocks from global memory (L2) two
+// steps ahead and write them with tcgen05.st in the replicated layout the block-scaled MMA reads
+// (lane i of every sub-partition holds rows i, i+32, i+64, i+96 of a block, one 32-bit column
+// each). A CTA holds the activation scales of its own 128 rows and the weight scales of all 256
+// rows of the tile, since its half of the MMA multiplies its rows by the whole of B.
 //
-// Warp roles (320 threads): warp 0 TMA producer; warp 1 tensor-memory owner and MMA issuer;
-// warps 2..5 scale-factor writers; warps 6..9 output stage (warp w reaches lanes 32 (w % 4)..).
-// The output stage drains the accumulator into a swizzled bf16 tile in shared memory, releases
-// it to the MMA warp, and writes the tile with TMA stores (which clip the M / N edges).
+// Warp roles (576 threads per CTA): warp 0 TMA producer; warp 1 tensor-memory owner and, in the
+// even CTA, MMA issuer; warps 2..9 scale-factor writers;
+// warps 10..17 output stage (warp w reaches lanes 32 (w % 4).. and drains columns
+// 128 ((w - 10) / 4)..). The output stage drains the
+// accumulator into a swizzled bf16 tile in shared memory, releases the accumulator, and writes
+// the tile with TMA stores (which clip the M / N edges).
+//
+// Synchronisation across the pair. Every barrier the MMA issuer waits on lives in the even CTA,
+// and it waits on one per step and one per tile: each barrier result the issuing thread consumes
+// costs the tensor pipe a bubble of about 200 cycles, because the MMA queue is short. The full
+// barrier of a stage counts the even CTA producer's arrival (which expects the bytes of both
+// CTAs' loads; the odd CTA's loads signal it across the pair) and one arrival per scale-writer
+// warp of either CTA; accempty counts one arrival per output warp of either CTA. The MMA
+// issuer's commits arrive on the empty and accfull barriers of both CTAs. Every wait is bounded:
+// a thread whose wait gives up records the error and either leaves its loop or, where it shares
+// named barriers, keeps stepping through them without touching tensor memory.
 #include "common.cuh"
 #include "internal.h"
 
 namespace svdq {
 namespace {
 
-constexpr int BM = 128;
-constexpr int BN = 256;
-constexpr int STAGES = 3;
-constexpr uint32_t A_BYTES = 128u * 128u;
-constexpr uint32_t B_BYTES = 256u * 128u;
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;  // 48 KiB
+constexpr int BM = 128;      // rows of X per CTA
+constexpr int BMP = 2 * BM;  // rows of X per pair tile
+constexpr int BN = 256;      // rows of W per pair tile
+constexpr int BNH = BN / 2;  // rows of W staged per CTA
+constexpr int STAGES = 5;
+constexpr uint32_t A_BYTES = BM * 128u;
+constexpr uint32_t B_BYTES = BNH * 128u;
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KiB
+constexpr uint32_t SF_BLOCK = 512;                   // scale bytes of 128 rows x 64 elements of K
 constexpr uint32_t DATA_BYTES = STAGES * STAGE_BYTES;
-constexpr uint32_t YST_BYTES = BM * BN * 2;          // bf16 output staging (4 boxes of 128 x 64)
+constexpr uint32_t YST_BYTES = BM * BN * 2;  // bf16 output staging: 4 boxes of 128 rows x 64 columns
 constexpr uint32_t BIAS_BYTES = BN * 4;
 constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM = DATA_BYTES + YST_BYTES + BIAS_BYTES + BAR_BYTES + 1024;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t SF_COL0 = 256;  // scale columns follow the accumulator
-constexpr uint32_t SF_COLS = 48;   // per stage: 4 k-blocks x (4 SFA + 8 SFB) columns
-constexpr int THREADS = 320;
+constexpr uint32_t SF_COL0 = 256;  // one scale slot per stage follows the accumulator
+constexpr uint32_t SF_COLS = 48;   // per slot: 4 k-blocks x (4 SFA + 8 SFB) columns
+constexpr int SF_WARP0 = 2;
+constexpr int EPI_WARP0 = 10;
+constexpr int THREADS = 576;
+// Arrivals the MMA issuer waits for, besides the producer's: one per scale-writer warp and one
+// per output warp, from both CTAs of the pair.
+constexpr uint32_t SF_WARPS = 8;
+constexpr uint32_t EPI_WARPS = 8;
+constexpr uint32_t FULL_COUNT = 1 + 2 * SF_WARPS;
+constexpr uint32_t ACCEMPTY_COUNT = 2 * EPI_WARPS;
+constexpr int N_BARS = 2 * STAGES + 2;
+static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1 KiB alignment of 128B-swizzled tiles");
+static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "scale slots exceed the tensor memory");
+static_assert(SMEM <= 232448, "shared memory per CTA");
+static_assert(N_BARS * 8 + 4 <= BAR_BYTES, "barrier area");
 
 struct GArgs {
   const uint8_t *xs;
@@ -53,7 +91,7 @@ struct GArgs {
   const float *bias;
   uint16_t *Y;
   int M, N, K;
-  int Mt, Nt;
+  int Mt, Nt;  // pair tiles along M (256 rows) and N (256 rows of W)
   float alpha;
   uint32_t *err;
 };
@@ -68,27 +106,35 @@ __global__ void __launch_bounds__(THREADS, 1)
   constexpr int N_LORA = RANK == 0 ? 0 : RANK / KC;
   constexpr uint32_t LORA_ROW = KC * 2;  // bytes per row of a low-rank tile
   constexpr uint32_t LORA_SWZ = LORA_ROW == 64 ? 4u : 6u;
-  constexpr uint32_t LORA_A_BYTES = 128u * LORA_ROW;
-  constexpr uint32_t LORA_B_BYTES = 256u * LORA_ROW;
+  constexpr uint32_t LORA_A_BYTES = BM * LORA_ROW;
+  constexpr uint32_t LORA_B_BYTES = BNH * LORA_ROW;
   constexpr uint32_t LORA_LO_OFF = 8192u;  // lo plane inside the A slot
+  static_assert(LORA_A_BYTES <= LORA_LO_OFF && LORA_LO_OFF + LORA_A_BYTES <= A_BYTES, "low-rank A slot");
+  static_assert(LORA_B_BYTES <= B_BYTES, "low-rank B slot");
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *ystage = smem + DATA_BYTES;
-  float *bias_s = reinterpret_cast<float *>(smem + DATA_BYTES + YST_BYTES);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + DATA_BYTES + YST_BYTES + BIAS_BYTES);
+  float *bias_s = reinterpret_cast<float *>(ystage + YST_BYTES);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ystage + YST_BYTES + BIAS_BYTES);
+  // full[s] (used in the even CTA): stage s is loaded in both CTAs and both CTAs' scales for it
+  // are in tensor memory; empty[s]: the MMAs reading stage s are done (both CTAs); accfull: the
+  // accumulator is complete (both CTAs); accempty (used in the even CTA): both CTAs' output
+  // stages have read it.
   const uint32_t bar_full = smem_u32(bars);
   const uint32_t bar_empty = bar_full + 8 * STAGES;
-  const uint32_t bar_sffull = bar_empty + 8 * STAGES;
-  const uint32_t bar_accfull = bar_sffull + 8 * STAGES;
+  const uint32_t bar_accfull = bar_empty + 8 * STAGES;
   const uint32_t bar_accempty = bar_accfull + 8;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 3 * STAGES + 2);
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + N_BARS);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t crank = cluster_ctarank();  // 0: issues the pair's MMAs; 1: its peer
+  const int pid = blockIdx.x >> 1;           // pair (cluster) index
+  const int npairs = gridDim.x >> 1;
   const int kblocks = a.K / 64;
   const int n_kt = FP4 ? (kblocks + 3) / 4 : 0;
-  const int total = N_LORA + n_kt;
+  const int total = N_LORA + n_kt;  // steps per tile
   const int tiles = a.Mt * a.Nt;
 
   auto a_tile = [&](int s) { return smem + s * STAGE_BYTES; };
@@ -96,25 +142,24 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < STAGES; ++s) {
-      mbar_init(bar_full + 8 * s, 1);
+      mbar_init(bar_full + 8 * s, FULL_COUNT);
       mbar_init(bar_empty + 8 * s, 1);
-      mbar_init(bar_sffull + 8 * s, 128);
     }
     mbar_init(bar_accfull, 1);
-    mbar_init(bar_accempty, 128);
+    mbar_init(bar_accempty, ACCEMPTY_COUNT);
     fence_mbar_init();
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(tmem_holder), TMEM_COLS);
-    tmem_relinquish();
+    tmem_alloc_pair(smem_u32(tmem_holder), TMEM_COLS);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  cluster_sync_all();  // both CTAs' barriers initialised and the pair's tensor memory allocated
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------------------ producer (both CTAs)
     if (lane == 0) {
       if (FP4) {
         tma_prefetch_desc(&tm_xq);
@@ -126,9 +171,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       uint32_t it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x) {
-        const int mt = tile % a.Mt;
-        const int nt = tile / a.Mt;
+      for (int t = pid; t < tiles && ok; t += npairs) {
+        const int mt = t % a.Mt;
+        const int nt = t / a.Mt;
+        const int row0 = mt * BMP + static_cast<int>(crank) * BM;  // this CTA's rows of X
+        const int wrow0 = nt * BN + static_cast<int>(crank) * BNH;  // this CTA's rows of W
         for (int j = 0; j < total; ++j, ++it) {
           const int s = it % STAGES;
           if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1, a.err, KID_GEMM, 1)) {
@@ -136,34 +183,43 @@ __global__ void __launch_bounds__(THREADS, 1)
             break;
           }
           const uint32_t fb = bar_full + 8 * s;
+          const uint32_t fb_lead = map_shared_rank(fb, 0);
+          const uint32_t at = smem_u32(a_tile(s));
+          const uint32_t bt = smem_u32(b_tile(s));
           if (j < N_LORA) {
-            mbar_arrive_expect_tx(fb, 2 * LORA_A_BYTES + LORA_B_BYTES);
-            tma_load_2d(smem_u32(a_tile(s)), &tm_la, j * KC, mt * BM, fb);
-            tma_load_2d(smem_u32(a_tile(s)) + LORA_LO_OFF, &tm_la, RANK + j * KC, mt * BM, fb);
-            tma_load_2d(smem_u32(b_tile(s)), &tm_l2, j * KC, nt * BN, fb);
+            if (crank == 0) mbar_arrive_expect_tx(fb, 2 * (2 * LORA_A_BYTES + LORA_B_BYTES));
+            tma_load_2d_pair(at, &tm_la, j * KC, row0, fb_lead);
+            tma_load_2d_pair(at + LORA_LO_OFF, &tm_la, RANK + j * KC, row0, fb_lead);
+            tma_load_2d_pair(bt, &tm_l2, j * KC, wrow0, fb_lead);
           } else {
             const int kt = j - N_LORA;
-            mbar_arrive_expect_tx(fb, A_BYTES + B_BYTES);
-            tma_load_2d(smem_u32(a_tile(s)), &tm_xq, kt * 128, mt * BM, fb);
-            tma_load_2d(smem_u32(b_tile(s)), &tm_wq, kt * 128, nt * BN, fb);
+            if (crank == 0) mbar_arrive_expect_tx(fb, 2 * STAGE_BYTES);
+            tma_load_2d_pair(at, &tm_xq, kt * 128, row0, fb_lead);
+            tma_load_2d_pair(bt, &tm_wq, kt * 128, wrow0, fb_lead);
           }
         }
       }
+      // The MMA issuer's last commits to this CTA's empty barriers have landed before it exits.
+      for (uint32_t i = it > STAGES ? it - STAGES : 0; ok && i < it; ++i)
+        ok = mbar_wait(bar_empty + 8 * (i % STAGES), (i / STAGES) & 1, a.err, KID_GEMM, 7);
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // ------------------------------------------------------------ MMA issuer (even CTA)
+    if (crank == 0 && lane == 0) {
       // kind::mxf4nvf4: A, B e2m1 (bits 7-9, 10-12 = 1), K-major, N = 256 (bits 17-22),
-      // scale type ue4m3 (bit 23 = 0), M = 128 (bits 24-28), scale ids 0, K = 64.
-      const uint32_t idesc_fp4 = (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BM) >> 4) << 24);
-      // kind::f16: D fp32, A, B bf16, N = 256, M = 128.
+      // scale type ue4m3 (bit 23 = 0), M = 256 across the pair (bits 24-28), scale ids 0, K = 64.
+      const uint32_t idesc_fp4 = (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BMP) >> 4) << 24);
+      // kind::f16: D fp32, A, B bf16, N = 256, M = 256 across the pair.
       const uint32_t idesc_bf16 =
-          (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BM) >> 4) << 24);
+          (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BMP) >> 4) << 24);
       uint32_t it = 0;
       uint32_t tcount = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < tiles && ok; tile += gridDim.x, ++tcount) {
-        if (tcount > 0 && !mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 2)) break;
+      for (int t = pid; t < tiles && ok; t += npairs, ++tcount) {
+        if (tcount > 0 && !mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 2)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         for (int j = 0; j < total; ++j, ++it) {
           const int s = it % STAGES;
@@ -172,154 +228,199 @@ __global__ void __launch_bounds__(THREADS, 1)
             ok = false;
             break;
           }
+          tc_fence_after();
+          const uint32_t st = smem_u32(a_tile(s));
           if (j < N_LORA) {
-            tc_fence_after();
-            const uint64_t ad = umma_desc(smem_u32(a_tile(s)), 16, 8 * LORA_ROW, LORA_SWZ);
-            const uint64_t ald = umma_desc(smem_u32(a_tile(s)) + LORA_LO_OFF, 16, 8 * LORA_ROW, LORA_SWZ);
-            const uint64_t bd = umma_desc(smem_u32(b_tile(s)), 16, 8 * LORA_ROW, LORA_SWZ);
+            const uint64_t ad = umma_desc(st, 16, 8 * LORA_ROW, LORA_SWZ);
+            const uint64_t ald = umma_desc(st + LORA_LO_OFF, 16, 8 * LORA_ROW, LORA_SWZ);
+            const uint64_t bd = umma_desc(st + A_BYTES, 16, 8 * LORA_ROW, LORA_SWZ);
 #pragma unroll
             for (int k = 0; k < KC / 16; ++k) {
-              mma_bf16(tbase, ad + 2u * k, bd + 2u * k, idesc_bf16, (j | k) != 0 ? 1u : 0u);
-              mma_bf16(tbase, ald + 2u * k, bd + 2u * k, idesc_bf16, 1u);
+              mma_bf16_pair(tbase, ad + 2u * k, bd + 2u * k, idesc_bf16, (j | k) != 0 ? 1u : 0u);
+              mma_bf16_pair(tbase, ald + 2u * k, bd + 2u * k, idesc_bf16, 1u);
             }
           } else {
-            if (!mbar_wait(bar_sffull + 8 * s, par, a.err, KID_GEMM, 5)) {
-              ok = false;
-              break;
-            }
-            tc_fence_after();
             const int kt = j - N_LORA;
             const int kbv = min(4, kblocks - 4 * kt);
             const uint32_t tsf = tbase + SF_COL0 + SF_COLS * s;
-            const uint64_t ad = umma_desc(smem_u32(a_tile(s)), 16, 1024, 2);
-            const uint64_t bd = umma_desc(smem_u32(b_tile(s)), 16, 1024, 2);
+            const uint64_t ad = umma_desc(st, 16, 1024, 2);
+            const uint64_t bd = umma_desc(st + A_BYTES, 16, 1024, 2);
             for (int kb = 0; kb < kbv; ++kb)
-              mma_nvfp4(tbase, ad + 2u * kb, bd + 2u * kb, idesc_fp4, tsf + 4 * kb, tsf + 16 + 8 * kb,
-                        (j | kb) != 0 ? 1u : 0u);
+              mma_nvfp4_pair(tbase, ad + 2u * kb, bd + 2u * kb, idesc_fp4, tsf + 4 * kb, tsf + 16 + 8 * kb,
+                             (j | kb) != 0 ? 1u : 0u);
           }
-          tc_commit(bar_empty + 8 * s);
+          tc_commit_pair_mc(bar_empty + 8 * s, 0x3);
         }
         if (!ok) break;
-        tc_commit(bar_accfull);
+        tc_commit_pair_mc(bar_accfull, 0x3);
       }
+      // both CTAs' output stages have released the last accumulator
+      if (ok && tcount > 0) mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 8);
     }
-  } else if (warp < 6) {
+  } else if (warp < EPI_WARP0) {
     // ------------------------------------------------------------ scale-factor writers
-    // Lane i of the warp for sub-partition q writes TMEM lane 32 q + i: per k-block the 16-byte
-    // line i of the activation block (4 columns) and of the two weight blocks (8 columns).
-    // The loads for step t + 1 are issued before step t is stored (two register sets).
+    // Warp (q, h) writes tensor-memory lanes 32 q .. 32 q + 31 for k-blocks 2 h and 2 h + 1 of
+    // every step: lane i stores the 16-byte line i of the CTA's activation block (4 columns) and
+    // of the tile's two weight blocks (8 columns) of each k-block. Loads run two steps ahead.
+    // Every step (low-rank ones too) is announced on the even CTA's full barrier, once per warp.
+    const int h = (warp - SF_WARP0) >> 2;
+    const uint32_t full_lead = map_shared_rank(bar_full, 0);
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int my_tiles = tiles > static_cast<int>(blockIdx.x) ? (tiles - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int my_tiles = tiles > pid ? (tiles - 1 - pid) / npairs + 1 : 0;
     const int nsteps = my_tiles * total;
-    auto load = [&](int step, uint32_t(&sa)[16], uint32_t(&sb)[32]) {
+    struct Lines {
+      uint32_t sa[8];   // activation words of k-blocks 2h, 2h + 1
+      uint32_t sb[16];  // weight words: k-block 2h rows 0-127, 128-255, then k-block 2h + 1
+    };
+    auto load = [&](int step, Lines &b) {
+      if (step >= nsteps) return;
       const int j = step % total;
-      if (j < N_LORA) return;
-      const int tile = blockIdx.x + (step / total) * gridDim.x;
-      const int mt = tile % a.Mt, nt = tile / a.Mt;
+      if (!FP4 || j < N_LORA) return;
+      const int t = pid + (step / total) * npairs;
+      const int mt = t % a.Mt, nt = t / a.Mt;
       const int kt = j - N_LORA;
       const int kbv = min(4, kblocks - 4 * kt);
-      const uint8_t *xs_t = a.xs + (static_cast<size_t>(mt) * kblocks + 4 * kt) * 512 + lane * 16;
-      const uint8_t *ws0 = a.ws + (static_cast<size_t>(2 * nt) * kblocks + 4 * kt) * 512 + lane * 16;
-      const uint8_t *ws1 = ws0 + static_cast<size_t>(kblocks) * 512;
+      const int mb = 2 * mt + static_cast<int>(crank);  // this CTA's 128-row block of X
+      const bool rows_ok = mb * BM < a.M;               // activation scales cover ceil(M / 128) blocks
 #pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
+      for (int e = 0; e < 2; ++e) {
+        const int kb = 2 * h + e;
         uint4 va = make_uint4(0, 0, 0, 0), v0 = va, v1 = va;
         if (kb < kbv) {
-          va = __ldg(reinterpret_cast<const uint4 *>(xs_t + kb * 512));
-          v0 = __ldg(reinterpret_cast<const uint4 *>(ws0 + kb * 512));
-          v1 = __ldg(reinterpret_cast<const uint4 *>(ws1 + kb * 512));
+          const size_t k0 = static_cast<size_t>(4 * kt + kb) * SF_BLOCK + lane * 16;
+          if (rows_ok) va = __ldg(reinterpret_cast<const uint4 *>(a.xs + static_cast<size_t>(mb) * kblocks * SF_BLOCK + k0));
+          v0 = __ldg(reinterpret_cast<const uint4 *>(a.ws + static_cast<size_t>(2 * nt) * kblocks * SF_BLOCK + k0));
+          v1 = __ldg(reinterpret_cast<const uint4 *>(a.ws + static_cast<size_t>(2 * nt + 1) * kblocks * SF_BLOCK + k0));
         }
-        sa[4 * kb + 0] = va.x; sa[4 * kb + 1] = va.y; sa[4 * kb + 2] = va.z; sa[4 * kb + 3] = va.w;
-        sb[8 * kb + 0] = v0.x; sb[8 * kb + 1] = v0.y; sb[8 * kb + 2] = v0.z; sb[8 * kb + 3] = v0.w;
-        sb[8 * kb + 4] = v1.x; sb[8 * kb + 5] = v1.y; sb[8 * kb + 6] = v1.z; sb[8 * kb + 7] = v1.w;
+        b.sa[4 * e + 0] = va.x; b.sa[4 * e + 1] = va.y; b.sa[4 * e + 2] = va.z; b.sa[4 * e + 3] = va.w;
+        b.sb[8 * e + 0] = v0.x; b.sb[8 * e + 1] = v0.y; b.sb[8 * e + 2] = v0.z; b.sb[8 * e + 3] = v0.w;
+        b.sb[8 * e + 4] = v1.x; b.sb[8 * e + 5] = v1.y; b.sb[8 * e + 6] = v1.z; b.sb[8 * e + 7] = v1.w;
       }
     };
-    auto put = [&](int step, const uint32_t(&sa)[16], const uint32_t(&sb)[32]) -> bool {
+    auto put = [&](int step, const Lines &b) -> bool {
       const int s = step % STAGES;
-      if (step >= STAGES && !mbar_wait(bar_empty + 8 * s, ((step / STAGES) - 1) & 1, a.err, KID_GEMM, 6))
-        return false;
-      if (step % total >= N_LORA) {
+      bool ok = true;
+      if (step >= STAGES) ok = mbar_wait(bar_empty + 8 * s, ((step / STAGES) - 1) & 1, a.err, KID_GEMM, 6);
+      if (!__all_sync(0xffffffffu, ok)) return false;
+      if (FP4 && step % total >= N_LORA) {
+        // slot columns: SFA k-block kb at 4 kb, SFB k-block kb at 16 + 8 kb (rows 0-127, then 128-255)
         const uint32_t tsf = tbase + lane_base + SF_COL0 + SF_COLS * s;
-        tmem_st16(tsf, sa);
-        tmem_st32(tsf + 16, sb);
+        tmem_st8(tsf + 8 * h, b.sa);
+        tmem_st16(tsf + 16 + 16 * h, b.sb);
         tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(bar_sffull + 8 * s);
+      __syncwarp();
+      if (lane == 0) mbar_arrive_remote(full_lead + 8 * s);
       return true;
     };
-    uint32_t sa0[16], sb0[32], sa1[16], sb1[32];
-    if (nsteps > 0) load(0, sa0, sb0);
-    for (int step = 0; step < nsteps; step += 2) {
-      if (step + 1 < nsteps) load(step + 1, sa1, sb1);
-      if (!put(step, sa0, sb0)) break;
-      if (step + 1 >= nsteps) break;
-      if (step + 2 < nsteps) load(step + 2, sa0, sb0);
-      if (!put(step + 1, sa1, sb1)) break;
+    Lines b0, b1, b2;
+    load(0, b0);
+    load(1, b1);
+    for (int step = 0; step < nsteps; step += 3) {
+      load(step + 2, b2);
+      if (!put(step, b0) || step + 1 >= nsteps) break;
+      load(step + 3, b0);
+      if (!put(step + 1, b1) || step + 2 >= nsteps) break;
+      load(step + 4, b1);
+      if (!put(step + 2, b2)) break;
     }
   } else {
     // ------------------------------------------------------------ output stage
+    // Two groups of four warps (named barriers 1 and 2), one per 128-column half of the tile;
+    // the warps of a group cover the four 32-lane sub-partitions. Thread (row, half) drains
+    // columns 128 half .. 128 half + 127 of its row in four 32-column chunks, the load of chunk
+    // c + 1 in flight while chunk c is converted.
+    const int half = (warp - EPI_WARP0) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const int et = threadIdx.x - 192;  // 0..127
+    const int et = (static_cast<int>(threadIdx.x) - EPI_WARP0 * 32) & 127;  // thread index in the group
+    const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16) + half * 128;
+    const uint32_t accempty_lead = map_shared_rank(bar_accempty, 0);
+    bool ok = true;
     uint32_t tcount = 0;
-    for (int tile = blockIdx.x; tile < tiles; tile += gridDim.x, ++tcount) {
-      const int mt = tile % a.Mt;
-      const int nt = tile / a.Mt;
+    for (int t = pid; t < tiles; t += npairs, ++tcount) {
+      const int mt = t % a.Mt;
+      const int nt = t / a.Mt;
       const int n0 = nt * BN;
-      const int m = mt * BM + row;
-      const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16);
+      const int row0 = mt * BMP + static_cast<int>(crank) * BM;
+      const int m = row0 + row;
       if constexpr (!ADD_Y) {
-        // previous tile: bias reads done (barrier) and its TMA stores finished reading ystage
+        // the group's previous TMA stores have finished reading the staging tile, and its
+        // threads are done with the previous bias values
         if (et == 0) bulk_wait_read0();
-        named_bar_sync(1, 128);
+        {
+          const int e = half * 128 + et;
+          bias_s[e] = (a.bias && n0 + e < a.N) ? __ldg(a.bias + n0 + e) : 0.0f;
+        }
+        named_bar_sync(1 + half, 128);
+        if (ok) ok = mbar_wait(bar_accfull, tcount & 1, a.err, KID_GEMM, 4);
+        ok = __all_sync(0xffffffffu, ok);
+        if (ok) {
+          tc_fence_after();
+          uint32_t r0[32], r1[32];
+          tmem_ld32(taddr, r0);
+          tmem_wait_ld_dep(r0);
 #pragma unroll
-        for (int e = et; e < BN; e += 128) bias_s[e] = (a.bias && n0 + e < a.N) ? __ldg(a.bias + n0 + e) : 0.0f;
-        named_bar_sync(1, 128);
-        if (!mbar_wait(bar_accfull, tcount & 1, a.err, KID_GEMM, 4)) break;
-        tc_fence_after();
-        // 4 boxes of 64 columns; row r of a box holds 128 bytes with 16-byte chunk c at c ^ (r % 8)
-#pragma unroll 1
-        for (int box = 0; box < BN / 64; ++box) {
-          uint32_t r[64];
-          tmem_ld32(taddr + box * 64, *reinterpret_cast<uint32_t(*)[32]>(r));
-          tmem_ld32(taddr + box * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(r + 32));
-          tmem_wait_ld();
-          uint8_t *rowp = ystage + box * (BM * 128) + row * 128;
-#pragma unroll
-          for (int ch = 0; ch < 8; ++ch) {  // 16-byte chunk ch = columns 8 ch .. 8 ch + 7 of the box
-            uint32_t p[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = box * 64 + ch * 8 + 2 * e;
-              p[e] = pack_bf16x2(fmaf(a.alpha, __uint_as_float(r[ch * 8 + 2 * e]), bias_s[c]),
-                                 fmaf(a.alpha, __uint_as_float(r[ch * 8 + 2 * e + 1]), bias_s[c + 1]));
+          for (int c = 0; c < 4; ++c) {
+            uint32_t(&cur)[32] = (c & 1) ? r1 : r0;
+            uint32_t(&nxt)[32] = (c & 1) ? r0 : r1;
+            if (c + 1 < 4) {
+              tmem_ld32(taddr + (c + 1) * 32, nxt);
+            } else {
+              // every column of this warp's rows has been read: release the accumulator
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive_remote(accempty_lead);
             }
-            *reinterpret_cast<uint4 *>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(p[0], p[1], p[2], p[3]);
+            // box (col0 / 64) holds 128 rows of 128 bytes, 16-byte chunk k of row r at k ^ (r % 8)
+            const int col0 = half * 128 + c * 32;
+            uint8_t *rowp = ystage + (col0 >> 6) * (BM * 128) + row * 128;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const int ch = ((col0 & 63) >> 3) + q;
+              const float4 b0 = *reinterpret_cast<const float4 *>(bias_s + col0 + 8 * q);
+              const float4 b1 = *reinterpret_cast<const float4 *>(bias_s + col0 + 8 * q + 4);
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(cur[8 * q + e]);
+              const uint32_t p0 = pack_bf16x2(fmaf(a.alpha, v[0], b0.x), fmaf(a.alpha, v[1], b0.y));
+              const uint32_t p1 = pack_bf16x2(fmaf(a.alpha, v[2], b0.z), fmaf(a.alpha, v[3], b0.w));
+              const uint32_t p2 = pack_bf16x2(fmaf(a.alpha, v[4], b1.x), fmaf(a.alpha, v[5], b1.y));
+              const uint32_t p3 = pack_bf16x2(fmaf(a.alpha, v[6], b1.z), fmaf(a.alpha, v[7], b1.w));
+              *reinterpret_cast<uint4 *>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(p0, p1, p2, p3);
+            }
+            if (c + 1 < 4) tmem_wait_ld_dep(nxt);
           }
         }
-        tc_fence_before();
-        mbar_arrive(bar_accempty);
         fence_proxy_async_smem();
-        named_bar_sync(1, 128);
+        named_bar_sync(1 + half, 128);
         if (et == 0) {
-          for (int box = 0; box < BN / 64; ++box)
-            if (n0 + 64 * box < a.N) tma_store_2d(&tm_y, smem_u32(ystage + box * (BM * 128)), n0 + 64 * box, mt * BM);
+          if (row0 < a.M) {
+            for (int b = 0; b < 2; ++b) {
+              const int box = half * 2 + b;
+              if (n0 + 64 * box < a.N)
+                tma_store_2d(&tm_y, smem_u32(ystage + box * (BM * 128)), n0 + 64 * box, row0);
+            }
+          }
           bulk_commit();
         }
       } else {
-        if (!mbar_wait(bar_accfull, tcount & 1, a.err, KID_GEMM, 4)) break;
-        tc_fence_after();
         // Unfused up-projection: Y = bf16(Y + alpha * acc), one 32-column chunk at a time.
-        for (int c = 0; c < BN / 32; ++c) {
+        if (ok) ok = mbar_wait(bar_accfull, tcount & 1, a.err, KID_GEMM, 4);
+        ok = __all_sync(0xffffffffu, ok);
+        if (!ok) break;
+        tc_fence_after();
+        for (int c = 0; c < 4; ++c) {
           uint32_t r[32];
           tmem_ld32(taddr + c * 32, r);
-          tmem_wait_ld();
-          if (c == BN / 32 - 1) {
+          tmem_wait_ld_dep(r);
+          if (c == 3) {
             tc_fence_before();
-            mbar_arrive(bar_accempty);
+            __syncwarp();
+            if (lane == 0) mbar_arrive_remote(accempty_lead);
           }
-          const int n = n0 + c * 32;
+          const int n = n0 + half * 128 + c * 32;
           if (n >= a.N || m >= a.M) continue;
           uint16_t *yrow = a.Y + static_cast<size_t>(m) * a.N + n;
 #pragma unroll
@@ -341,28 +442,74 @@ __global__ void __launch_bounds__(THREADS, 1)
   }
 
   __syncthreads();
+  tc_fence_before();
+  cluster_sync_all();  // neither CTA frees the pair's tensor memory while the other still uses it
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tbase, TMEM_COLS);
+    tmem_dealloc_pair(tbase, TMEM_COLS);
   }
+}
+
+// Pairs that can be resident at once (clusters of two, one CTA per SM), per device.
+template <int RANK, bool FP4, bool ADD_Y>
+int pair_slots(cudaError_t *err) {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev < 0 || dev >= 64) {
+    *err = cudaErrorInvalidDevice;
+    return 0;
+  }
+  if (cache[dev] > 0) return cache[dev];
+  auto kern = k2_gemm_w4a4_lora_up<RANK, FP4, ADD_Y>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  if (e != cudaSuccess) {
+    *err = e;
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+  if (e != cudaSuccess || n <= 0) {
+    *err = e != cudaSuccess ? e : cudaErrorLaunchOutOfResources;
+    return 0;
+  }
+  cache[dev] = n;
+  return n;
 }
 
 template <int RANK, bool FP4, bool ADD_Y>
 cudaError_t launch_t(const GemmLaunch &g) {
-  auto kern = k2_gemm_w4a4_lora_up<RANK, FP4, ADD_Y>;
-  static int attr_done[64] = {0};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
-    if (e != cudaSuccess) return e;
-    attr_done[dev] = 1;
-  }
-  GArgs a{g.xs, g.ws, g.bias, g.Y, g.M, g.N, g.K, (g.M + BM - 1) / BM, (g.N + BN - 1) / BN, g.alpha, g.err};
+  cudaError_t e = cudaSuccess;
+  const int slots = pair_slots<RANK, FP4, ADD_Y>(&e);
+  if (slots <= 0) return e;
+  GArgs a{g.xs, g.ws, g.bias, g.Y, g.M, g.N, g.K, (g.M + BMP - 1) / BMP, (g.N + BN - 1) / BN, g.alpha, g.err};
   const int tiles = a.Mt * a.Nt;
-  const int grid = tiles < g.num_sms ? tiles : g.num_sms;
-  kern<<<grid, THREADS, SMEM, g.stream>>>(g.tm_xq, g.tm_wq, g.tm_la, g.tm_l2, g.tm_y, a);
-  return cudaGetLastError();
+  const int pairs = tiles < slots ? tiles : slots;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * pairs, 1, 1);
+  cfg.blockDim = dim3(THREADS, 1, 1);
+  cfg.dynamicSmemBytes = SMEM;
+  cfg.stream = g.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, k2_gemm_w4a4_lora_up<RANK, FP4, ADD_Y>, g.tm_xq, g.tm_wq, g.tm_la, g.tm_l2,
+                            g.tm_y, a);
 }
 
 }  // namespace
@@ -386,5 +533,6 @@ cudaError_t launch_gemm(const GemmLaunch &g) {
   }
   return cudaErrorInvalidValue;
 }
+
 
 }  // namespace svdq

@@ -31,12 +31,12 @@ int quant_act_splits(int M, int K, int rank, bool quantize, bool lora, int num_s
 // K2 (and the unfused 4-bit GEMM / up-projection baselines).
 struct GemmLaunch {
   CUtensorMap tm_xq;  // xq, u8 [M, K/2], box 128 x 128, 128B swizzle
-  CUtensorMap tm_wq;  // wq, u8 [N, K/2], box 128 x 256, 128B swizzle
+  CUtensorMap tm_wq;  // wq, u8 [N, K/2], box 128 x 128 (half a pair tile), 128B swizzle
   CUtensorMap tm_la;  // lora_act, bf16 [M, 2 rank] (hi | lo planes), box kc x 128
-  CUtensorMap tm_l2;  // L2t, bf16 [N, rank], box kc x 256
+  CUtensorMap tm_l2;  // L2t, bf16 [N, rank], box kc x 128 (half a pair tile)
   CUtensorMap tm_y;   // Y, bf16 [M, N], box 64 x 128, 128B swizzle (output stores)
-  const uint8_t *xs;
-  const uint8_t *ws;
+  const uint8_t *xs;  // activation scales (block layout, ceil(M / 128) row blocks)
+  const uint8_t *ws;  // weight scales (block layout, rows padded to 256)
   const float *bias;
   uint16_t *Y;
   int M, N, K, rank;

@@ -65,7 +65,7 @@ def _e2m1_vals(c):
     return O.e2m1_decode(c)
 
 
-@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (200, 272, 576), (1, 16, 64)])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (200, 272, 576), (1, 16, 64), (520, 320, 320)])
 def test_k2_exact_on_power_of_two_scales(lib, M, N, K):
     # With power-of-two group scales, alpha = 1 and no bias every partial sum is exact in
     # fp32, so Y must equal bf16(exact dot product) bit for bit. Pins the operand and
