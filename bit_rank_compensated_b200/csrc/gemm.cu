@@ -178,7 +178,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int wrow0 = nt * BN + static_cast<int>(crank) * BNH;  // this CTA's rows of W
         for (int j = 0; j < total; ++j, ++it) {
           const int s = it % STAGES;
-          if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1, a.err, KID_GEMM, 1)) {
+          if (it >= STAGES && !mbar_wait_parked(bar_empty + 8 * s, ((it / STAGES) - 1) & 1, a.err, KID_GEMM, 1)) {
             ok = false;
             break;
           }
@@ -300,7 +300,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto put = [&](int step, const Lines &b) -> bool {
       const int s = step % STAGES;
       bool ok = true;
-      if (step >= STAGES) ok = mbar_wait(bar_empty + 8 * s, ((step / STAGES) - 1) & 1, a.err, KID_GEMM, 6);
+      if (step >= STAGES) ok = mbar_wait_parked(bar_empty + 8 * s, ((step / STAGES) - 1) & 1, a.err, KID_GEMM, 6);
       if (!__all_sync(0xffffffffu, ok)) return false;
       if (FP4 && step % total >= N_LORA) {
         // slot columns: SFA k-block kb at 4 kb, SFB k-block kb at 16 + 8 kb (rows 0-127, then 128-255)
@@ -354,7 +354,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           bias_s[e] = (a.bias && n0 + e < a.N) ? __ldg(a.bias + n0 + e) : 0.0f;
         }
         named_bar_sync(1 + half, 128);
-        if (ok) ok = mbar_wait(bar_accfull, tcount & 1, a.err, KID_GEMM, 4);
+        if (ok) ok = mbar_wait_parked(bar_accfull, tcount & 1, a.err, KID_GEMM, 4);
         ok = __all_sync(0xffffffffu, ok);
         if (ok) {
           tc_fence_after();
@@ -407,7 +407,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       } else {
         // Unfused up-projection: Y = bf16(Y + alpha * acc), one 32-column chunk at a time.
-        if (ok) ok = mbar_wait(bar_accfull, tcount & 1, a.err, KID_GEMM, 4);
+        if (ok) ok = mbar_wait_parked(bar_accfull, tcount & 1, a.err, KID_GEMM, 4);
         ok = __all_sync(0xffffffffu, ok);
         if (!ok) break;
         tc_fence_after();
