@@ -37,7 +37,9 @@ struct QCfg {
   static constexpr uint32_t L1_BYTES = RANK * 128u;
   static constexpr uint32_t IL_BYTES = 64u * 4u;
   static constexpr uint32_t STAGE_BYTES = (X_BYTES + OP_BYTES + L1_BYTES + IL_BYTES + 1023u) & ~1023u;
-  static constexpr uint32_t RED_BYTES = RANK * 128u * 4u;
+  // split-K partials: 128 rows of RANK fp32, row stride RANK + 4 (16-byte accesses spread over banks)
+  static constexpr uint32_t RED_STRIDE = RANK + 4;
+  static constexpr uint32_t RED_BYTES = RED_STRIDE * 128u * 4u;
   static constexpr uint32_t DATA_BYTES =
       (STAGES * STAGE_BYTES > RED_BYTES) ? STAGES * STAGE_BYTES : RED_BYTES;
   static constexpr uint32_t BAR_BYTES = 256;
@@ -197,7 +199,8 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
 
   if constexpr (RANK > 0) {
     // ------------------------------------------------------------ split-K reduction
-    float *red = reinterpret_cast<float *>(smem);  // [RANK][128] fp32, aliases the stages
+    float *red = reinterpret_cast<float *>(smem);  // [128][RED_STRIDE] fp32, aliases the stages
+    constexpr uint32_t RS = C::RED_STRIDE;
     if (warp >= 2) {
       const int quad = warp & 3;
       const int row = quad * 32 + lane;
@@ -205,13 +208,18 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
       const bool ok = mbar_wait(bar_acc, 0, a.err, KID_QUANT, 5) && n_local > 0;
       tc_fence_after();
       const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16);
+      float *dst = red + row * RS;
       if constexpr (RANK == 16) {
         if (grp == 0) {
           uint32_t r[16];
           tmem_ld16(taddr, r);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j) red[j * 128 + row] = ok ? __uint_as_float(r[j]) : 0.0f;
+          for (int j = 0; j < 16; j += 4)
+            *reinterpret_cast<float4 *>(dst + j) =
+                ok ? make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                 __uint_as_float(r[j + 3]))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
         }
       } else {
         constexpr int CPG = RANK / 4;  // columns per group: 8, 16 or 32
@@ -222,33 +230,44 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
         else tmem_ld32(taddr + cb, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < CPG; ++j) red[(cb + j) * 128 + row] = ok ? __uint_as_float(r[j]) : 0.0f;
+        for (int j = 0; j < CPG; j += 4)
+          *reinterpret_cast<float4 *>(dst + cb + j) =
+              ok ? make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                               __uint_as_float(r[j + 3]))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       tc_fence_before();
     }
     cluster_sync_all();
+    // Rows r0 .. r1 - 1 of the tile: sum the partials of all CTAs of the cluster in rank order,
+    // four columns per thread.
     const int rows_per = (128 + nsplit - 1) / nsplit;
     const int r0 = split * rows_per;
     const int r1 = min(128, r0 + rows_per);
     const uint32_t red_addr = smem_u32(red);
-    constexpr int PAIRS = RANK / 2;
-    for (int idx = threadIdx.x; idx < (r1 - r0) * PAIRS; idx += C::THREADS) {
-      const int row = r0 + idx / PAIRS;
-      const int c = 2 * (idx % PAIRS);
-      float s0 = 0.0f, s1 = 0.0f;
+    constexpr int QUADS = RANK / 4;
+    for (int idx = threadIdx.x; idx < (r1 - r0) * QUADS; idx += C::THREADS) {
+      const int row = r0 + idx / QUADS;
+      const int c = 4 * (idx % QUADS);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
       for (int src = 0; src < nsplit; ++src) {
-        s0 += ld_shared_cluster_f32(map_shared_rank(red_addr + (c * 128 + row) * 4, src));
-        s1 += ld_shared_cluster_f32(map_shared_rank(red_addr + ((c + 1) * 128 + row) * 4, src));
+        const float4 v = ld_shared_cluster_f32x4(map_shared_rank(red_addr + (row * RS + c) * 4, src));
+        acc.x += v.x;
+        acc.y += v.y;
+        acc.z += v.z;
+        acc.w += v.w;
       }
       if (m0 + row < a.M) {
         // lora_act row = [hi(0..RANK-1) | lo(0..RANK-1)], v ~ hi + lo with hi = bf16(v),
         // lo = bf16(v - hi): the pair carries ~16 significant bits of the fp32 value.
-        const float v0 = __fmul_rn(s0, a.inv_alpha), v1 = __fmul_rn(s1, a.inv_alpha);
-        const uint32_t hi = pack_bf16x2(v0, v1);
-        const uint32_t lo = pack_bf16x2(__fsub_rn(v0, bf16_lo(hi)), __fsub_rn(v1, bf16_hi(hi)));
-        uint16_t *dst = a.lora_act + static_cast<size_t>(m0 + row) * (2 * RANK) + c;
-        *reinterpret_cast<uint32_t *>(dst) = hi;
-        *reinterpret_cast<uint32_t *>(dst + RANK) = lo;
+        const float v0 = __fmul_rn(acc.x, a.inv_alpha), v1 = __fmul_rn(acc.y, a.inv_alpha);
+        const float v2 = __fmul_rn(acc.z, a.inv_alpha), v3 = __fmul_rn(acc.w, a.inv_alpha);
+        const uint32_t h01 = pack_bf16x2(v0, v1), h23 = pack_bf16x2(v2, v3);
+        const uint32_t l01 = pack_bf16x2(__fsub_rn(v0, bf16_lo(h01)), __fsub_rn(v1, bf16_hi(h01)));
+        const uint32_t l23 = pack_bf16x2(__fsub_rn(v2, bf16_lo(h23)), __fsub_rn(v3, bf16_hi(h23)));
+        uint16_t *out = a.lora_act + static_cast<size_t>(m0 + row) * (2 * RANK) + c;
+        *reinterpret_cast<uint2 *>(out) = make_uint2(h01, h23);
+        *reinterpret_cast<uint2 *>(out + RANK) = make_uint2(l01, l23);
       }
     }
     cluster_sync_all();
