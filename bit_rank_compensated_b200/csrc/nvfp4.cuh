@@ -66,20 +66,23 @@ __device__ __forceinline__ uint32_t scale_code(float amax, float d, float inv_d)
   return lo == hi ? lo : e4m3_code(__fdiv_rn(amax, d));
 }
 
-// Quantizes v[0..15]; writes the 16 codes as two 32-bit words (element i of the group in
-// bits [4(i % 8), 4(i % 8) + 4) of word i / 8) and returns the e4m3 scale code.
-__device__ __forceinline__ uint32_t nvfp4_group16(const float *v, float s, float d, float inv_d, uint32_t &w0,
-                                                  uint32_t &w1) {
+// Quantizes v[0..15] in two phases so that callers can interleave several groups: the first
+// phase has no branches; the second, needed only when the first reports `exact` (the bracket
+// ends disagree for some element, which is rare), recomputes the codes with correctly rounded
+// divisions. Codes: element i of the group in bits [4(i % 8), 4(i % 8) + 4) of word i / 8.
+struct Group16 {
+  uint32_t w0, w1, sc;
+  float eff;    // sg * s
+  bool exact;   // the codes must be recomputed by nvfp4_group16_exact
+};
+
+__device__ __forceinline__ Group16 nvfp4_group16_fast(const float *v, float s, float d, float inv_d) {
+  Group16 g;
   const float amax = absmax16(v);
-  const uint32_t sc = scale_code(amax, d, inv_d);
-  const float sg = e4m3_value(sc);
-  if (sg == 0.0f) {
-    w0 = 0u;
-    w1 = 0u;
-    return sc;
-  }
-  const float eff = __fmul_rn(sg, s);
-  const float r = rcp_approx(eff);
+  g.sc = scale_code(amax, d, inv_d);
+  const float sg = e4m3_value(g.sc);
+  g.eff = __fmul_rn(sg, s);
+  const float r = rcp_approx(g.eff);  // +inf when sg == 0; the codes are then forced to zero
   const f2 r2 = mk2(r, r), blo = mk2(kBracketLo, kBracketLo), bhi = mk2(kBracketHi, kBracketHi);
   float lo[16], hi[16];
 #pragma unroll
@@ -90,16 +93,29 @@ __device__ __forceinline__ uint32_t nvfp4_group16(const float *v, float s, float
   }
   const uint32_t l0 = e2m1x8(lo), l1 = e2m1x8(lo + 8);
   const uint32_t h0 = e2m1x8(hi), h1 = e2m1x8(hi + 8);
-  if ((l0 == h0) & (l1 == h1)) {
-    w0 = l0;
-    w1 = l1;
-    return sc;
-  }
+  const bool zero = sg == 0.0f;
+  g.w0 = zero ? 0u : l0;
+  g.w1 = zero ? 0u : l1;
+  g.exact = !zero && ((l0 != h0) | (l1 != h1));
+  return g;
+}
+
+__device__ __forceinline__ void nvfp4_group16_exact(const float *v, Group16 &g) {
+  float q[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) lo[i] = __fdiv_rn(v[i], eff);
-  w0 = e2m1x8(lo);
-  w1 = e2m1x8(lo + 8);
-  return sc;
+  for (int i = 0; i < 16; ++i) q[i] = __fdiv_rn(v[i], g.eff);
+  g.w0 = e2m1x8(q);
+  g.w1 = e2m1x8(q + 8);
+}
+
+// Both phases; writes the codes to w0, w1 and returns the e4m3 scale code.
+__device__ __forceinline__ uint32_t nvfp4_group16(const float *v, float s, float d, float inv_d, uint32_t &w0,
+                                                  uint32_t &w1) {
+  Group16 g = nvfp4_group16_fast(v, s, d, inv_d);
+  if (g.exact) nvfp4_group16_exact(v, g);
+  w0 = g.w0;
+  w1 = g.w1;
+  return g.sc;
 }
 
 }  // namespace svdq

@@ -3,7 +3,9 @@
 // "Svdq Int4 Flux.1 Canny Dev" model card, "Nunchaku 引擎設計" (b): the down-projection and
 // the quantizer consume the same input, so one kernel serves both.
 //
-// Work decomposition: a CTA owns 128 rows and a contiguous range of 64-column chunks of K.
+// Work decomposition: a CTA owns 128 rows and a contiguous range of 64-column chunks of K,
+// taken two chunks per pipeline stage so that every quantizer thread has two independent
+// groups in flight (the quantizer is latency-bound with one).
 // The CTAs that share a row tile form a thread-block cluster along K (sized so that the grid
 // fits the GPU in one wave); their fp32 partial down-projections are summed through
 // distributed shared memory in cluster-rank order, so the result is deterministic and nothing
@@ -13,13 +15,14 @@
 // bf16 values (hi + lo), so the fp32 result reaches K2 without a 16-bit rounding.
 //
 // Warp roles (576 threads):
-//   warp 0       TMA producer: per chunk the X tile (128 x 64 bf16, 128B swizzle), the L1t
-//                tile (rank x 64 bf16, 128B swizzle) and 64 inv_lambda values.
+//   warp 0       TMA producer: per chunk of a stage the X tile (128 x 64 bf16, 128B swizzle),
+//                the L1t tile (rank x 64 bf16, 128B swizzle), and the stage's inv_lambda values.
 //   warp 1       owns the tensor-memory accumulator (128 lanes x rank fp32 columns) and issues
 //                the bf16 tcgen05 MMAs  acc += bf16(X_hat chunk) * L1 chunk.
 //   warps 2..17  quantizers: lane l of quantizer warp q handles row 8q + l/4 and the 16-element
-//                group l%4 of the chunk: X_hat = fp32(X * inv_lambda), the group's scale and
-//                codes, and bf16(X_hat) into the MMA operand tile (same swizzle as the X tile).
+//                group l%4 of each chunk of the stage: X_hat = fp32(X * inv_lambda), the group's
+//                scale and codes, and bf16(X_hat) into the MMA operand tile (same swizzle as the
+//                X tile).
 #include "common.cuh"
 #include "internal.h"
 #include "nvfp4.cuh"
@@ -29,14 +32,16 @@ namespace {
 
 template <int RANK>
 struct QCfg {
-  static constexpr int STAGES = 4;
+  static constexpr int SUB = 2;  // 64-column chunks per stage
+  static constexpr int STAGES = RANK <= 32 ? 3 : 2;
   static constexpr int QWARPS = 16;
   static constexpr int THREADS = 64 + 32 * QWARPS;
-  static constexpr uint32_t X_BYTES = 128u * 128u;
+  static constexpr uint32_t X_BYTES = 128u * 128u;           // per chunk
   static constexpr uint32_t OP_BYTES = RANK ? 128u * 128u : 0u;
   static constexpr uint32_t L1_BYTES = RANK * 128u;
   static constexpr uint32_t IL_BYTES = 64u * 4u;
-  static constexpr uint32_t STAGE_BYTES = (X_BYTES + OP_BYTES + L1_BYTES + IL_BYTES + 1023u) & ~1023u;
+  // stage: X[SUB] | OP[SUB] | L1[SUB] | inv_lambda[SUB x 64]
+  static constexpr uint32_t STAGE_BYTES = (SUB * (X_BYTES + OP_BYTES + L1_BYTES + IL_BYTES) + 1023u) & ~1023u;
   // split-K partials: 128 rows of RANK fp32, row stride RANK + 4 (16-byte accesses spread over banks)
   static constexpr uint32_t RED_STRIDE = RANK + 4;
   static constexpr uint32_t RED_BYTES = RED_STRIDE * 128u * 4u;
@@ -85,10 +90,16 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
   if (n_local > a.chunks_per_split) n_local = a.chunks_per_split;
   if (n_local < 0) n_local = 0;
 
-  auto x_tile = [&](int s) { return smem + s * C::STAGE_BYTES; };
-  auto op_tile = [&](int s) { return smem + s * C::STAGE_BYTES + C::X_BYTES; };
-  auto l1_tile = [&](int s) { return smem + s * C::STAGE_BYTES + C::X_BYTES + C::OP_BYTES; };
-  auto il_tile = [&](int s) { return smem + s * C::STAGE_BYTES + C::X_BYTES + C::OP_BYTES + C::L1_BYTES; };
+  constexpr int SUB = C::SUB;
+  const int n_stages = (n_local + SUB - 1) / SUB;
+  auto x_tile = [&](int s, int u) { return smem + s * C::STAGE_BYTES + u * C::X_BYTES; };
+  auto op_tile = [&](int s, int u) { return smem + s * C::STAGE_BYTES + SUB * C::X_BYTES + u * C::OP_BYTES; };
+  auto l1_tile = [&](int s, int u) {
+    return smem + s * C::STAGE_BYTES + SUB * (C::X_BYTES + C::OP_BYTES) + u * C::L1_BYTES;
+  };
+  auto il_tile = [&](int s, int u) {
+    return smem + s * C::STAGE_BYTES + SUB * (C::X_BYTES + C::OP_BYTES + C::L1_BYTES) + u * C::IL_BYTES;
+  };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
@@ -113,14 +124,19 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tm_x);
       if (RANK) tma_prefetch_desc(&tm_l1);
-      for (int i = 0; i < n_local; ++i) {
+      for (int i = 0; i < n_stages; ++i) {
         const int s = i % ST;
         if (i >= ST && !mbar_wait(bar_empty + 8 * s, ((i / ST) - 1) & 1, a.err, KID_QUANT, 1)) break;
-        mbar_arrive_expect_tx(bar_full + 8 * s, C::X_BYTES + C::L1_BYTES + C::IL_BYTES);
-        const int kx = (c_begin + i) * 64;
-        tma_load_2d(smem_u32(x_tile(s)), &tm_x, kx, m0, bar_full + 8 * s);
-        if (RANK) tma_load_2d(smem_u32(l1_tile(s)), &tm_l1, kx, 0, bar_full + 8 * s);
-        bulk_load(smem_u32(il_tile(s)), a.inv_lambda + kx, C::IL_BYTES, bar_full + 8 * s);
+        // chunks of this stage that lie inside the CTA's range (the last stage may hold one)
+        const int nu = min(SUB, n_local - i * SUB);
+        const uint32_t fb = bar_full + 8 * s;
+        mbar_arrive_expect_tx(fb, nu * (C::X_BYTES + C::L1_BYTES + C::IL_BYTES));
+        for (int u = 0; u < nu; ++u) {
+          const int kx = (c_begin + i * SUB + u) * 64;
+          tma_load_2d(smem_u32(x_tile(s, u)), &tm_x, kx, m0, fb);
+          if (RANK) tma_load_2d(smem_u32(l1_tile(s, u)), &tm_l1, kx, 0, fb);
+          bulk_load(smem_u32(il_tile(s, u)), a.inv_lambda + kx, C::IL_BYTES, fb);
+        }
       }
     }
   } else if (warp == 1) {
@@ -129,17 +145,20 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
       // kind::f16: D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9, 10-12 = 1), K-major,
       // N = RANK (bits 17-22 = N >> 3), M = 128 (bits 24-28 = M >> 4).
       const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(RANK) >> 3) << 17) | ((128u >> 4) << 24);
-      for (int i = 0; i < n_local; ++i) {
+      for (int i = 0; i < n_stages; ++i) {
         const int s = i % ST;
         const uint32_t par = (i / ST) & 1;
         if (!mbar_wait(bar_opfull + 8 * s, par, a.err, KID_QUANT, 2)) break;
         if (!mbar_wait(bar_full + 8 * s, par, a.err, KID_QUANT, 3)) break;
         tc_fence_after();
-        const uint64_t ad = umma_desc(smem_u32(op_tile(s)), 16, 1024, 2);
-        const uint64_t bd = umma_desc(smem_u32(l1_tile(s)), 16, 1024, 2);
+        const int nu = min(SUB, n_local - i * SUB);
+        for (int u = 0; u < nu; ++u) {
+          const uint64_t ad = umma_desc(smem_u32(op_tile(s, u)), 16, 1024, 2);
+          const uint64_t bd = umma_desc(smem_u32(l1_tile(s, u)), 16, 1024, 2);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_bf16(tbase, ad + 2u * k, bd + 2u * k, idesc, (i | k) != 0 ? 1u : 0u);
+          for (int k = 0; k < 4; ++k)
+            mma_bf16(tbase, ad + 2u * k, bd + 2u * k, idesc, (i | u | k) != 0 ? 1u : 0u);
+        }
         tc_commit(bar_empty + 8 * s);
       }
       tc_commit(bar_acc);
@@ -153,42 +172,57 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
     // per-chunk output addresses advance by 32 code bytes and one 512-byte scale block
     uint8_t *xq_p = a.xq + static_cast<size_t>(m) * (a.K / 2) + c_begin * 32 + 8 * g;
     uint8_t *xs_p = a.xs + scale_offset(m, c_begin * 4 + g, a.K / 16);
-    for (int i = 0; i < n_local; ++i, xq_p += 32, xs_p += 512) {
+    for (int i = 0; i < n_stages; ++i, xq_p += 32 * SUB, xs_p += 512 * SUB) {
       const int s = i % ST;
       if (!mbar_wait(bar_full + 8 * s, (i / ST) & 1, a.err, KID_QUANT, 4)) break;
-      const uint8_t *xt = x_tile(s) + row * 128;
-      const uint4 raw0 = *reinterpret_cast<const uint4 *>(xt + (c0 << 4));
-      const uint4 raw1 = *reinterpret_cast<const uint4 *>(xt + (c1 << 4));
-      const float4 *il4 = reinterpret_cast<const float4 *>(il_tile(s) + g * 64);
-      const float4 l0 = il4[0], l1 = il4[1], l2 = il4[2], l3 = il4[3];
-      const uint32_t w[8] = {raw0.x, raw0.y, raw0.z, raw0.w, raw1.x, raw1.y, raw1.z, raw1.w};
-      const float il[16] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w,
-                            l2.x, l2.y, l2.z, l2.w, l3.x, l3.y, l3.z, l3.w};
-      float xh[16];
+      const int nu = min(SUB, n_local - i * SUB);
+      // The chunks of the stage are independent and computed without branches (a chunk past the
+      // CTA's range computes on stale data and stores nothing), so their arithmetic interleaves.
+      float xh[SUB][16];
 #pragma unroll
-      for (int e = 0; e < 8; ++e)
-        un2(mul2(mk2(bf16_lo(w[e]), bf16_hi(w[e])), mk2(il[2 * e], il[2 * e + 1])), xh[2 * e], xh[2 * e + 1]);
+      for (int u = 0; u < SUB; ++u) {
+        const uint8_t *xt = x_tile(s, u) + row * 128;
+        const uint4 raw0 = *reinterpret_cast<const uint4 *>(xt + (c0 << 4));
+        const uint4 raw1 = *reinterpret_cast<const uint4 *>(xt + (c1 << 4));
+        const float4 *il4 = reinterpret_cast<const float4 *>(il_tile(s, u) + g * 64);
+        const float4 l0 = il4[0], l1 = il4[1], l2 = il4[2], l3 = il4[3];
+        const uint32_t w[8] = {raw0.x, raw0.y, raw0.z, raw0.w, raw1.x, raw1.y, raw1.z, raw1.w};
+        const float il[16] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w,
+                              l2.x, l2.y, l2.z, l2.w, l3.x, l3.y, l3.z, l3.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          un2(mul2(mk2(bf16_lo(w[e]), bf16_hi(w[e])), mk2(il[2 * e], il[2 * e + 1])), xh[u][2 * e], xh[u][2 * e + 1]);
+      }
       if (QUANT) {
-        uint2 codes;
-        const uint32_t sc = nvfp4_group16(xh, a.s_x, a.d_x, a.inv_d, codes.x, codes.y);
-        if (m < a.M) *reinterpret_cast<uint2 *>(xq_p) = codes;
-        *xs_p = static_cast<uint8_t>(sc);
+        Group16 q[SUB];
+#pragma unroll
+        for (int u = 0; u < SUB; ++u) q[u] = nvfp4_group16_fast(xh[u], a.s_x, a.d_x, a.inv_d);
+#pragma unroll
+        for (int u = 0; u < SUB; ++u) {
+          if (u >= nu) break;
+          if (q[u].exact) nvfp4_group16_exact(xh[u], q[u]);
+          if (m < a.M) *reinterpret_cast<uint2 *>(xq_p + 32 * u) = make_uint2(q[u].w0, q[u].w1);
+          xs_p[512 * u] = static_cast<uint8_t>(q[u].sc);
+        }
       }
       if (RANK) {
-        uint8_t *ot = op_tile(s) + row * 128;
-        uint4 v0, v1;
-        v0.x = pack_bf16x2(xh[0], xh[1]);
-        v0.y = pack_bf16x2(xh[2], xh[3]);
-        v0.z = pack_bf16x2(xh[4], xh[5]);
-        v0.w = pack_bf16x2(xh[6], xh[7]);
-        v1.x = pack_bf16x2(xh[8], xh[9]);
-        v1.y = pack_bf16x2(xh[10], xh[11]);
-        v1.z = pack_bf16x2(xh[12], xh[13]);
-        v1.w = pack_bf16x2(xh[14], xh[15]);
-        *reinterpret_cast<uint4 *>(ot + (c0 << 4)) = v0;
-        *reinterpret_cast<uint4 *>(ot + (c1 << 4)) = v1;
-        fence_proxy_async_smem();
+#pragma unroll
+        for (int u = 0; u < SUB; ++u) {
+          uint8_t *ot = op_tile(s, u) + row * 128;
+          uint4 v0, v1;
+          v0.x = pack_bf16x2(xh[u][0], xh[u][1]);
+          v0.y = pack_bf16x2(xh[u][2], xh[u][3]);
+          v0.z = pack_bf16x2(xh[u][4], xh[u][5]);
+          v0.w = pack_bf16x2(xh[u][6], xh[u][7]);
+          v1.x = pack_bf16x2(xh[u][8], xh[u][9]);
+          v1.y = pack_bf16x2(xh[u][10], xh[u][11]);
+          v1.z = pack_bf16x2(xh[u][12], xh[u][13]);
+          v1.w = pack_bf16x2(xh[u][14], xh[u][15]);
+          *reinterpret_cast<uint4 *>(ot + (c0 << 4)) = v0;
+          *reinterpret_cast<uint4 *>(ot + (c1 << 4)) = v1;
+        }
       }
+      if (RANK) fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) {
         mbar_arrive(bar_empty + 8 * s);
