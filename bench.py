@@ -1,6 +1,7 @@
 """Benchmark of the SVDQuant NVFP4 W4A4 + low-rank linear (libsvdq) on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--workload qkv]
+    python bench.py --suite [names] [--steps K]     (one line per workload; rank-overhead sweep)
 
 One step = one forward pass of the layer over one batch of synthetic tokens: K1
 (svdq_quant_act_lora_down: smoothing, NVFP4 activation quantization, low-rank down-projection)
@@ -9,6 +10,10 @@ Default workload: the FLUX-like fused QKV projection, M = 4608 tokens, K = 3072,
 rank 32. Inputs are resident in HBM when the timed region starts; successive steps rotate
 over three buffer sets (inputs, activations, outputs and layer copies, >3x the 126 MB L2) so
 that no step finds its operands in L2.
+
+The timed loop replays CUDA graphs captured from the library calls (one K1 and one K2 graph
+per buffer set), so it measures the device rather than per-call host work; the e2e number goes
+through the host-buffer entry point call by call.
 
 Metric: layer TFLOPS = (2MNK + 2MNr + 2MKr) / step time, summed over ranks (weak scaling:
 every rank runs its own replica on its own batch, no collective on the data path).
@@ -198,6 +203,132 @@ def workload_name(shape):
     return f"{shape.name}: SVDQuant NVFP4 W4A4+LoRA linear M={shape.M} K={shape.K} N={shape.N} rank={shape.rank}"
 
 
+def capture_steps(nb, parts_of):
+    """CUDA graphs of the layer's kernels for each of `nb` buffer sets: [(graph_k1, graph_k2)].
+    parts_of(j) returns two callables (the second may be None) that launch on a given stream.
+    Replaying a graph submits the kernels without the per-call host work (argument checks,
+    tensor-map encoding), so the timed loop measures the device."""
+    import torch
+
+    out = []
+    side = torch.cuda.Stream()
+    for j in range(nb):
+        pair = []
+        for fn in parts_of(j):
+            if fn is None:
+                pair.append(None)
+                continue
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=side):
+                fn(torch.cuda.current_stream())
+            pair.append(g)
+        out.append(tuple(pair))
+    torch.cuda.synchronize()
+    return out
+
+
+SUITE = ["qkv", "mlp_up", "mlp_down", "sweep_m256", "sweep_m1024", "sweep_m4096", "sweep_m16384",
+         "sweep_r0", "sweep_r16", "sweep_r32", "sweep_r64", "sweep_r128"]
+
+
+def time_layer(shape, steps, warmup, dev, stream, unfused=False, nb=3):
+    """Mean device time (ms) per step of the layer on one GPU over `nb` rotating buffer sets:
+    fused K1 + K2, or the unfused four-kernel path. Returns (step_ms, k1_ms, k2_ms)."""
+    import torch
+    from bit_rank_compensated_b200 import svdq
+
+    M, K, N, r = shape.M, shape.K, shape.N, shape.rank
+    Xb, W, b, _ = make_inputs(shape, seed=0)
+    X0 = torch.from_numpy(Xb.view(np.int16)).to(dev).view(torch.bfloat16)
+    ax = svdq.act_absmax(X0)
+    L = svdq.prepare_weights(torch.from_numpy(W).to(dev), torch.from_numpy(b).to(dev), ax, r)
+    Xs = [X0] + [X0.clone() for _ in range(nb - 1)]
+    bufs = [svdq.alloc_activations(M, L, dev) for _ in range(nb)]
+    Ys = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(nb)]
+
+    def step_on(j):
+        # part 0: K1 (or the whole unfused path), part 1: K2 (None when unfused)
+        xq, xs, la = bufs[j]
+        if unfused:
+            return (lambda st: svdq.unfused_forward(Xs[j], L, bufs[j], Ys[j], st)), None
+        return ((lambda st: svdq.quant_act_lora_down(Xs[j], L, xq, xs, la, st)),
+                (lambda st: svdq.gemm_w4a4_lora_up(xq, xs, la, M, L, Ys[j], st)))
+
+    def step(i):
+        a, b = step_on(i % nb)
+        a(stream)
+        if b is not None:
+            b(stream)
+
+    for i in range(warmup):
+        step(i)
+    torch.cuda.synchronize()
+    graphs = capture_steps(nb, step_on)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(steps):
+        g1, g2 = graphs[i % nb]
+        if not unfused:
+            ev[i][0].record(stream)
+        g1.replay()
+        if not unfused:
+            ev[i][1].record(stream)
+        if g2 is not None:
+            g2.replay()
+        if not unfused:
+            ev[i][2].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    assert svdq.last_device_error() == 0
+    total = t0.elapsed_time(t1) / steps
+    if unfused:
+        return total, None, None
+    return (total, statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
+            statistics.mean(e[1].elapsed_time(e[2]) for e in ev))
+
+
+def run_suite(args):
+    """One JSON line per named workload (device time, fused path; the rank sweep also times
+    rank 0 and the unfused four-kernel path at the same rank). Not part of the default run."""
+    import torch
+    from bit_rank_compensated_b200 import build, svdq
+
+    if not os.path.exists(svdq.LIB_PATH):
+        build.build()
+    svdq.load()
+    dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    hbm_gbs, bf16_tf, peak_kind = read_peaks()
+    fp4_peak = bf16_tf * FP4_OVER_BF16
+    r0_ms = None
+    for name in args.suite.split(","):
+        shape = CONFIGS[name]
+        M, K, N, r = shape.M, shape.K, shape.N, shape.rank
+        step_ms, k1_ms, k2_ms = time_layer(shape, args.steps, args.warmup, dev, stream)
+        line = {"metric": METRIC, "value": layer_flops(M, K, N, r) / (step_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+                "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+                "higher_is_better": True, "dtype": "nvfp4", "data": "synthetic",
+                "config": {"workload": workload_name(shape), "M": M, "K": K, "N": N, "rank": r},
+                "k1": {"us": k1_ms * 1e3, "gbs": k1_bytes(M, K, r) / (k1_ms * 1e-3) / 1e9,
+                       "frac_hbm": k1_bytes(M, K, r) / (k1_ms * 1e-3) / 1e9 / hbm_gbs},
+                "k2": {"us": k2_ms * 1e3, "tflops": k2_flops(M, K, N, r) / (k2_ms * 1e-3) / 1e12,
+                       "frac_fp4": k2_flops(M, K, N, r) / (k2_ms * 1e-3) / 1e12 / fp4_peak},
+                "tokens_per_s": M / (step_ms * 1e-3), "peaks": peak_kind}
+        if name.startswith("sweep_r"):
+            if r == 0:
+                r0_ms = step_ms
+            else:
+                unf_ms, _, _ = time_layer(shape, args.steps, args.warmup, dev, stream, unfused=True)
+                line["unfused_ms"] = unf_ms
+                line["unfused_over_fused"] = unf_ms / step_ms
+                if r0_ms is not None:
+                    line["lowrank_overhead_vs_r0"] = step_ms / r0_ms - 1.0
+        print(json.dumps(line), flush=True)
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -207,8 +338,12 @@ def main(argv=None):
     ap.add_argument("--workload", default="qkv", choices=sorted(CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--suite", nargs="?", const=",".join(SUITE), default=None,
+                    help="time a comma-separated list of workloads (default: all) and print one line each")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
+    if args.suite:
+        return run_suite(args)
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -269,6 +404,17 @@ def main(argv=None):
     torch.cuda.synchronize()
     assert svdq.last_device_error() == 0
 
+    def parts(j):
+        xq, xs, la = bufs[j]
+        return ((lambda st: svdq.quant_act_lora_down(Xs[j], layers[j], xq, xs, la, st)),
+                (lambda st: svdq.gemm_w4a4_lora_up(xq, xs, la, M, layers[j], Ys[j], st)))
+
+    graphs = capture_steps(NB, parts)
+    for i in range(NB):  # one warm replay of each graph
+        graphs[i][0].replay()
+        graphs[i][1].replay()
+    torch.cuda.synchronize()
+
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True),
            torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
@@ -281,12 +427,11 @@ def main(argv=None):
         t_end = torch.cuda.Event(enable_timing=True)
         t_start.record(stream)
         for i in range(args.steps):
-            j = i % NB
-            xq, xs, la = bufs[j]
+            g1, g2 = graphs[i % NB]
             ev[i][0].record(stream)
-            svdq.quant_act_lora_down(Xs[j], layers[j], xq, xs, la, stream)
+            g1.replay()
             ev[i][1].record(stream)
-            svdq.gemm_w4a4_lora_up(xq, xs, la, M, layers[j], Ys[j], stream)
+            g2.replay()
             ev[i][2].record(stream)
         t_end.record(stream)
         torch.cuda.synchronize()
