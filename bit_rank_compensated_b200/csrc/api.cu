@@ -121,7 +121,7 @@ svdq_status run_quant(const uint16_t *X, int M, const svdq_layer *L, uint8_t *xq
   QuantLaunch q;
   memset(&q, 0, sizeof(q));
   const int K = L->K, r = lora ? L->rank : 0;
-  if (!make_map(&q.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, static_cast<uint64_t>(K) * 2, 64, 128,
+  if (!make_map(&q.tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, X, K, M, static_cast<uint64_t>(K) * 2, 64, kQuantRows,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return SVDQ_ERR_CUDA;
   if (r > 0) {

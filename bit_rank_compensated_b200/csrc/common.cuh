@@ -372,6 +372,28 @@ __device__ __forceinline__ uint32_t map_shared_rank(uint32_t addr, uint32_t rank
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
   return r;
 }
+// 16-byte load from this CTA's shared memory (explicit state space: a generic load of a shared
+// address costs the generic-to-shared resolution on every access).
+__device__ __forceinline__ uint4 ld_shared_u32x4(uint32_t addr) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_shared_u16(uint32_t addr) {
+  uint16_t v;
+  asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_shared_u32(uint32_t addr) {
+  uint32_t v;
+  asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ void st_shared_u32x4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
 __device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t addr) {
   float4 v;
   asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
@@ -400,9 +422,10 @@ __device__ __forceinline__ float e4m3_value(uint32_t code) {
   return __half2float(__ushort_as_half(static_cast<uint16_t>(h2 & 0xFFFF)));
 }
 
-// Eight fp32 values -> eight e2m1 codes (round to nearest even, saturating to +-6),
-// element i in bits [4i, 4i + 4). Negative values that round to zero are encoded as +0.
-__device__ __forceinline__ uint32_t e2m1x8(const float *v) {
+// Eight fp32 values -> eight e2m1 codes as the conversion produces them (round to nearest
+// even, saturating to +-6), element i in bits [4i, 4i + 4); a negative value that rounds to
+// zero comes out as -0 (code 8).
+__device__ __forceinline__ uint32_t e2m1x8_raw(const float *v) {
   uint32_t w;
   asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
@@ -412,12 +435,18 @@ __device__ __forceinline__ uint32_t e2m1x8(const float *v) {
       "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
       : "=r"(w)
       : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
-  // Clear the sign bit of every nibble whose magnitude is zero: adding 7 to a 3-bit
-  // magnitude sets bit 3 exactly when the magnitude is non-zero (no carry between nibbles).
-  const uint32_t mag = w & 0x77777777u;
-  const uint32_t nonzero = (mag + 0x77777777u) & 0x88888888u;
-  return mag | (w & nonzero);
+  return w;
 }
+
+// Clears the sign bit of every nibble whose magnitude is zero (-0 becomes +0): adding 7 to a
+// 3-bit magnitude sets bit 3 exactly when the magnitude is non-zero (no carry between nibbles).
+__device__ __forceinline__ uint32_t e2m1_clear_neg_zero(uint32_t w) {
+  const uint32_t nonzero = ((w & 0x77777777u) + 0x77777777u) & 0x88888888u;
+  return w & (0x77777777u | nonzero);
+}
+
+// Eight fp32 values -> eight e2m1 codes, negative values that round to zero encoded as +0.
+__device__ __forceinline__ uint32_t e2m1x8(const float *v) { return e2m1_clear_neg_zero(e2m1x8_raw(v)); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

@@ -8,8 +8,10 @@
 namespace svdq {
 
 // K1 (and the unfused down-projection / quantize baselines).
+// Rows per K1 tile: the TMA box height of X and the M of its tensor-core down-projection.
+constexpr int kQuantRows = 64;
 struct QuantLaunch {
-  CUtensorMap tm_x;   // X, bf16 [M, K], box 64 x 128, 128B swizzle
+  CUtensorMap tm_x;   // X, bf16 [M, K], box 64 x kQuantRows, 128B swizzle
   CUtensorMap tm_l1;  // L1t, bf16 [rank, K], box 64 x rank, 128B swizzle (unused at rank 0)
   const float *inv_lambda;
   uint8_t *xq;

@@ -6,12 +6,16 @@
 //   code_i = 0 when scale == 0, else e2m1_rn_satfinite(fp32(v_i / fp32(scale * s)))
 // Division means the correctly rounded fp32 quotient.
 //
-// Both divisions go through a reciprocal: q = x * r with r = rcp.approx(y) (at most 1 ulp from
-// 1/y) satisfies |q - x/y| < 2^-21.5 |x/y|, and so does the correctly rounded quotient f. The
-// code (e4m3 or e2m1, both monotone in the value) of any number in [q (1 - 2^-20), q (1 + 2^-20)]
-// is therefore the code of f whenever the codes of the two ends agree; when they differ the
-// group is recomputed with correctly rounded divisions (a rare case: the quotient is within
-// 2^-20 of a rounding threshold).
+// Both divisions go through a reciprocal r = rcp.approx(y), at most 1 ulp (relative 2^-23) from
+// 1/y. For the scale: q = x * r satisfies |q - x/y| < 2^-21.5 |x/y|, and so does the correctly
+// rounded quotient f, so the e4m3 code (monotone in the value) of any number in
+// [q (1 - 2^-20), q (1 + 2^-20)] is the code of f whenever the codes of the two ends agree.
+// For the element codes the bracket is moved onto the reciprocal: with r_lo = RN(r (1 - 2^-20))
+// and r_hi = RN(r (1 + 2^-20)), r_lo < (1 - 2^-21)/y and r_hi > (1 + 2^-21)/y, hence
+// |RN(x r_lo)| < |x/y| (1 - 2^-22) < |f| < |x/y| (1 + 2^-22) < |RN(x r_hi)|, and the e2m1 code of f
+// is the common code of the two products whenever they agree. When the ends disagree the group
+// is recomputed with correctly rounded divisions (a rare case: the quotient is within 2^-20 of
+// a rounding threshold).
 #pragma once
 
 #include "common.cuh"
@@ -57,13 +61,19 @@ __device__ __forceinline__ float absmax16(const float *v) {
   return fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
 }
 
+// e4m3 code of the correctly rounded quotient fp32(amax / d). Kept out of line: it is needed only
+// when the bracket ends disagree, and an inlined division gets evaluated on every group.
+static __device__ __noinline__ uint32_t e4m3_code_of_quotient(float amax, float d) {
+  return e4m3_code(__fdiv_rn(amax, d));
+}
+
 // e4m3 code of fp32(amax / d) for amax >= 0, d > 0, with inv_d = rcp.approx(d).
 __device__ __forceinline__ uint32_t scale_code(float amax, float d, float inv_d) {
   const float q = __fmul_rn(amax, inv_d);
   uint16_t both;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(both) : "f"(__fmul_rn(q, kBracketHi)), "f"(__fmul_rn(q, kBracketLo)));
   const uint32_t lo = both & 0xFFu, hi = both >> 8;
-  return lo == hi ? lo : e4m3_code(__fdiv_rn(amax, d));
+  return lo == hi ? lo : e4m3_code_of_quotient(amax, d);
 }
 
 // Quantizes v[0..15] in two phases so that callers can interleave several groups: the first
@@ -72,8 +82,9 @@ __device__ __forceinline__ uint32_t scale_code(float amax, float d, float inv_d)
 // divisions. Codes: element i of the group in bits [4(i % 8), 4(i % 8) + 4) of word i / 8.
 struct Group16 {
   uint32_t w0, w1, sc;
-  float eff;    // sg * s
-  bool exact;   // the codes must be recomputed by nvfp4_group16_exact
+  uint32_t d0, d1;  // raw codes of the two bracket ends XORed: non-zero nibbles mark undecided elements
+  float eff;        // sg * s
+  bool exact;       // some element is undecided: its code needs the correctly rounded quotient
 };
 
 __device__ __forceinline__ Group16 nvfp4_group16_fast(const float *v, float s, float d, float inv_d) {
@@ -83,21 +94,33 @@ __device__ __forceinline__ Group16 nvfp4_group16_fast(const float *v, float s, f
   const float sg = e4m3_value(g.sc);
   g.eff = __fmul_rn(sg, s);
   const float r = rcp_approx(g.eff);  // +inf when sg == 0; the codes are then forced to zero
-  const f2 r2 = mk2(r, r), blo = mk2(kBracketLo, kBracketLo), bhi = mk2(kBracketHi, kBracketHi);
+  const float rl = __fmul_rn(r, kBracketLo), rh = __fmul_rn(r, kBracketHi);
+  const f2 rl2 = mk2(rl, rl), rh2 = mk2(rh, rh);
   float lo[16], hi[16];
 #pragma unroll
-  for (int i = 0; i < 16; i += 2) {
-    const f2 q = mul2(mk2(v[i], v[i + 1]), r2);
-    un2(mul2(q, blo), lo[i], lo[i + 1]);
-    un2(mul2(q, bhi), hi[i], hi[i + 1]);
+  for (int e = 0; e < 8; ++e) {
+    const f2 p = mk2(v[2 * e], v[2 * e + 1]);
+    un2(mul2(p, rl2), lo[2 * e], lo[2 * e + 1]);
+    un2(mul2(p, rh2), hi[2 * e], hi[2 * e + 1]);
   }
-  const uint32_t l0 = e2m1x8(lo), l1 = e2m1x8(lo + 8);
-  const uint32_t h0 = e2m1x8(hi), h1 = e2m1x8(hi + 8);
+  // Both ends carry the sign of v, so their raw codes agree exactly when the magnitudes do.
+  const uint32_t l0 = e2m1x8_raw(lo), l1 = e2m1x8_raw(lo + 8);
+  const uint32_t h0 = e2m1x8_raw(hi), h1 = e2m1x8_raw(hi + 8);
   const bool zero = sg == 0.0f;
-  g.w0 = zero ? 0u : l0;
-  g.w1 = zero ? 0u : l1;
-  g.exact = !zero && ((l0 != h0) | (l1 != h1));
+  g.w0 = zero ? 0u : e2m1_clear_neg_zero(l0);
+  g.w1 = zero ? 0u : e2m1_clear_neg_zero(l1);
+  g.d0 = l0 ^ h0;
+  g.d1 = l1 ^ h1;
+  g.exact = !zero && ((g.d0 | g.d1) != 0u);
   return g;
+}
+
+// e2m1 code (4 bits) of one fp32 value, -0 encoded as +0.
+__device__ __forceinline__ uint32_t e2m1_code1(float q) {
+  uint16_t b;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}" : "=h"(b) : "f"(0.0f), "f"(q));
+  const uint32_t c = b & 0xFu;
+  return (c & 7u) ? c : 0u;
 }
 
 __device__ __forceinline__ void nvfp4_group16_exact(const float *v, Group16 &g) {

@@ -230,30 +230,34 @@ __device__ __forceinline__ double bf16_to_f64(uint16_t b) {
   return static_cast<double>(__uint_as_float(static_cast<uint32_t>(b) << 16));
 }
 
-// L1t[j][k] = bf16(P[k][j] sqrt(sig_j)), L2t[n][j] = bf16(sqrt(sig_j) Q[n][j]).
-__global__ void k_make_branch(const double *P, const double *Q, const double *sig, int K, int N, int r,
-                              uint16_t *L1t, uint16_t *L2t) {
+// L1t[j][k] = bf16(P[k][j] sqrt(sig_j) / lambda_k) (the smoothing folded into the first factor,
+// so that the down-projection reads X itself), L2t[n][j] = bf16(sqrt(sig_j) Q[n][j]).
+__global__ void k_make_branch(const double *P, const double *Q, const double *sig, const float *lam, int K, int N,
+                              int r, uint16_t *L1t, uint16_t *L2t) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx < K * r) {
     const int k = idx / r, j = idx % r;
-    L1t[static_cast<size_t>(j) * K + k] = f64_to_bf16_rne(P[idx] * sqrt(sig[j]));
+    L1t[static_cast<size_t>(j) * K + k] = f64_to_bf16_rne(P[idx] * sqrt(sig[j]) / static_cast<double>(lam[k]));
   }
   if (idx < N * r) {
-    const int n = idx / r, j = idx % r;
+    const int j = idx % r;
     L2t[idx] = f64_to_bf16_rne(sqrt(sig[j]) * Q[idx]);
   }
 }
 
-// R[n][k] = fp32(W[n][k] lambda[k] - sum_j L1[k][j] L2[j][n]) in fp64; rmax collects max|R|.
+// R[n][k] = fp32(W[n][k] lambda[k] - sum_j lambda[k] L1s[k][j] L2[j][n]) in fp64 (each product
+// exact); rmax collects max|R|.
 __global__ void k_residual(const float *W, const float *lam, const uint16_t *L1t, const uint16_t *L2t, int N, int K,
                            int r, float *R, float *rmax) {
   const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   float mx = 0.0f;
   if (idx < static_cast<size_t>(N) * K) {
     const int n = static_cast<int>(idx / K), k = static_cast<int>(idx % K);
+    const double lk = static_cast<double>(lam[k]);
     double lr = 0.0;
-    for (int j = 0; j < r; ++j) lr += bf16_to_f64(L1t[static_cast<size_t>(j) * K + k]) * bf16_to_f64(L2t[static_cast<size_t>(n) * r + j]);
-    const double what = static_cast<double>(W[idx]) * static_cast<double>(lam[k]);
+    for (int j = 0; j < r; ++j)
+      lr += (lk * bf16_to_f64(L1t[static_cast<size_t>(j) * K + k])) * bf16_to_f64(L2t[static_cast<size_t>(n) * r + j]);
+    const double what = static_cast<double>(W[idx]) * lk;
     const float v = __double2float_rn(what - lr);
     R[idx] = v;
     mx = fabsf(v);
@@ -504,7 +508,7 @@ PrepStatus prepare_run(const PrepArgs &p) {
     k_fix_sign<<<r, 256, 0, st>>>(P, K, Q, N, r);
     PCHK(cudaGetLastError());
     const int nb = (K > N ? K : N) * r;
-    k_make_branch<<<(nb + 255) / 256, 256, 0, st>>>(P, Q, sig, K, N, r, p.L1t, p.L2t);
+    k_make_branch<<<(nb + 255) / 256, 256, 0, st>>>(P, Q, sig, lam, K, N, r, p.L1t, p.L2t);
     PCHK(cudaGetLastError());
   }
   const size_t nk = static_cast<size_t>(N) * K;

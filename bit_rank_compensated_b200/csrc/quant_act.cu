@@ -1,28 +1,34 @@
 // K1: smoothing + NVFP4 activation quantization + low-rank down-projection in one read of X.
 //
 // "Svdq Int4 Flux.1 Canny Dev" model card, "Nunchaku 引擎設計" (b): the down-projection and
-// the quantizer consume the same input, so one kernel serves both.
+// the quantizer consume the same input, so one kernel serves both. The smoothing is folded
+// into the stored factor (L1s = diag(lambda)^-1 L1, prepared offline), so the tensor cores
+// read the bf16 X tile exactly as TMA delivered it and only the quantizer computes
+// X_hat = fp32(X * inv_lambda).
 //
-// Work decomposition: a CTA owns 128 rows and a contiguous range of 64-column chunks of K,
-// taken two chunks per pipeline stage so that every quantizer thread has two independent
-// groups in flight (the quantizer is latency-bound with one).
-// The CTAs that share a row tile form a thread-block cluster along K (sized so that the grid
-// fits the GPU in one wave); their fp32 partial down-projections are summed through
-// distributed shared memory in cluster-rank order, so the result is deterministic and nothing
-// goes through global scratch memory.
+// Work decomposition: a CTA owns a tile of kQuantRows (64) rows and a contiguous range of
+// 64-column chunks of K, taken four chunks (32 KB of X) per pipeline stage. The row tiles cover
+// the activation scale buffer's padded rows (a multiple of 128), so the padding scales are
+// written as zero. The CTAs that share a row tile form a thread-block cluster along K (sized
+// so that the grid fits the GPU in one wave; 64-row tiles let two-CTA clusters fill it for
+// the common shapes, which clusters of three or four cannot); their fp32 partial
+// down-projections are summed through distributed shared memory in cluster-rank order, so
+// the result is deterministic and nothing goes through global scratch memory.
 //
 // The down-projection is stored pre-divided by alpha = s_x s_w as an unevaluated sum of two
 // bf16 values (hi + lo), so the fp32 result reaches K2 without a 16-bit rounding.
 //
 // Warp roles (576 threads):
-//   warp 0       TMA producer: per chunk of a stage the X tile (128 x 64 bf16, 128B swizzle),
-//                the L1t tile (rank x 64 bf16, 128B swizzle), and the stage's inv_lambda values.
-//   warp 1       owns the tensor-memory accumulator (128 lanes x rank fp32 columns) and issues
-//                the bf16 tcgen05 MMAs  acc += bf16(X_hat chunk) * L1 chunk.
-//   warps 2..17  quantizers: lane l of quantizer warp q handles row 8q + l/4 and the 16-element
-//                group l%4 of each chunk of the stage: X_hat = fp32(X * inv_lambda), the group's
-//                scale and codes, and bf16(X_hat) into the MMA operand tile (same swizzle as the
-//                X tile).
+//   warp 0       TMA producer: per chunk of a stage the X tile (rows x 64 bf16, 128B swizzle),
+//                the L1s tile (rank x 64 bf16, 128B swizzle) and the chunk's inv_lambda values.
+//   warp 1       owns the tensor-memory accumulator (rows x rank fp32) and issues the bf16
+//                tcgen05 MMAs (M = rows)  acc += X chunk * L1s chunk  straight from the X tile.
+//   warps 2..17  quantizers. With W = rows / 16 warps per chunk, warp 2 + W u + t handles chunk
+//                u of the stage, rows 16t .. 16t + 15; lane l takes the 16-column group l / 8 of
+//                rows 16t + l % 8 and 16t + 8 + l % 8.
+//                Each quarter-warp reads eight consecutive rows of one group (conflict-free
+//                under the 128B swizzle) and one broadcast copy of the group's 16 inv_lambda
+//                values, which serve both of the lane's rows.
 #include "common.cuh"
 #include "internal.h"
 #include "nvfp4.cuh"
@@ -30,26 +36,33 @@
 namespace svdq {
 namespace {
 
-template <int RANK>
+template <int RANK, bool QUANT>
 struct QCfg {
-  static constexpr int SUB = 2;  // 64-column chunks per stage
-  static constexpr int STAGES = RANK <= 32 ? 3 : 2;
+  static constexpr int ROWS = kQuantRows;
   static constexpr int QWARPS = 16;
+  static constexpr int WARPS_PER_CHUNK = ROWS / 16;
+  static constexpr int SUB = QWARPS / WARPS_PER_CHUNK;  // 64-column chunks per stage
   static constexpr int THREADS = 64 + 32 * QWARPS;
-  static constexpr uint32_t X_BYTES = 128u * 128u;           // per chunk
-  static constexpr uint32_t OP_BYTES = RANK ? 128u * 128u : 0u;
+  static constexpr uint32_t X_BYTES = ROWS * 128u;  // per chunk
   static constexpr uint32_t L1_BYTES = RANK * 128u;
-  static constexpr uint32_t IL_BYTES = 64u * 4u;
-  // stage: X[SUB] | OP[SUB] | L1[SUB] | inv_lambda[SUB x 64]
-  static constexpr uint32_t STAGE_BYTES = (SUB * (X_BYTES + OP_BYTES + L1_BYTES + IL_BYTES) + 1023u) & ~1023u;
-  // split-K partials: 128 rows of RANK fp32, row stride RANK + 4 (16-byte accesses spread over banks)
+  static constexpr uint32_t IL_BYTES = QUANT ? 64u * 4u : 0u;
+  // stage: X[SUB] | L1s[SUB] | inv_lambda[SUB x 64]
+  static constexpr uint32_t STAGE_BYTES = (SUB * (X_BYTES + L1_BYTES + IL_BYTES) + 1023u) & ~1023u;
+  static constexpr uint32_t STAGE_BUDGET = 200u * 1024u;
+  static constexpr int STAGES = (STAGE_BUDGET / STAGE_BYTES) > 6 ? 6 : static_cast<int>(STAGE_BUDGET / STAGE_BYTES);
+  // split-K partials: ROWS rows of RANK fp32, row stride RANK + 4 (16-byte accesses spread over banks)
   static constexpr uint32_t RED_STRIDE = RANK + 4;
-  static constexpr uint32_t RED_BYTES = RED_STRIDE * 128u * 4u;
+  static constexpr uint32_t RED_BYTES = RED_STRIDE * ROWS * 4u;
   static constexpr uint32_t DATA_BYTES =
       (STAGES * STAGE_BYTES > RED_BYTES) ? STAGES * STAGE_BYTES : RED_BYTES;
   static constexpr uint32_t BAR_BYTES = 256;
   static constexpr uint32_t SMEM = DATA_BYTES + BAR_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = RANK <= 32 ? 32u : static_cast<uint32_t>(RANK);
+  // arrivals that free a stage: one per quantizer warp, one MMA commit
+  static constexpr uint32_t EMPTY_COUNT = (QUANT ? QWARPS : 0) + (RANK ? 1 : 0);
+  static_assert(ROWS == 64 || ROWS == 128, "tensor-core M");
+  static_assert(STAGES >= 2, "pipeline needs two stages");
+  static_assert(2 * STAGES + 2 <= static_cast<int>(BAR_BYTES / 8), "barrier area");
 };
 
 struct QArgs {
@@ -63,49 +76,66 @@ struct QArgs {
   uint32_t *err;
 };
 
+// Settles the undecided elements of one group (the non-zero nibbles of d0 / d1, where the two
+// bracket ends gave different codes) with the correctly rounded quotient X_hat / eff, recomputed
+// from the stage buffers (x0, x1: the group's two 16-byte pieces of X; il: its 16 inv_lambda
+// values). Out of line so that the compiler keeps this rare path off the common one.
+__device__ __noinline__ uint2 group_codes_settle(uint32_t x0, uint32_t x1, uint32_t il, float eff, uint32_t w0,
+                                                 uint32_t w1, uint32_t d0, uint32_t d1) {
+  uint32_t w[2] = {w0, w1};
+  const uint32_t dd[2] = {d0, d1};
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    uint32_t m = dd[j];
+    while (m) {
+      const int nib = (__ffs(m) - 1) >> 2;
+      const float x = __uint_as_float(ld_shared_u16((j ? x1 : x0) + 2 * nib) << 16);
+      const float l = __uint_as_float(ld_shared_u32(il + 4 * (8 * j + nib)));
+      const uint32_t c = e2m1_code1(__fdiv_rn(__fmul_rn(x, l), eff));
+      w[j] = (w[j] & ~(0xFu << (4 * nib))) | (c << (4 * nib));
+      m &= ~(0xFu << (4 * nib));
+    }
+  }
+  return make_uint2(w[0], w[1]);
+}
+
 template <int RANK, bool QUANT>
-__global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
+__global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
     k1_quant_act_lora_down(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_l1,
                            QArgs a) {
-  using C = QCfg<RANK>;
+  using C = QCfg<RANK, QUANT>;
   constexpr int ST = C::STAGES;
+  constexpr int SUB = C::SUB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::DATA_BYTES);
-  // bars: full[ST] | empty[ST] | opfull[ST] | accfull | tmem holder
+  // bars: full[ST] | empty[ST] | accfull | tmem holder
   const uint32_t bar_full = smem_u32(bars);
   const uint32_t bar_empty = bar_full + 8 * ST;
-  const uint32_t bar_opfull = bar_empty + 8 * ST;
-  const uint32_t bar_acc = bar_opfull + 8 * ST;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 3 * ST + 1);
+  const uint32_t bar_acc = bar_empty + 8 * ST;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * ST + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int split = blockIdx.x;
   const int nsplit = gridDim.x;
-  const int m0 = blockIdx.y * 128;
+  const int m0 = blockIdx.y * C::ROWS;
   const int nch = a.K / 64;
   const int c_begin = split * a.chunks_per_split;
   int n_local = nch - c_begin;
   if (n_local > a.chunks_per_split) n_local = a.chunks_per_split;
   if (n_local < 0) n_local = 0;
-
-  constexpr int SUB = C::SUB;
   const int n_stages = (n_local + SUB - 1) / SUB;
   auto x_tile = [&](int s, int u) { return smem + s * C::STAGE_BYTES + u * C::X_BYTES; };
-  auto op_tile = [&](int s, int u) { return smem + s * C::STAGE_BYTES + SUB * C::X_BYTES + u * C::OP_BYTES; };
-  auto l1_tile = [&](int s, int u) {
-    return smem + s * C::STAGE_BYTES + SUB * (C::X_BYTES + C::OP_BYTES) + u * C::L1_BYTES;
-  };
+  auto l1_tile = [&](int s, int u) { return smem + s * C::STAGE_BYTES + SUB * C::X_BYTES + u * C::L1_BYTES; };
   auto il_tile = [&](int s, int u) {
-    return smem + s * C::STAGE_BYTES + SUB * (C::X_BYTES + C::OP_BYTES + C::L1_BYTES) + u * C::IL_BYTES;
+    return smem + s * C::STAGE_BYTES + SUB * (C::X_BYTES + C::L1_BYTES) + u * C::IL_BYTES;
   };
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < ST; ++s) {
       mbar_init(bar_full + 8 * s, 1);
-      mbar_init(bar_empty + 8 * s, C::QWARPS + (RANK ? 1 : 0));
-      mbar_init(bar_opfull + 8 * s, C::QWARPS);
+      mbar_init(bar_empty + 8 * s, C::EMPTY_COUNT);
     }
     mbar_init(bar_acc, 1);
     fence_mbar_init();
@@ -126,7 +156,7 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
       if (RANK) tma_prefetch_desc(&tm_l1);
       for (int i = 0; i < n_stages; ++i) {
         const int s = i % ST;
-        if (i >= ST && !mbar_wait(bar_empty + 8 * s, ((i / ST) - 1) & 1, a.err, KID_QUANT, 1)) break;
+        if (i >= ST && !mbar_wait_parked(bar_empty + 8 * s, ((i / ST) - 1) & 1, a.err, KID_QUANT, 1)) break;
         // chunks of this stage that lie inside the CTA's range (the last stage may hold one)
         const int nu = min(SUB, n_local - i * SUB);
         const uint32_t fb = bar_full + 8 * s;
@@ -135,7 +165,7 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
           const int kx = (c_begin + i * SUB + u) * 64;
           tma_load_2d(smem_u32(x_tile(s, u)), &tm_x, kx, m0, fb);
           if (RANK) tma_load_2d(smem_u32(l1_tile(s, u)), &tm_l1, kx, 0, fb);
-          bulk_load(smem_u32(il_tile(s, u)), a.inv_lambda + kx, C::IL_BYTES, fb);
+          if (QUANT) bulk_load(smem_u32(il_tile(s, u)), a.inv_lambda + kx, C::IL_BYTES, fb);
         }
       }
     }
@@ -143,17 +173,16 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
     // ------------------------------------------------------------ MMA issuer
     if (RANK && lane == 0) {
       // kind::f16: D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9, 10-12 = 1), K-major,
-      // N = RANK (bits 17-22 = N >> 3), M = 128 (bits 24-28 = M >> 4).
-      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(RANK) >> 3) << 17) | ((128u >> 4) << 24);
+      // N = RANK (bits 17-22 = N >> 3), M = ROWS (bits 24-28 = M >> 4).
+      const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(RANK) >> 3) << 17) |
+                             ((uint32_t(C::ROWS) >> 4) << 24);
       for (int i = 0; i < n_stages; ++i) {
         const int s = i % ST;
-        const uint32_t par = (i / ST) & 1;
-        if (!mbar_wait(bar_opfull + 8 * s, par, a.err, KID_QUANT, 2)) break;
-        if (!mbar_wait(bar_full + 8 * s, par, a.err, KID_QUANT, 3)) break;
+        if (!mbar_wait_parked(bar_full + 8 * s, (i / ST) & 1, a.err, KID_QUANT, 2)) break;
         tc_fence_after();
         const int nu = min(SUB, n_local - i * SUB);
         for (int u = 0; u < nu; ++u) {
-          const uint64_t ad = umma_desc(smem_u32(op_tile(s, u)), 16, 1024, 2);
+          const uint64_t ad = umma_desc(smem_u32(x_tile(s, u)), 16, 1024, 2);
           const uint64_t bd = umma_desc(smem_u32(l1_tile(s, u)), 16, 1024, 2);
 #pragma unroll
           for (int k = 0; k < 4; ++k)
@@ -163,83 +192,82 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
       }
       tc_commit(bar_acc);
     }
-  } else {
+  } else if (QUANT) {
     // ------------------------------------------------------------ quantizers
-    const int row = 8 * (warp - 2) + (lane >> 2);
-    const int g = lane & 3;
+    const int qw = warp - 2;
+    const int u = qw / C::WARPS_PER_CHUNK;  // chunk of the stage
+    const int g = lane >> 3;                // 16-column group of the chunk
+    const int rl = lane & 7;
+    const int row = 16 * (qw % C::WARPS_PER_CHUNK) + rl;  // and row + 8 (same swizzle phase: row & 7 == rl)
     const int m = m0 + row;
-    const int c0 = (2 * g) ^ (row & 7), c1 = (2 * g + 1) ^ (row & 7);  // swizzled 16-byte chunks
-    // per-chunk output addresses advance by 32 code bytes and one 512-byte scale block
-    uint8_t *xq_p = a.xq + static_cast<size_t>(m) * (a.K / 2) + c_begin * 32 + 8 * g;
-    uint8_t *xs_p = a.xs + scale_offset(m, c_begin * 4 + g, a.K / 16);
+    const uint32_t xoff0 = row * 128 + ((((2 * g) ^ rl)) << 4);
+    const uint32_t xoff1 = row * 128 + ((((2 * g + 1) ^ rl)) << 4);
+    const size_t row_bytes = static_cast<size_t>(a.K) / 2;
+    // per stage the codes advance by SUB chunks of 32 bytes and the scales by SUB 512-byte blocks;
+    // row + 8 sits 8 code rows further and 8 x 16 bytes further in the same scale block (the
+    // tile starts at a multiple of 64 rows, so rows row and row + 8 share one 32-row group)
+    uint8_t *xq_p = a.xq + static_cast<size_t>(m) * row_bytes + (c_begin + u) * 32 + 8 * g;
+    uint8_t *xs_p = a.xs + scale_offset(m, (c_begin + u) * 4 + g, a.K / 16);
+    const bool ok0 = m < a.M, ok1 = m + 8 < a.M;
     for (int i = 0; i < n_stages; ++i, xq_p += 32 * SUB, xs_p += 512 * SUB) {
       const int s = i % ST;
-      if (!mbar_wait(bar_full + 8 * s, (i / ST) & 1, a.err, KID_QUANT, 4)) break;
-      const int nu = min(SUB, n_local - i * SUB);
-      // The chunks of the stage are independent and computed without branches (a chunk past the
-      // CTA's range computes on stale data and stores nothing), so their arithmetic interleaves.
-      float xh[SUB][16];
+      if (!mbar_wait_parked(bar_full + 8 * s, (i / ST) & 1, a.err, KID_QUANT, 4)) break;
+      if (i * SUB + u < n_local) {
+        const uint32_t il4 = smem_u32(il_tile(s, u)) + g * 64;
+        const uint4 l0 = ld_shared_u32x4(il4), l1 = ld_shared_u32x4(il4 + 16), l2 = ld_shared_u32x4(il4 + 32),
+                    l3 = ld_shared_u32x4(il4 + 48);
+        const f2 il[8] = {mk2(__uint_as_float(l0.x), __uint_as_float(l0.y)), mk2(__uint_as_float(l0.z), __uint_as_float(l0.w)),
+                          mk2(__uint_as_float(l1.x), __uint_as_float(l1.y)), mk2(__uint_as_float(l1.z), __uint_as_float(l1.w)),
+                          mk2(__uint_as_float(l2.x), __uint_as_float(l2.y)), mk2(__uint_as_float(l2.z), __uint_as_float(l2.w)),
+                          mk2(__uint_as_float(l3.x), __uint_as_float(l3.y)), mk2(__uint_as_float(l3.z), __uint_as_float(l3.w))};
+        const uint32_t xt = smem_u32(x_tile(s, u));
+        // both rows' groups are independent and computed without branches, so they interleave
+        float xh[2][16];
 #pragma unroll
-      for (int u = 0; u < SUB; ++u) {
-        const uint8_t *xt = x_tile(s, u) + row * 128;
-        const uint4 raw0 = *reinterpret_cast<const uint4 *>(xt + (c0 << 4));
-        const uint4 raw1 = *reinterpret_cast<const uint4 *>(xt + (c1 << 4));
-        const float4 *il4 = reinterpret_cast<const float4 *>(il_tile(s, u) + g * 64);
-        const float4 l0 = il4[0], l1 = il4[1], l2 = il4[2], l3 = il4[3];
-        const uint32_t w[8] = {raw0.x, raw0.y, raw0.z, raw0.w, raw1.x, raw1.y, raw1.z, raw1.w};
-        const float il[16] = {l0.x, l0.y, l0.z, l0.w, l1.x, l1.y, l1.z, l1.w,
-                              l2.x, l2.y, l2.z, l2.w, l3.x, l3.y, l3.z, l3.w};
+        for (int h = 0; h < 2; ++h) {
+          const uint4 raw0 = ld_shared_u32x4(xt + h * 1024 + xoff0);
+          const uint4 raw1 = ld_shared_u32x4(xt + h * 1024 + xoff1);
+          const uint32_t w[8] = {raw0.x, raw0.y, raw0.z, raw0.w, raw1.x, raw1.y, raw1.z, raw1.w};
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          un2(mul2(mk2(bf16_lo(w[e]), bf16_hi(w[e])), mk2(il[2 * e], il[2 * e + 1])), xh[u][2 * e], xh[u][2 * e + 1]);
-      }
-      if (QUANT) {
-        Group16 q[SUB];
-#pragma unroll
-        for (int u = 0; u < SUB; ++u) q[u] = nvfp4_group16_fast(xh[u], a.s_x, a.d_x, a.inv_d);
-#pragma unroll
-        for (int u = 0; u < SUB; ++u) {
-          if (u >= nu) break;
-          if (q[u].exact) nvfp4_group16_exact(xh[u], q[u]);
-          if (m < a.M) *reinterpret_cast<uint2 *>(xq_p + 32 * u) = make_uint2(q[u].w0, q[u].w1);
-          xs_p[512 * u] = static_cast<uint8_t>(q[u].sc);
+          for (int e = 0; e < 8; ++e) un2(mul2(mk2(bf16_lo(w[e]), bf16_hi(w[e])), il[e]), xh[h][2 * e], xh[h][2 * e + 1]);
         }
-      }
-      if (RANK) {
+        Group16 q[2];
 #pragma unroll
-        for (int u = 0; u < SUB; ++u) {
-          uint8_t *ot = op_tile(s, u) + row * 128;
-          uint4 v0, v1;
-          v0.x = pack_bf16x2(xh[u][0], xh[u][1]);
-          v0.y = pack_bf16x2(xh[u][2], xh[u][3]);
-          v0.z = pack_bf16x2(xh[u][4], xh[u][5]);
-          v0.w = pack_bf16x2(xh[u][6], xh[u][7]);
-          v1.x = pack_bf16x2(xh[u][8], xh[u][9]);
-          v1.y = pack_bf16x2(xh[u][10], xh[u][11]);
-          v1.z = pack_bf16x2(xh[u][12], xh[u][13]);
-          v1.w = pack_bf16x2(xh[u][14], xh[u][15]);
-          *reinterpret_cast<uint4 *>(ot + (c0 << 4)) = v0;
-          *reinterpret_cast<uint4 *>(ot + (c1 << 4)) = v1;
-        }
+        for (int h = 0; h < 2; ++h) q[h] = nvfp4_group16_fast(xh[h], a.s_x, a.d_x, a.inv_d);
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          if (q[h].exact) {
+            const uint2 c = group_codes_settle(xt + h * 1024 + xoff0, xt + h * 1024 + xoff1, il4, q[h].eff, q[h].w0,
+                                               q[h].w1, q[h].d0, q[h].d1);
+            q[h].w0 = c.x;
+            q[h].w1 = c.y;
+          }
+        if (ok0) *reinterpret_cast<uint2 *>(xq_p) = make_uint2(q[0].w0, q[0].w1);
+        if (ok1) *reinterpret_cast<uint2 *>(xq_p + 8 * row_bytes) = make_uint2(q[1].w0, q[1].w1);
+        xs_p[0] = static_cast<uint8_t>(q[0].sc);
+        xs_p[128] = static_cast<uint8_t>(q[1].sc);
       }
-      if (RANK) fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(bar_empty + 8 * s);
-        if (RANK) mbar_arrive(bar_opfull + 8 * s);
-      }
+      if (lane == 0) mbar_arrive(bar_empty + 8 * s);
     }
   }
 
   if constexpr (RANK > 0) {
     // ------------------------------------------------------------ split-K reduction
-    float *red = reinterpret_cast<float *>(smem);  // [128][RED_STRIDE] fp32, aliases the stages
+    float *red = reinterpret_cast<float *>(smem);  // [ROWS][RED_STRIDE] fp32, aliases the stages
     constexpr uint32_t RS = C::RED_STRIDE;
     if (warp >= 2) {
+      // A warp reads the 32 tensor-memory lanes of its quadrant (warp % 4). Accumulator row r
+      // sits in lane r for M = 128 and in lane 32 (r / 16) + r % 16 for M = 64 (the upper 16
+      // lanes of each quadrant then hold nothing).
       const int quad = warp & 3;
-      const int row = quad * 32 + lane;
+      const bool row_ok = C::ROWS == 128 || lane < 16;
+      const int row = C::ROWS == 128 ? quad * 32 + lane : quad * 16 + (lane & 15);
       const int grp = (warp - 2) >> 2;  // 0..3: column group
-      const bool ok = mbar_wait(bar_acc, 0, a.err, KID_QUANT, 5) && n_local > 0;
+      const bool ok = mbar_wait_parked(bar_acc, 0, a.err, KID_QUANT, 5) && n_local > 0;
+      // The partials overwrite the stage buffers: every quantizer warp must be done reading
+      // them (the MMA commit above covers only the tensor-core reads).
+      if (QUANT) named_bar_sync(1, 32 * C::QWARPS);
       tc_fence_after();
       const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16);
       float *dst = red + row * RS;
@@ -250,7 +278,7 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; j += 4)
-            *reinterpret_cast<float4 *>(dst + j) =
+            if (row_ok) *reinterpret_cast<float4 *>(dst + j) =
                 ok ? make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
                                  __uint_as_float(r[j + 3]))
                    : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -265,7 +293,7 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < CPG; j += 4)
-          *reinterpret_cast<float4 *>(dst + cb + j) =
+          if (row_ok) *reinterpret_cast<float4 *>(dst + cb + j) =
               ok ? make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
                                __uint_as_float(r[j + 3]))
                  : make_float4(0.f, 0.f, 0.f, 0.f);
@@ -275,9 +303,9 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
     cluster_sync_all();
     // Rows r0 .. r1 - 1 of the tile: sum the partials of all CTAs of the cluster in rank order,
     // four columns per thread.
-    const int rows_per = (128 + nsplit - 1) / nsplit;
+    const int rows_per = (C::ROWS + nsplit - 1) / nsplit;
     const int r0 = split * rows_per;
-    const int r1 = min(128, r0 + rows_per);
+    const int r1 = min(C::ROWS, r0 + rows_per);
     const uint32_t red_addr = smem_u32(red);
     constexpr int QUADS = RANK / 4;
     for (int idx = threadIdx.x; idx < (r1 - r0) * QUADS; idx += C::THREADS) {
@@ -314,6 +342,9 @@ __global__ void __launch_bounds__(QCfg<RANK>::THREADS, 1)
   }
 }
 
+// Row tiles of K1: enough to cover the activation scale buffer's rows (M padded to 128).
+int quant_tiles(int M) { return (M + 127) / 128 * (128 / kQuantRows); }
+
 template <int RANK, bool QUANT>
 cudaError_t set_attrs() {
   static int attr_done[64] = {0};
@@ -321,7 +352,7 @@ cudaError_t set_attrs() {
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
     cudaError_t e = cudaFuncSetAttribute(k1_quant_act_lora_down<RANK, QUANT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, QCfg<RANK>::SMEM);
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, QCfg<RANK, QUANT>::SMEM);
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
@@ -339,8 +370,8 @@ int max_active_clusters(int splits) {
   if (set_attrs<RANK, QUANT>() != cudaSuccess) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(splits, 1, 1);
-  cfg.blockDim = dim3(QCfg<RANK>::THREADS, 1, 1);
-  cfg.dynamicSmemBytes = QCfg<RANK>::SMEM;
+  cfg.blockDim = dim3(QCfg<RANK, QUANT>::THREADS, 1, 1);
+  cfg.dynamicSmemBytes = QCfg<RANK, QUANT>::SMEM;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = splits;
@@ -358,7 +389,7 @@ int max_active_clusters(int splits) {
 // per-CTA fixed cost (pipeline fill, reduction); every CTA gets at least one chunk.
 template <int RANK, bool QUANT>
 int pick_splits_t(int M, int K) {
-  const int tiles = (M + 127) / 128;
+  const int tiles = quant_tiles(M);
   const int nch = K / 64;
   int best = 1;
   long best_cost = -1;
@@ -379,13 +410,13 @@ int pick_splits_t(int M, int K) {
 
 template <int RANK, bool QUANT>
 cudaError_t launch_t(const QuantLaunch &q) {
-  using C = QCfg<RANK>;
+  using C = QCfg<RANK, QUANT>;
   auto kern = k1_quant_act_lora_down<RANK, QUANT>;
   cudaError_t e0 = set_attrs<RANK, QUANT>();
   if (e0 != cudaSuccess) return e0;
   QArgs a{q.inv_lambda, q.xq, q.xs, q.lora_act, q.M, q.K, q.s_x, q.d_x, 1.0f / q.d_x, q.inv_alpha, q.chunks_per_split, q.err};
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(q.splits, (q.M + 127) / 128, 1);
+  cfg.gridDim = dim3(q.splits, quant_tiles(q.M), 1);
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = q.stream;
@@ -404,10 +435,13 @@ cudaError_t launch_t(const QuantLaunch &q) {
 int quant_act_splits(int M, int K, int rank, bool quantize, bool lora, int num_sms) {
   const int r = lora ? rank : 0;
   if (r == 0) {
-    // no cross-CTA reduction: enough CTAs for two per SM, at least one chunk each
-    const int tiles = (M + 127) / 128, nch = K / 64;
-    int sp = 1;
-    while (sp < 16 && tiles * sp < 2 * num_sms && nch >= 2 * sp) sp *= 2;
+    // no cross-CTA reduction: as many CTAs along K as fit one wave, none of them empty
+    const int tiles = quant_tiles(M), nch = K / 64;
+    int sp = num_sms / tiles;
+    if (sp > nch) sp = nch;
+    if (sp > 16) sp = 16;
+    if (sp < 1) sp = 1;
+    while (sp > 1 && (sp - 1) * ((nch + sp - 1) / sp) >= nch) --sp;
     return sp;
   }
   if (quantize) {

@@ -78,7 +78,8 @@ typedef struct svdq_layer {
   uint8_t *ws;              /* svdq_weight_scale_bytes(N, K) bytes: e4m3 group scales of R */
   float *inv_lambda;        /* K floats: fp32(1 / lambda_j) */
   float *lambda;            /* K floats: lambda_j (optional; written by prepare when not NULL) */
-  uint16_t *L1t;            /* rank * K bf16: L1 transposed (row j = column j of L1); NULL if rank 0 */
+  uint16_t *L1t;            /* rank * K bf16: L1s = diag(lambda)^-1 L1 transposed (row j = column j
+                               of L1s; the smoothing folded into the first factor); NULL if rank 0 */
   uint16_t *L2t;            /* N * rank bf16: L2 transposed (row n = column n of L2); NULL if rank 0 */
   float *bias;              /* N floats, or NULL for no bias */
 } svdq_layer;
@@ -112,8 +113,10 @@ SVDQ_API size_t svdq_prepare_workspace_bytes(int N, int K, int rank, svdq_status
  *   either is 0; inv_lambda_j = fp32(1 / lambda_j); W_hat = W diag(lambda) (fp64);
  *   truncated SVD W_hat^T = P S Q^T (fp64, from the eigen-decomposition of the smaller Gram
  *   matrix), sign fixed so that the largest-magnitude entry of each column of P is positive;
- *   L1 = bf16(P_r S_r^1/2), L2 = bf16(S_r^1/2 Q_r^T); R = fp32(W_hat - (L1 L2)^T) (fp64 before
- *   the final rounding); s_w, s_x as in svdq_layer; R quantized to NVFP4 with s_w.
+ *   L1s = bf16(diag(lambda)^-1 P_r S_r^1/2) (the smoothing folded into the first factor, so
+ *   that the down-projection reads X itself: X_hat L1 = X diag(lambda)^-1 L1, "Nunchaku 引擎設計"
+ *   (b)), L2 = bf16(S_r^1/2 Q_r^T); R = fp32(W_hat - (diag(lambda) L1s L2)^T) (fp64 before the
+ *   final rounding); s_w, s_x as in svdq_layer; R quantized to NVFP4 with s_w.
  *   W           device, N x K fp32.
  *   bias        device, N fp32, or NULL. Copied into layer->bias when both are non-NULL.
  *   act_absmax  device, K fp32: calibration maxima a_x (e.g. from svdq_act_absmax).
@@ -142,9 +145,10 @@ SVDQ_API svdq_status svdq_quantize_rows(const float *A, int rows, int K, float s
  * the same input, so they run as one kernel):
  *   X_hat[m, k] = fp32(X[m, k] * inv_lambda[k]);
  *   xq, xs   = NVFP4(X_hat) with tensor scale s_x (same rule as svdq_quantize_rows);
- *   v[m, :]  = fp32( (sum_k bf16(X_hat[m, k]) L1[k, :]) / alpha ),  alpha = fp32(s_x * s_w),
- *              accumulated in fp32 on the tensor cores. The 1/alpha pre-scaling lets K2 add
- *              the branch to the same fp32 accumulator as the 4-bit product.
+ *   v[m, :]  = fp32( (sum_k X[m, k] L1s[k, :]) / alpha ),  alpha = fp32(s_x * s_w), with L1s
+ *              the smoothing-folded factor (so the sum equals X_hat L1), accumulated in fp32 on
+ *              the tensor cores straight from the bf16 input. The 1/alpha pre-scaling lets K2
+ *              add the branch to the same fp32 accumulator as the 4-bit product.
  *   lora_act row m = [hi | lo] (2 * rank bf16): hi = bf16(v), lo = bf16(v - hi), so hi + lo
  *              carries v with ~16 significant bits (no 16-bit rounding of the branch's
  *              intermediate before the up-projection).
@@ -184,7 +188,7 @@ SVDQ_API svdq_status svdq_linear_forward_host(const uint16_t *X_host, int M, con
 /* Unfused baseline: the low-rank branch as separate kernels around the 4-bit GEMM
  * ("Nunchaku 引擎設計" (a): the branch run naively re-reads the 16-bit input in the
  * down-projection and re-writes the 16-bit output in the up-projection).
- *   svdq_baseline_lora_down: lora_act = hi/lo pair of sum_k bf16(X_hat) L1 / alpha (reads X).
+ *   svdq_baseline_lora_down: lora_act = hi/lo pair of sum_k X L1s / alpha (reads X).
  *   svdq_baseline_quantize:  xq, xs = NVFP4(X_hat) (reads X again).
  *   svdq_baseline_gemm_w4a4: Y = bf16(alpha * 4-bit product + bias) (no branch).
  *   svdq_baseline_lora_up:   Y = bf16(Y + alpha * lora_act L2) (reads and rewrites Y).

@@ -16,11 +16,17 @@ What it computes, in the order the method states it:
 2. Low-rank split.  Same card, stage 3: W_hat^T = P S Q^T (SVD), the rank-r branch
    L1 = P_r S_r^1/2 (K x r), L2 = S_r^1/2 Q_r^T (r x N) runs in 16 bits (bf16), and the
    residual R = W_hat - (L1 L2)^T absorbs the rest, including the branch's bf16 rounding.
+   Reading: the down-projection reads the layer input itself.  The engine notes of the
+   same card, item (b), say that the down-projection and the quantizer consume the same
+   input, so the smoothing is folded into the first factor once, offline:
+   X_hat L1 = X (diag(lambda)^-1 L1).  The stored factor is L1s = bf16(diag(lambda)^-1 L1)
+   and the residual is taken against the branch as stored,
+   R = W_hat - (diag(lambda) L1s L2)^T.
 3. 4-bit quantization of R and of X_hat.  "Nunchaku Lite in Diffusers", section
    "التحميل الأصلي في الناشرون" (the ``quantization_config`` block: precision nvfp4,
    group_size 16, rank 32).  NVFP4 = e2m1 codes, one e4m3 scale per 16 consecutive
    elements along K, and one fp32 tensor scale per tensor.
-4. The layer output Y = Q(X_hat) Q(R)^T + (X_hat L1) L2 + b.
+4. The layer output Y = Q(X_hat) Q(R)^T + (X L1s) L2 + b.
 
 Every fp32 operation of the method is emulated as "compute in fp64, round once to
 fp32"; for + - * / and sqrt that equals the correctly rounded fp32 result (double
@@ -220,7 +226,7 @@ class Layer:
     rank: int
     lam: np.ndarray  # (K,) fp32 values
     inv_lam: np.ndarray  # (K,)
-    L1: np.ndarray  # (K, r) bf16 values (fp64 in "fp64" branch mode)
+    L1: np.ndarray  # (K, r) L1s = diag(lambda)^-1 P_r S_r^1/2: bf16 values (fp64 in "fp64" branch mode)
     L2: np.ndarray  # (r, N)
     R: np.ndarray  # (N, K) residual the weight quantizer sees (fp32 values)
     s_w: float
@@ -250,12 +256,12 @@ def prepare(W, b, a_x, rank: int, branch: str = "bf16", unit_lambda: bool = Fals
     if rank > 0:
         P, sig, Q = svd_split(What.T, rank)
         rs = np.sqrt(sig)
-        L1 = P * rs[None, :]
+        L1 = (P * rs[None, :]) / lam[:, None]  # smoothing folded into the first factor
         L2 = rs[:, None] * Q.T
         if branch == "bf16":
             L1 = bf16_round(L1)
             L2 = bf16_round(L2)
-        R = What - (L1 @ L2).T
+        R = What - ((lam[:, None] * L1) @ L2).T
     else:
         L1 = np.zeros((K, 0))
         L2 = np.zeros((0, N))
@@ -280,16 +286,17 @@ def smooth_activations(Xv, layer: Layer):
 
 
 def quant_act_lora_down(Xv, layer: Layer):
-    """Activation side of the layer: NVFP4 codes/scales of X_hat and La = X_hat L1.
+    """Activation side of the layer: NVFP4 codes/scales of X_hat and La = X L1s.
 
-    The down-projection input is bf16(X_hat) (16-bit branch); La is kept in fp64.
-    Returns (codes [M, K], scale codes [M, K/16], La [M, r]).
+    The down-projection reads the layer input X (bf16 values, exact in fp64) against the
+    smoothing-folded factor L1s, so La = X_hat L1 up to the rounding of L1s; La is kept
+    in fp64.  Returns (codes [M, K], scale codes [M, K/16], La [M, r]).
     """
+    Xv = np.asarray(Xv, dtype=np.float64)
     Xh = smooth_activations(Xv, layer)
     codes, scales = nvfp4_quantize(f32(Xh), layer.s_x)
     if layer.rank:
-        Xb = Xh if layer.branch == "fp64" else bf16_round(Xh)
-        La = Xb @ layer.L1
+        La = Xv @ layer.L1
     else:
         La = np.zeros((Xh.shape[0], 0))
     return codes, scales, La

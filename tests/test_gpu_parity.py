@@ -356,3 +356,31 @@ def test_quantize_rows_near_ties(lib):
     wc, wsc = O.nvfp4_quantize(A.astype(np.float64), 1.0)
     np.testing.assert_array_equal(codes.cpu().numpy().reshape(A.shape[0], -1), O.pack_codes(wc))
     np.testing.assert_array_equal(F.blocked_to_scales(scales.cpu().numpy(), A.shape[0], 4), wsc)
+
+
+@pytest.mark.parametrize("rank", [0, 32])
+def test_k1_near_ties_take_the_exact_path(lib, rank):
+    # Smoothed activations whose quotients by the group scale sit on, or within a few ulps of,
+    # every e2m1 rounding threshold; the scale 1.125 has an inexact reciprocal. The bracket ends
+    # disagree for nearly every group, so the activation kernel's correctly rounded fallback
+    # decides the codes (ties to even included).
+    rng = np.random.default_rng(12)
+    M, K, N = 200, 512, 128
+    t = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    X = rng.choice(t, (M, K)) * 1.125 * rng.choice([-1.0, 1.0], (M, K))
+    X[:, ::16] = 6.75 * rng.choice([-1.0, 1.0], (M, K // 16))  # group amax: scale 1.125 at s_x = 1
+    il = (1.0 + rng.integers(-6, 7, K) * 2.0 ** -23).astype(np.float32)
+    il[::16] = 1.0
+    Xb = f32_to_bf16_bits(X.astype(np.float32))
+    assert np.array_equal(bf16_bits_to_f32(Xb).astype(np.float64), X)  # the values are bf16-exact
+    Ld = lib.Layer.from_arrays(N=N, K=K, rank=rank, wq=np.zeros((N, K // 2), np.uint8),
+                               ws=np.zeros(lib.weight_scale_bytes(N, K), np.uint8), inv_lambda=il,
+                               L1t=np.zeros((rank, K), np.uint16) if rank else None,
+                               L2t=np.zeros((N, rank), np.uint16) if rank else None, bias=None, s_w=1.0, s_x=1.0)
+    xq, xs, _ = lib.quant_act_lora_down(x_to_device(Xb), Ld)
+    torch.cuda.synchronize()
+    codes, scales = O.nvfp4_quantize(O.f32(X * il.astype(np.float64)[None, :]), 1.0)
+    np.testing.assert_array_equal(xq.cpu().numpy().reshape(M, K // 2), O.pack_codes(codes))
+    Mp = (M + 127) // 128 * 128
+    np.testing.assert_array_equal(F.blocked_to_scales(xs.cpu().numpy(), Mp, K // 16)[:M], scales)
+    assert lib.last_device_error() == 0

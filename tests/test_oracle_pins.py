@@ -274,7 +274,6 @@ def test_brute_force_dot_products():
     xc, xs, La = O.quant_act_lora_down(X, layer)
     Y = O.gemm_w4a4_lora_up(xc, xs, La, layer)
     rng = np.random.default_rng(9)
-    Xh = O.f32(X * layer.inv_lam)
     for m, n in zip(rng.integers(0, X.shape[0], 20), rng.integers(0, W.shape[0], 20)):
         acc = 0.0
         for k in range(X.shape[1]):
@@ -286,7 +285,7 @@ def test_brute_force_dot_products():
         for j in range(layer.rank):
             xb = 0.0
             for k in range(X.shape[1]):
-                xb += O.bf16_round(Xh[m, k]) * layer.L1[k, j]
+                xb += X[m, k] * layer.L1[k, j]
             lora += xb * layer.L2[j, n]
         want = layer.s_x * layer.s_w * acc + lora + b[n]
         assert abs(Y[m, n] - want) <= 1e-12 * max(1.0, abs(want))
@@ -307,11 +306,25 @@ def test_low_rank_branch_absorbs_outliers():
     assert e_r64 < e_r16 < e_smooth < e_plain
 
 
+def test_folded_branch_equals_smoothed_input_branch():
+    # Unrounded branch: X L1s equals X_hat (P_r S_r^1/2), the down-projection of the smoothed
+    # input, with P, S from an SVD of W_hat^T taken here (the factor's sign choice cancels in
+    # the projector P_r P_r^T, so compare the rank-r products against L2).
+    X, W, b = _tiny_problem()
+    r = 8
+    layer = O.prepare(W, b, O.calibration_absmax(X), r, branch="fp64")
+    Xh = X / layer.lam[None, :]
+    U, S, Vh = np.linalg.svd((W * layer.lam[None, :]).T, full_matrices=False)
+    want = Xh @ U[:, :r] @ np.diag(S[:r]) @ Vh[:r]
+    got = (X @ layer.L1) @ layer.L2
+    assert np.abs(got - want).max() <= 1e-10 * np.abs(want).max()
+
+
 def test_residual_absorbs_bf16_branch_rounding():
     X, W, b = _tiny_problem()
     layer = O.prepare(W, b, O.calibration_absmax(X), 16)
     What = W * layer.lam[None, :]
-    recon = layer.R + (layer.L1 @ layer.L2).T
+    recon = layer.R + ((layer.lam[:, None] * layer.L1) @ layer.L2).T
     assert np.abs(recon - What).max() <= 2.0 ** -24 * np.abs(layer.R).max() * 1.0001
 
 
