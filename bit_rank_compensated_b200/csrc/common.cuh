@@ -364,6 +364,25 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
 }
+// Programmatic dependent launch. A kernel launched with programmatic stream serialization may
+// start while the previous kernel of the stream is still running; grid_dep_wait() returns once
+// that kernel has completed and its memory operations are visible, so a kernel that touches no
+// global memory before it behaves exactly as under plain stream order. grid_dep_launch()
+// lets the next such kernel of the stream be scheduled before this one finishes.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Split cluster barrier: arrive (release) early, wait (acquire) when the other CTAs' progress is
+// needed. Every thread of every CTA of the cluster executes both.
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// 16-byte store into a CTA of the cluster (addr, bar: shared::cluster addresses of that CTA) that
+// counts its bytes against the transaction count of the mbarrier bar there.
+__device__ __forceinline__ void st_async_f32x4(uint32_t addr, float4 v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(addr),
+               "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(bar)
+               : "memory");
+}
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }

@@ -157,6 +157,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   cluster_sync_all();  // both CTAs' barriers initialised and the pair's tensor memory allocated
   tc_fence_after();
   const uint32_t tbase = *tmem_holder;
+  // The prologue above overlaps the previous kernel of the stream; global memory only after it.
+  grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -501,13 +504,15 @@ cudaError_t launch_t(const GemmLaunch &g) {
   cfg.blockDim = dim3(THREADS, 1, 1);
   cfg.dynamicSmemBytes = SMEM;
   cfg.stream = g.stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, k2_gemm_w4a4_lora_up<RANK, FP4, ADD_Y>, g.tm_xq, g.tm_wq, g.tm_la, g.tm_l2,
                             g.tm_y, a);
 }

@@ -50,9 +50,10 @@ struct QCfg {
   static constexpr uint32_t STAGE_BYTES = (SUB * (X_BYTES + L1_BYTES + IL_BYTES) + 1023u) & ~1023u;
   static constexpr uint32_t STAGE_BUDGET = 200u * 1024u;
   static constexpr int STAGES = (STAGE_BUDGET / STAGE_BYTES) > 6 ? 6 : static_cast<int>(STAGE_BUDGET / STAGE_BYTES);
-  // split-K partials: ROWS rows of RANK fp32, row stride RANK + 4 (16-byte accesses spread over banks)
+  // split-K slots: nsplit x ceil(ROWS / nsplit) <= ROWS + 7 rows of RANK fp32, row stride RANK + 4
+  // (16-byte accesses spread over banks)
   static constexpr uint32_t RED_STRIDE = RANK + 4;
-  static constexpr uint32_t RED_BYTES = RED_STRIDE * ROWS * 4u;
+  static constexpr uint32_t RED_BYTES = RED_STRIDE * (ROWS + 8) * 4u;
   static constexpr uint32_t DATA_BYTES =
       (STAGES * STAGE_BYTES > RED_BYTES) ? STAGES * STAGE_BYTES : RED_BYTES;
   static constexpr uint32_t BAR_BYTES = 256;
@@ -62,7 +63,7 @@ struct QCfg {
   static constexpr uint32_t EMPTY_COUNT = (QUANT ? QWARPS : 0) + (RANK ? 1 : 0);
   static_assert(ROWS == 64 || ROWS == 128, "tensor-core M");
   static_assert(STAGES >= 2, "pipeline needs two stages");
-  static_assert(2 * STAGES + 2 <= static_cast<int>(BAR_BYTES / 8), "barrier area");
+  static_assert(2 * STAGES + 3 <= static_cast<int>(BAR_BYTES / 8), "barrier area");
 };
 
 struct QArgs {
@@ -109,11 +110,12 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::DATA_BYTES);
-  // bars: full[ST] | empty[ST] | accfull | tmem holder
+  // bars: full[ST] | empty[ST] | accfull | recv | tmem holder
   const uint32_t bar_full = smem_u32(bars);
   const uint32_t bar_empty = bar_full + 8 * ST;
   const uint32_t bar_acc = bar_empty + 8 * ST;
-  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * ST + 1);
+  const uint32_t bar_recv = bar_acc + 8;
+  uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + 2 * ST + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -126,6 +128,10 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
   if (n_local > a.chunks_per_split) n_local = a.chunks_per_split;
   if (n_local < 0) n_local = 0;
   const int n_stages = (n_local + SUB - 1) / SUB;
+  // split-K reduction: CTA j of the cluster owns rows [j rows_per, min(ROWS, (j + 1) rows_per))
+  const int rows_per = (C::ROWS + nsplit - 1) / nsplit;
+  const int own_r0 = min(C::ROWS, split * rows_per);
+  const int own_r1 = min(C::ROWS, own_r0 + rows_per);
   auto x_tile = [&](int s, int u) { return smem + s * C::STAGE_BYTES + u * C::X_BYTES; };
   auto l1_tile = [&](int s, int u) { return smem + s * C::STAGE_BYTES + SUB * C::X_BYTES + u * C::L1_BYTES; };
   auto il_tile = [&](int s, int u) {
@@ -138,7 +144,10 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
       mbar_init(bar_empty + 8 * s, C::EMPTY_COUNT);
     }
     mbar_init(bar_acc, 1);
+    mbar_init(bar_recv, 1);
     fence_mbar_init();
+    // the other CTAs of the cluster each send RANK fp32 per owned row
+    if (RANK) mbar_arrive_expect_tx(bar_recv, static_cast<uint32_t>((nsplit - 1) * (own_r1 - own_r0) * RANK * 4));
   }
   if (RANK && warp == 1) {
     tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
@@ -148,6 +157,9 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = RANK ? *tmem_holder : 0u;
+  // The prologue above overlaps the previous kernel of the stream; global memory only after it.
+  grid_dep_wait();
+  grid_dep_launch();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -254,8 +266,15 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
 
   if constexpr (RANK > 0) {
     // ------------------------------------------------------------ split-K reduction
-    float *red = reinterpret_cast<float *>(smem);  // [ROWS][RED_STRIDE] fp32, aliases the stages
+    // Each CTA keeps, in its stage memory, one slot per cluster rank for the rows it owns:
+    // slot[src][row - own_r0] = partial of CTA src (RS fp32 per row). Partials of rows owned by
+    // another CTA go there with st.async, counted on that CTA's recv barrier; the owner sums
+    // the slots in rank order (deterministic) once its own writes and the remote bytes are in.
+    // The stage memory of every CTA must be idle first: a split cluster barrier, arrived at as
+    // soon as this CTA's quantizer warps and MMAs are done with it.
     constexpr uint32_t RS = C::RED_STRIDE;
+    const uint32_t slot_bytes = static_cast<uint32_t>(rows_per) * RS * 4u;
+    const uint32_t red_base = smem_u32(smem);
     if (warp >= 2) {
       // A warp reads the 32 tensor-memory lanes of its quadrant (warp % 4). Accumulator row r
       // sits in lane r for M = 128 and in lane 32 (r / 16) + r % 16 for M = 64 (the upper 16
@@ -265,74 +284,80 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
       const int row = C::ROWS == 128 ? quad * 32 + lane : quad * 16 + (lane & 15);
       const int grp = (warp - 2) >> 2;  // 0..3: column group
       const bool ok = mbar_wait_parked(bar_acc, 0, a.err, KID_QUANT, 5) && n_local > 0;
-      // The partials overwrite the stage buffers: every quantizer warp must be done reading
-      // them (the MMA commit above covers only the tensor-core reads).
+      // every quantizer warp must be done reading the stage buffers (the MMA commit above covers
+      // only the tensor-core reads)
       if (QUANT) named_bar_sync(1, 32 * C::QWARPS);
+      cluster_arrive();
       tc_fence_after();
       const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16);
-      float *dst = red + row * RS;
-      if constexpr (RANK == 16) {
-        if (grp == 0) {
-          uint32_t r[16];
-          tmem_ld16(taddr, r);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; j += 4)
-            if (row_ok) *reinterpret_cast<float4 *>(dst + j) =
-                ok ? make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                                 __uint_as_float(r[j + 3]))
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-      } else {
-        constexpr int CPG = RANK / 4;  // columns per group: 8, 16 or 32
-        const int cb = grp * CPG;
-        uint32_t r[CPG];
+      constexpr int CPG = RANK == 16 ? 16 : RANK / 4;  // columns per warp: rank 16 uses one group
+      const int cb = grp * CPG;
+      uint32_t r[CPG];
+      if (RANK != 16 || grp == 0) {
         if constexpr (CPG == 8) tmem_ld8(taddr + cb, r);
         else if constexpr (CPG == 16) tmem_ld16(taddr + cb, r);
         else tmem_ld32(taddr + cb, r);
         tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < CPG; j += 4)
-          if (row_ok) *reinterpret_cast<float4 *>(dst + cb + j) =
-              ok ? make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                               __uint_as_float(r[j + 3]))
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
       }
       tc_fence_before();
-    }
-    cluster_sync_all();
-    // Rows r0 .. r1 - 1 of the tile: sum the partials of all CTAs of the cluster in rank order,
-    // four columns per thread.
-    const int rows_per = (C::ROWS + nsplit - 1) / nsplit;
-    const int r0 = split * rows_per;
-    const int r1 = min(C::ROWS, r0 + rows_per);
-    const uint32_t red_addr = smem_u32(red);
-    constexpr int QUADS = RANK / 4;
-    for (int idx = threadIdx.x; idx < (r1 - r0) * QUADS; idx += C::THREADS) {
-      const int row = r0 + idx / QUADS;
-      const int c = 4 * (idx % QUADS);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      for (int src = 0; src < nsplit; ++src) {
-        const float4 v = ld_shared_cluster_f32x4(map_shared_rank(red_addr + (row * RS + c) * 4, src));
-        acc.x += v.x;
-        acc.y += v.y;
-        acc.z += v.z;
-        acc.w += v.w;
+      cluster_wait();
+      if (row_ok && (RANK != 16 || grp == 0)) {
+        const int owner = row / rows_per;
+        const uint32_t off = static_cast<uint32_t>(split) * slot_bytes +
+                             static_cast<uint32_t>((row - owner * rows_per) * RS + cb) * 4u;
+        if (owner == split) {
+#pragma unroll
+          for (int j = 0; j < CPG; j += 4)
+            *reinterpret_cast<float4 *>(smem + off + 4 * j) =
+                ok ? make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                 __uint_as_float(r[j + 3]))
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        } else {
+          const uint32_t dst = map_shared_rank(red_base + off, owner);
+          const uint32_t rbar = map_shared_rank(bar_recv, owner);
+#pragma unroll
+          for (int j = 0; j < CPG; j += 4)
+            st_async_f32x4(dst + 4 * j,
+                           ok ? make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
+                                            __uint_as_float(r[j + 3]))
+                              : make_float4(0.f, 0.f, 0.f, 0.f),
+                           rbar);
+        }
       }
-      if (m0 + row < a.M) {
-        // lora_act row = [hi(0..RANK-1) | lo(0..RANK-1)], v ~ hi + lo with hi = bf16(v),
-        // lo = bf16(v - hi): the pair carries ~16 significant bits of the fp32 value.
-        const float v0 = __fmul_rn(acc.x, a.inv_alpha), v1 = __fmul_rn(acc.y, a.inv_alpha);
-        const float v2 = __fmul_rn(acc.z, a.inv_alpha), v3 = __fmul_rn(acc.w, a.inv_alpha);
-        const uint32_t h01 = pack_bf16x2(v0, v1), h23 = pack_bf16x2(v2, v3);
-        const uint32_t l01 = pack_bf16x2(__fsub_rn(v0, bf16_lo(h01)), __fsub_rn(v1, bf16_hi(h01)));
-        const uint32_t l23 = pack_bf16x2(__fsub_rn(v2, bf16_lo(h23)), __fsub_rn(v3, bf16_hi(h23)));
-        uint16_t *out = a.lora_act + static_cast<size_t>(m0 + row) * (2 * RANK) + c;
-        *reinterpret_cast<uint2 *>(out) = make_uint2(h01, h23);
-        *reinterpret_cast<uint2 *>(out + RANK) = make_uint2(l01, l23);
+      named_bar_sync(1, 32 * C::QWARPS);
+      mbar_wait_parked(bar_recv, 0, a.err, KID_QUANT, 6);
+      // rows own_r0 .. own_r1 - 1: sum the slots in rank order, four columns per thread
+      constexpr int QUADS = RANK / 4;
+      for (int idx = threadIdx.x - 64; idx < (own_r1 - own_r0) * QUADS; idx += 32 * C::QWARPS) {
+        const int lr = idx / QUADS;
+        const int c = 4 * (idx % QUADS);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int src = 0; src < nsplit; ++src) {
+          const float4 v =
+              *reinterpret_cast<const float4 *>(smem + src * slot_bytes + static_cast<uint32_t>(lr * RS + c) * 4u);
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        const int m = m0 + own_r0 + lr;
+        if (m < a.M) {
+          // lora_act row = [hi(0..RANK-1) | lo(0..RANK-1)], v ~ hi + lo with hi = bf16(v),
+          // lo = bf16(v - hi): the pair carries ~16 significant bits of the fp32 value.
+          const float v0 = __fmul_rn(acc.x, a.inv_alpha), v1 = __fmul_rn(acc.y, a.inv_alpha);
+          const float v2 = __fmul_rn(acc.z, a.inv_alpha), v3 = __fmul_rn(acc.w, a.inv_alpha);
+          const uint32_t h01 = pack_bf16x2(v0, v1), h23 = pack_bf16x2(v2, v3);
+          const uint32_t l01 = pack_bf16x2(__fsub_rn(v0, bf16_lo(h01)), __fsub_rn(v1, bf16_hi(h01)));
+          const uint32_t l23 = pack_bf16x2(__fsub_rn(v2, bf16_lo(h23)), __fsub_rn(v3, bf16_hi(h23)));
+          uint16_t *out = a.lora_act + static_cast<size_t>(m) * (2 * RANK) + c;
+          *reinterpret_cast<uint2 *>(out) = make_uint2(h01, h23);
+          *reinterpret_cast<uint2 *>(out + RANK) = make_uint2(l01, l23);
+        }
       }
+    } else {
+      cluster_arrive();
+      cluster_wait();
     }
-    cluster_sync_all();
   }
 
   __syncthreads();
@@ -420,13 +445,15 @@ cudaError_t launch_t(const QuantLaunch &q) {
   cfg.blockDim = dim3(C::THREADS, 1, 1);
   cfg.dynamicSmemBytes = C::SMEM;
   cfg.stream = q.stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = q.splits;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = q.splits;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = RANK ? 1 : 0;
+  cfg.numAttrs = RANK ? 2 : 1;
   return cudaLaunchKernelEx(&cfg, kern, q.tm_x, q.tm_l1, a);
 }
 
