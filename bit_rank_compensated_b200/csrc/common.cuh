@@ -67,12 +67,18 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 
 // Waits for the phase of the given parity to complete. Gives up after kWaitLimitNs, records
 // the error and returns false; the caller then leaves its loop.
+// The time limit is checked once every kTriesPerCheck tries: a timer read and a 64-bit compare
+// per try would otherwise be most of what a spinning warp issues.
+constexpr int kTriesPerCheck = 16;
+
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *err,
                                           uint32_t kid, uint32_t site) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+#pragma unroll 1
+    for (int i = 0; i < kTriesPerCheck; ++i)
+      if (mbar_try_wait(bar, parity)) return true;
     if (globaltimer() - t0 > kWaitLimitNs) {
       record_error(err, kid, site);
       return false;
@@ -99,7 +105,9 @@ __device__ __forceinline__ bool mbar_wait_parked(uint32_t bar, uint32_t parity, 
   if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
-    if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
+#pragma unroll 1
+    for (int i = 0; i < kTriesPerCheck; ++i)
+      if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
     if (globaltimer() - t0 > kWaitLimitNs) {
       record_error(err, kid, site);
       return false;
