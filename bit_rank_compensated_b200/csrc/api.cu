@@ -395,6 +395,17 @@ svdq_status svdq_baseline_lora_up(const uint16_t *lora_act, int M, const svdq_la
   return run_gemm(nullptr, nullptr, lora_act, M, layer, Y, false, true, true, stream);
 }
 
+svdq_status svdq_selftest_wait_timeout(uint32_t limit_us, void *stream) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  if (limit_us < 1 || limit_us > 1000000) return SVDQ_ERR_INVALID_ARG;
+  return launch_selftest_wait(d->err, static_cast<uint64_t>(limit_us) * 1000ull, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? SVDQ_OK
+             : SVDQ_ERR_CUDA;
+}
+
 svdq_status svdq_last_device_error(void *stream, uint32_t *code) {
   DeviceState *d = nullptr;
   svdq_status st = device_check(&d);

@@ -13,7 +13,7 @@ namespace svdq {
 // ---------------------------------------------------------------- error word
 // A kernel that gives up on a bounded wait records (kernel << 16) | (site << 8) | 1 into the
 // library's device error word (first error wins) and leaves its loops.
-enum KernelId : uint32_t { KID_QUANT = 1, KID_GEMM = 2, KID_PREP = 3, KID_BASE = 4 };
+enum KernelId : uint32_t { KID_QUANT = 1, KID_GEMM = 2, KID_PREP = 3, KID_BASE = 4, KID_SELFTEST = 5 };
 
 // About two seconds of %globaltimer (ns) before a wait is declared lost.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -72,14 +72,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
 constexpr int kTriesPerCheck = 16;
 
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, uint32_t *err,
-                                          uint32_t kid, uint32_t site) {
+                                          uint32_t kid, uint32_t site, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < kTriesPerCheck; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       record_error(err, kid, site);
       return false;
     }
@@ -101,14 +101,15 @@ __device__ __forceinline__ bool mbar_try_wait_hint(uint32_t bar, uint32_t parity
   return ok != 0;
 }
 __device__ __forceinline__ bool mbar_wait_parked(uint32_t bar, uint32_t parity, uint32_t *err, uint32_t kid,
-                                                 uint32_t site, uint32_t hint_ns = 20000) {
+                                                 uint32_t site, uint32_t hint_ns = 20000,
+                                                 uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < kTriesPerCheck; ++i)
       if (mbar_try_wait_hint(bar, parity, hint_ns)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       record_error(err, kid, site);
       return false;
     }

@@ -51,6 +51,9 @@ struct GemmLaunch {
 };
 cudaError_t launch_gemm(const GemmLaunch &g);
 
+// Failure-path self-test (selftest.cu): bounded waits on an mbarrier nobody signals.
+cudaError_t launch_selftest_wait(uint32_t *err, uint64_t limit_ns, cudaStream_t st);
+
 // Offline preparation pieces (prepare.cu).
 cudaError_t launch_col_absmax_f32(const float *A, int rows, int cols, float *out, cudaStream_t st);
 cudaError_t launch_col_absmax_bf16(const uint16_t *A, int rows, int cols, float *out, cudaStream_t st);

@@ -28,7 +28,7 @@ EXPORTED = (
     "svdq_prepare_workspace_bytes", "svdq_prepare_weights", "svdq_quantize_rows", "svdq_quant_act_lora_down",
     "svdq_gemm_w4a4_lora_up", "svdq_linear_forward", "svdq_linear_forward_host", "svdq_baseline_lora_down",
     "svdq_baseline_quantize", "svdq_baseline_gemm_w4a4", "svdq_baseline_lora_up", "svdq_last_device_error",
-    "svdq_smoothing_factors_noalloc",
+    "svdq_smoothing_factors_noalloc", "svdq_selftest_wait_timeout",
 )
 
 
@@ -79,6 +79,7 @@ def load() -> ctypes.CDLL:
         "svdq_baseline_gemm_w4a4": ([P, P, I, LP, P, P], I),
         "svdq_baseline_lora_up": ([P, I, LP, P, P], I),
         "svdq_last_device_error": ([P, ctypes.POINTER(ctypes.c_uint32)], I),
+        "svdq_selftest_wait_timeout": ([ctypes.c_uint32, P], I),
         "svdq_smoothing_factors_noalloc": ([P, P, I, I, P, P, P, P], I),
     }
     for name, (args, res) in sig.items():
@@ -296,6 +297,12 @@ def unfused_forward(X, layer, bufs, Y, stream=None):
     if layer.rank:
         baseline_lora_up(la, M, layer, Y, stream)
     return Y
+
+
+def selftest_wait_timeout(limit_us: int, stream=None) -> None:
+    """Runs the failure-path self-test kernel (bounded waits on an mbarrier nothing signals);
+    read the recorded timeout with last_device_error()."""
+    _check("svdq_selftest_wait_timeout", load().svdq_selftest_wait_timeout(int(limit_us), _stream(stream)))
 
 
 def last_device_error(stream=None) -> int:

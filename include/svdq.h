@@ -224,6 +224,14 @@ SVDQ_API svdq_status svdq_smoothing_factors_noalloc(const float *W, const float 
                                                     float *lambda, float *inv_lambda, float *x_tensor_scale,
                                                     void *stream);
 
+/* Failure-path self-test. Launches one CTA whose bounded waits (the same code every kernel of
+ * the library uses) wait on an mbarrier that nothing signals; each gives up after limit_us
+ * microseconds (1 .. 1000000) and records the timeout as a stalled kernel would, and the kernel
+ * then returns normally: no trap, no fault, the context stays usable. A following
+ * svdq_last_device_error returns SVDQ_ERR_TIMEOUT with *code = (5 << 16) | (1 << 8) | 1.
+ * Asynchronous on stream. */
+SVDQ_API svdq_status svdq_selftest_wait_timeout(uint32_t limit_us, void *stream);
+
 /* Reads and clears the device-side error word after synchronizing stream. *code is 0 when
  * no kernel gave up on a wait; otherwise (kernel id << 16) | (site << 8) | 1.
  * Returns SVDQ_ERR_TIMEOUT when *code != 0. */

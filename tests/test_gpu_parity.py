@@ -384,3 +384,21 @@ def test_k1_near_ties_take_the_exact_path(lib, rank):
     Mp = (M + 127) // 128 * 128
     np.testing.assert_array_equal(F.blocked_to_scales(xs.cpu().numpy(), Mp, K // 16)[:M], scales)
     assert lib.last_device_error() == 0
+
+
+def test_bounded_wait_gives_up_and_context_survives(lib):
+    # The bounded waits every kernel uses, against an mbarrier nothing signals, with a 2 ms
+    # limit: the wait gives up, records the timeout (kernel id 5, site 1) and the kernel
+    # returns; the context stays usable for the next layer call.
+    import time
+    t0 = time.perf_counter()
+    lib.selftest_wait_timeout(2000)
+    code = lib.last_device_error()
+    assert time.perf_counter() - t0 < 5.0
+    assert code == (5 << 16) | (1 << 8) | 1
+    assert lib.last_device_error() == 0  # read clears the word
+    Xb, X, W, b = _problem(CONFIGS["tiny"])
+    layer_o = O.prepare(W, b, O.calibration_absmax(X), 16)
+    _, xq, xs, la = _k1_outputs(lib, Xb, layer_o)
+    _assert_k1_matches(Xb, X, layer_o, xq, xs, la)
+    assert lib.last_device_error() == 0
