@@ -160,6 +160,15 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 // Arrives once on the mbarrier when all previously issued tcgen05 async ops of this thread finish.
+// One lane of a converged warp (the lowest active lane, so the same lane every time the whole
+// warp executes it): MMA issue loops run warp-wide so that their descriptor arithmetic stays
+// warp-uniform, and the elected lane issues the MMAs and the commit that tracks them.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t p;
+  asm volatile("{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\tselp.u32 %0, 1, 0, e;\n\t}" : "=r"(p));
+  return p != 0;
+}
+
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");

@@ -183,26 +183,34 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (RANK && lane == 0) {
+    // The whole warp runs the loop (descriptors stay warp-uniform); one elected lane issues.
+    if (RANK) {
       // kind::f16: D fp32 (bits 4-5 = 1), A and B bf16 (bits 7-9, 10-12 = 1), K-major,
       // N = RANK (bits 17-22 = N >> 3), M = ROWS (bits 24-28 = M >> 4).
       const uint32_t idesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(RANK) >> 3) << 17) |
                              ((uint32_t(C::ROWS) >> 4) << 24);
       for (int i = 0; i < n_stages; ++i) {
         const int s = i % ST;
-        if (!mbar_wait_parked(bar_full + 8 * s, (i / ST) & 1, a.err, KID_QUANT, 2)) break;
+        if (!__all_sync(0xffffffffu, mbar_wait_parked(bar_full + 8 * s, (i / ST) & 1, a.err, KID_QUANT, 2))) break;
         tc_fence_after();
         const int nu = min(SUB, n_local - i * SUB);
-        for (int u = 0; u < nu; ++u) {
-          const uint64_t ad = umma_desc(smem_u32(x_tile(s, u)), 16, 1024, 2);
-          const uint64_t bd = umma_desc(smem_u32(l1_tile(s, u)), 16, 1024, 2);
+        const uint64_t ad0 = umma_desc(smem_u32(x_tile(s, 0)), 16, 1024, 2);
+        const uint64_t bd0 = umma_desc(smem_u32(l1_tile(s, 0)), 16, 1024, 2);
+        if (elect_one()) {
+          for (int u = 0; u < nu; ++u) {
+            // chunk u's tiles sit u * X_BYTES and u * L1_BYTES further (descriptor units of 16 bytes)
+            const uint64_t ad = ad0 + static_cast<uint64_t>(u * (C::X_BYTES >> 4));
+            const uint64_t bd = bd0 + static_cast<uint64_t>(u * (C::L1_BYTES >> 4));
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16(tbase, ad + 2u * k, bd + 2u * k, idesc, (i | u | k) != 0 ? 1u : 0u);
+            for (int k = 0; k < 4; ++k)
+              mma_bf16(tbase, ad + 2u * k, bd + 2u * k, idesc, (i | u | k) != 0 ? 1u : 0u);
+          }
+          tc_commit(bar_empty + 8 * s);
         }
-        tc_commit(bar_empty + 8 * s);
+        __syncwarp();
       }
-      tc_commit(bar_acc);
+      if (elect_one()) tc_commit(bar_acc);
+      __syncwarp();
     }
   } else if (QUANT) {
     // ------------------------------------------------------------ quantizers
