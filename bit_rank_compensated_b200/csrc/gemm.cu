@@ -208,7 +208,9 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (even CTA)
-    if (crank == 0 && lane == 0) {
+    // The whole warp runs the loops, so the descriptor arithmetic stays warp-uniform (no
+    // per-instruction register moves); one elected lane issues the MMAs and their commits.
+    if (crank == 0) {
       // kind::mxf4nvf4: A, B e2m1 (bits 7-9, 10-12 = 1), K-major, N = 256 (bits 17-22),
       // scale type ue4m3 (bit 23 = 0), M = 256 across the pair (bits 24-28), scale ids 0, K = 64.
       const uint32_t idesc_fp4 = (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BMP) >> 4) << 24);
@@ -219,7 +221,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       uint32_t tcount = 0;
       bool ok = true;
       for (int t = pid; t < tiles && ok; t += npairs, ++tcount) {
-        if (tcount > 0 && !mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 2)) {
+        if (tcount > 0 && !__all_sync(0xffffffffu, mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 2))) {
           ok = false;
           break;
         }
@@ -227,7 +229,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int j = 0; j < total; ++j, ++it) {
           const int s = it % STAGES;
           const uint32_t par = (it / STAGES) & 1;
-          if (!mbar_wait(bar_full + 8 * s, par, a.err, KID_GEMM, 3)) {
+          if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, par, a.err, KID_GEMM, 3))) {
             ok = false;
             break;
           }
@@ -237,10 +239,13 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint64_t ad = umma_desc(st, 16, 8 * LORA_ROW, LORA_SWZ);
             const uint64_t ald = umma_desc(st + LORA_LO_OFF, 16, 8 * LORA_ROW, LORA_SWZ);
             const uint64_t bd = umma_desc(st + A_BYTES, 16, 8 * LORA_ROW, LORA_SWZ);
+            if (elect_one()) {
 #pragma unroll
-            for (int k = 0; k < KC / 16; ++k) {
-              mma_bf16_pair(tbase, ad + 2u * k, bd + 2u * k, idesc_bf16, (j | k) != 0 ? 1u : 0u);
-              mma_bf16_pair(tbase, ald + 2u * k, bd + 2u * k, idesc_bf16, 1u);
+              for (int k = 0; k < KC / 16; ++k) {
+                mma_bf16_pair(tbase, ad + 2u * k, bd + 2u * k, idesc_bf16, (j | k) != 0 ? 1u : 0u);
+                mma_bf16_pair(tbase, ald + 2u * k, bd + 2u * k, idesc_bf16, 1u);
+              }
+              tc_commit_pair_mc(bar_empty + 8 * s, 0x3);
             }
           } else {
             const int kt = j - N_LORA;
@@ -248,14 +253,18 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t tsf = tbase + SF_COL0 + SF_COLS * s;
             const uint64_t ad = umma_desc(st, 16, 1024, 2);
             const uint64_t bd = umma_desc(st + A_BYTES, 16, 1024, 2);
-            for (int kb = 0; kb < kbv; ++kb)
-              mma_nvfp4_pair(tbase, ad + 2u * kb, bd + 2u * kb, idesc_fp4, tsf + 4 * kb, tsf + 16 + 8 * kb,
-                             (j | kb) != 0 ? 1u : 0u);
+            if (elect_one()) {
+              for (int kb = 0; kb < kbv; ++kb)
+                mma_nvfp4_pair(tbase, ad + 2u * kb, bd + 2u * kb, idesc_fp4, tsf + 4 * kb, tsf + 16 + 8 * kb,
+                               (j | kb) != 0 ? 1u : 0u);
+              tc_commit_pair_mc(bar_empty + 8 * s, 0x3);
+            }
           }
-          tc_commit_pair_mc(bar_empty + 8 * s, 0x3);
+          __syncwarp();
         }
         if (!ok) break;
-        tc_commit_pair_mc(bar_accfull, 0x3);
+        if (elect_one()) tc_commit_pair_mc(bar_accfull, 0x3);
+        __syncwarp();
       }
       // both CTAs' output stages have released the last accumulator
       if (ok && tcount > 0) mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 8);
