@@ -181,7 +181,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         const int wrow0 = nt * BN + static_cast<int>(crank) * BNH;  // this CTA's rows of W
         for (int j = 0; j < total; ++j, ++it) {
           const int s = it % STAGES;
-          if (it >= STAGES && !mbar_wait_parked(bar_empty + 8 * s, ((it / STAGES) - 1) & 1, a.err, KID_GEMM, 1)) {
+          // spin rather than park: a parked thread wakes measurably later, and this round trip
+          // (slot released -> loads issued -> stage full) is the kernel's critical path
+          if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1, a.err, KID_GEMM, 1)) {
             ok = false;
             break;
           }
@@ -312,7 +314,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     auto put = [&](int step, const Lines &b) -> bool {
       const int s = step % STAGES;
       bool ok = true;
-      if (step >= STAGES) ok = mbar_wait_parked(bar_empty + 8 * s, ((step / STAGES) - 1) & 1, a.err, KID_GEMM, 6);
+      if (step >= STAGES) ok = mbar_wait(bar_empty + 8 * s, ((step / STAGES) - 1) & 1, a.err, KID_GEMM, 6);
       if (!__all_sync(0xffffffffu, ok)) return false;
       if (FP4 && step % total >= N_LORA) {
         // slot columns: SFA k-block kb at 4 kb, SFB k-block kb at 16 + 8 kb (rows 0-127, then 128-255)
