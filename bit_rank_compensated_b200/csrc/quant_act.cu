@@ -229,6 +229,7 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
     uint8_t *xq_p = a.xq + static_cast<size_t>(m) * row_bytes + (c_begin + u) * 32 + 8 * g;
     uint8_t *xs_p = a.xs + scale_offset(m, (c_begin + u) * 4 + g, a.K / 16);
     const bool ok0 = m < a.M, ok1 = m + 8 < a.M;
+    const float s_x = a.s_x, d_x = a.d_x, inv_d = a.inv_d;
     for (int i = 0; i < n_stages; ++i, xq_p += 32 * SUB, xs_p += 512 * SUB) {
       const int s = i % ST;
       if (!mbar_wait_parked(bar_full + 8 * s, (i / ST) & 1, a.err, KID_QUANT, 4)) break;
@@ -253,15 +254,17 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
         }
         Group16 q[2];
 #pragma unroll
-        for (int h = 0; h < 2; ++h) q[h] = nvfp4_group16_fast(xh[h], a.s_x, a.d_x, a.inv_d);
+        for (int h = 0; h < 2; ++h) q[h] = nvfp4_group16_fast(xh[h], s_x, d_x, inv_d);
+        if (q[0].exact | q[1].exact) {  // rare: one branch for both groups
 #pragma unroll
-        for (int h = 0; h < 2; ++h)
-          if (q[h].exact) {
-            const uint2 c = group_codes_settle(xt + h * 1024 + xoff0, xt + h * 1024 + xoff1, il4, q[h].eff, q[h].w0,
-                                               q[h].w1, q[h].d0, q[h].d1);
-            q[h].w0 = c.x;
-            q[h].w1 = c.y;
-          }
+          for (int h = 0; h < 2; ++h)
+            if (q[h].exact) {
+              const uint2 c = group_codes_settle(xt + h * 1024 + xoff0, xt + h * 1024 + xoff1, il4, q[h].eff,
+                                                 q[h].w0, q[h].w1, q[h].d0, q[h].d1);
+              q[h].w0 = c.x;
+              q[h].w1 = c.y;
+            }
+        }
         if (ok0) *reinterpret_cast<uint2 *>(xq_p) = make_uint2(q[0].w0, q[0].w1);
         if (ok1) *reinterpret_cast<uint2 *>(xq_p + 8 * row_bytes) = make_uint2(q[1].w0, q[1].w1);
         xs_p[0] = static_cast<uint8_t>(q[0].sc);
