@@ -13,7 +13,8 @@
 // step this stages 32 KiB of operands for 512 tensor-core cycles; a one-CTA tile of 128 x 256
 // needs 48 KiB.
 //
-// Per tile the k-loop is a sequence of pipeline steps through a 5-stage shared-memory ring:
+// Per tile the k-loop is a sequence of pipeline steps through a 5-stage shared-memory ring
+// (38 KiB per stage: operands and scale blocks):
 //   - rank / kc low-rank steps, kc = min(rank, 32): per CTA the hi and lo planes of lora_act
 //     (128 x kc bf16 each) and half of an L2t tile (128 x kc bf16); bf16 MMAs (K = 16 each),
 //     hi and lo against the same L2t tile;
@@ -22,21 +23,26 @@
 // All steps accumulate into one fp32 accumulator. lora_act arrives pre-divided by
 // alpha = s_x s_w, so the output stage computes Y = bf16(alpha * acc + bias) for every element.
 //
-// Scale factors reach tensor memory through registers: tcgen05.st moves them several times
-// faster than the tensor-memory copy unit, which has to replicate every 512-byte block four
-// times. Eight warps per CTA, two per 32-lane sub-partition, each own two of a step's four
-// k-blocks: they load the 16-byte lines of the step's scale blocks from global memory (L2) two
-// steps ahead and write them with tcgen05.st in the replicated layout the block-scaled MMA reads
-// (lane i of every sub-partition holds rows i, i+32, i+64, i+96 of a block, one 32-bit column
-// each). A CTA holds the activation scales of its own 128 rows and the weight scales of all 256
-// rows of the tile, since its half of the MMA multiplies its rows by the whole of B.
+// Scale factors reach tensor memory through shared memory and registers. With each 4-bit step
+// the producer bulk-copies three 2 KiB scale blocks into the stage (the CTA's activation block
+// and the tile's two weight blocks, four k-blocks each), signalled on a per-stage sffull barrier;
+// eight warps per CTA, two per 32-lane sub-partition, each owning two of a step's four k-blocks,
+// read the lines and write them with tcgen05.st in the replicated layout the block-scaled MMA
+// reads (lane i of every sub-partition holds rows i, i+32, i+64, i+96 of a block, one 32-bit
+// column each). tcgen05.st moves them several times faster than the tensor-memory copy unit,
+// which has to replicate every 512-byte block four times; staging the blocks with the stage
+// gives them the ring's whole latency tolerance (loaded from L2 by the writers themselves, two
+// steps ahead, they set the kernel's pace: a scratch copy without those loads ran 35% faster).
+// A CTA holds the activation scales of its own 128 rows and the weight scales of all 256 rows of
+// the tile, since its half of the MMA multiplies its rows by the whole of B.
 //
 // Warp roles (576 threads per CTA): warp 0 TMA producer; warp 1 tensor-memory owner and, in the
 // even CTA, MMA issuer; warps 2..9 scale-factor writers;
 // warps 10..17 output stage (warp w reaches lanes 32 (w % 4).. and drains columns
-// 128 ((w - 10) / 4)..). The output stage drains the
-// accumulator into a swizzled bf16 tile in shared memory, releases the accumulator, and writes
-// the tile with TMA stores (which clip the M / N edges).
+// 128 ((w - 10) / 4)..). The output stage drains the accumulator into a swizzled bf16 box in
+// shared memory (one box of 64 columns per half, filled twice per tile), releases the
+// accumulator once all its chunks are in registers, and writes the boxes with TMA stores (which
+// clip the M / N edges).
 //
 // Synchronisation across the pair. Every barrier the MMA issuer waits on lives in the even CTA,
 // and it waits on one per step and one per tile: each barrier result the issuing thread consumes
@@ -60,10 +66,14 @@ constexpr int BNH = BN / 2;  // rows of W staged per CTA
 constexpr int STAGES = 5;
 constexpr uint32_t A_BYTES = BM * 128u;
 constexpr uint32_t B_BYTES = BNH * 128u;
-constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES;  // 32 KiB
-constexpr uint32_t SF_BLOCK = 512;                   // scale bytes of 128 rows x 64 elements of K
+constexpr uint32_t SF_BLOCK = 512;  // scale bytes of 128 rows x 64 elements of K
+// per 4-bit step: the CTA's activation scale block and the tile's two weight scale blocks
+// (rows 0-127, 128-255), four k-blocks each, bulk-copied with the stage
+constexpr uint32_t SF_OFF = A_BYTES + B_BYTES;
+constexpr uint32_t SF_STAGE_BYTES = 3 * 4 * SF_BLOCK;                 // 6 KiB
+constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SF_STAGE_BYTES;  // 38 KiB
 constexpr uint32_t DATA_BYTES = STAGES * STAGE_BYTES;
-constexpr uint32_t YST_BYTES = BM * BN * 2;  // bf16 output staging: 4 boxes of 128 rows x 64 columns
+constexpr uint32_t YST_BYTES = BM * 64 * 2 * 2;  // bf16 output staging: one box of 128 rows x 64 columns per half
 constexpr uint32_t BIAS_BYTES = BN * 4;
 constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM = DATA_BYTES + YST_BYTES + BIAS_BYTES + BAR_BYTES + 1024;
@@ -79,7 +89,7 @@ constexpr uint32_t SF_WARPS = 8;
 constexpr uint32_t EPI_WARPS = 8;
 constexpr uint32_t FULL_COUNT = 1 + 2 * SF_WARPS;
 constexpr uint32_t ACCEMPTY_COUNT = 2 * EPI_WARPS;
-constexpr int N_BARS = 2 * STAGES + 2;
+constexpr int N_BARS = 3 * STAGES + 2;
 static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1 KiB alignment of 128B-swizzled tiles");
 static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "scale slots exceed the tensor memory");
 static_assert(SMEM <= 232448, "shared memory per CTA");
@@ -125,6 +135,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t bar_empty = bar_full + 8 * STAGES;
   const uint32_t bar_accfull = bar_empty + 8 * STAGES;
   const uint32_t bar_accempty = bar_accfull + 8;
+  // sffull[s]: the stage's scale blocks have landed in this CTA (and, by the producer's order,
+  // the MMAs that last read slot s are done)
+  const uint32_t bar_sf = bar_accempty + 8;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + N_BARS);
 
   const int warp = threadIdx.x >> 5;
@@ -147,6 +160,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(bar_accfull, 1);
     mbar_init(bar_accempty, ACCEMPTY_COUNT);
+    for (int s = 0; s < STAGES; ++s) mbar_init(bar_sf + 8 * s, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -192,13 +206,26 @@ __global__ void __launch_bounds__(THREADS, 1)
           const uint32_t at = smem_u32(a_tile(s));
           const uint32_t bt = smem_u32(b_tile(s));
           if (j < N_LORA) {
+            mbar_arrive(bar_sf + 8 * s);  // no scales for a low-rank step; the phase still advances
             if (crank == 0) mbar_arrive_expect_tx(fb, 2 * (2 * LORA_A_BYTES + LORA_B_BYTES));
             tma_load_2d_pair(at, &tm_la, j * KC, row0, fb_lead);
             tma_load_2d_pair(at + LORA_LO_OFF, &tm_la, RANK + j * KC, row0, fb_lead);
             tma_load_2d_pair(bt, &tm_l2, j * KC, wrow0, fb_lead);
           } else {
             const int kt = j - N_LORA;
-            if (crank == 0) mbar_arrive_expect_tx(fb, 2 * STAGE_BYTES);
+            const int kbv = min(4, kblocks - 4 * kt);
+            const int mb = 2 * mt + static_cast<int>(crank);  // this CTA's 128-row block of X
+            const bool rows_ok = mb * BM < a.M;               // activation scales cover ceil(M / 128) blocks
+            const uint32_t sfb = bar_sf + 8 * s;
+            const uint32_t blk = static_cast<uint32_t>(kbv) * SF_BLOCK;
+            mbar_arrive_expect_tx(sfb, (rows_ok ? 3u : 2u) * blk);
+            if (rows_ok)
+              bulk_load(at + SF_OFF, a.xs + (static_cast<size_t>(mb) * kblocks + 4 * kt) * SF_BLOCK, blk, sfb);
+            bulk_load(at + SF_OFF + 4 * SF_BLOCK, a.ws + (static_cast<size_t>(2 * nt) * kblocks + 4 * kt) * SF_BLOCK,
+                      blk, sfb);
+            bulk_load(at + SF_OFF + 8 * SF_BLOCK,
+                      a.ws + (static_cast<size_t>(2 * nt + 1) * kblocks + 4 * kt) * SF_BLOCK, blk, sfb);
+            if (crank == 0) mbar_arrive_expect_tx(fb, 2 * (A_BYTES + B_BYTES));
             tma_load_2d_pair(at, &tm_xq, kt * 128, row0, fb_lead);
             tma_load_2d_pair(bt, &tm_wq, kt * 128, wrow0, fb_lead);
           }
@@ -274,70 +301,50 @@ __global__ void __launch_bounds__(THREADS, 1)
   } else if (warp < EPI_WARP0) {
     // ------------------------------------------------------------ scale-factor writers
     // Warp (q, h) writes tensor-memory lanes 32 q .. 32 q + 31 for k-blocks 2 h and 2 h + 1 of
-    // every step: lane i stores the 16-byte line i of the CTA's activation block (4 columns) and
-    // of the tile's two weight blocks (8 columns) of each k-block. Loads run two steps ahead.
-    // Every step (low-rank ones too) is announced on the even CTA's full barrier, once per warp.
+    // every step: lane i moves the 16-byte line i of the CTA's activation block (4 columns) and of
+    // the tile's two weight blocks (8 columns) of each k-block from the stage's scale region into
+    // the step's slot. Every step (low-rank ones too) is announced on the even CTA's full
+    // barrier, once per warp.
     const int h = (warp - SF_WARP0) >> 2;
     const uint32_t full_lead = map_shared_rank(bar_full, 0);
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int my_tiles = tiles > pid ? (tiles - 1 - pid) / npairs + 1 : 0;
     const int nsteps = my_tiles * total;
-    struct Lines {
-      uint32_t sa[8];   // activation words of k-blocks 2h, 2h + 1
-      uint32_t sb[16];  // weight words: k-block 2h rows 0-127, 128-255, then k-block 2h + 1
-    };
-    auto load = [&](int step, Lines &b) {
-      if (step >= nsteps) return;
-      const int j = step % total;
-      if (!FP4 || j < N_LORA) return;
-      const int t = pid + (step / total) * npairs;
-      const int mt = t % a.Mt, nt = t / a.Mt;
-      const int kt = j - N_LORA;
-      const int kbv = min(4, kblocks - 4 * kt);
-      const int mb = 2 * mt + static_cast<int>(crank);  // this CTA's 128-row block of X
-      const bool rows_ok = mb * BM < a.M;               // activation scales cover ceil(M / 128) blocks
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int kb = 2 * h + e;
-        uint4 va = make_uint4(0, 0, 0, 0), v0 = va, v1 = va;
-        if (kb < kbv) {
-          const size_t k0 = static_cast<size_t>(4 * kt + kb) * SF_BLOCK + lane * 16;
-          if (rows_ok) va = __ldg(reinterpret_cast<const uint4 *>(a.xs + static_cast<size_t>(mb) * kblocks * SF_BLOCK + k0));
-          v0 = __ldg(reinterpret_cast<const uint4 *>(a.ws + static_cast<size_t>(2 * nt) * kblocks * SF_BLOCK + k0));
-          v1 = __ldg(reinterpret_cast<const uint4 *>(a.ws + static_cast<size_t>(2 * nt + 1) * kblocks * SF_BLOCK + k0));
-        }
-        b.sa[4 * e + 0] = va.x; b.sa[4 * e + 1] = va.y; b.sa[4 * e + 2] = va.z; b.sa[4 * e + 3] = va.w;
-        b.sb[8 * e + 0] = v0.x; b.sb[8 * e + 1] = v0.y; b.sb[8 * e + 2] = v0.z; b.sb[8 * e + 3] = v0.w;
-        b.sb[8 * e + 4] = v1.x; b.sb[8 * e + 5] = v1.y; b.sb[8 * e + 6] = v1.z; b.sb[8 * e + 7] = v1.w;
-      }
-    };
-    auto put = [&](int step, const Lines &b) -> bool {
+    for (int step = 0; step < nsteps; ++step) {
       const int s = step % STAGES;
-      bool ok = true;
-      if (step >= STAGES) ok = mbar_wait(bar_empty + 8 * s, ((step / STAGES) - 1) & 1, a.err, KID_GEMM, 6);
-      if (!__all_sync(0xffffffffu, ok)) return false;
-      if (FP4 && step % total >= N_LORA) {
+      const int j = step % total;
+      // sffull of this step: its scale blocks are in shared memory and slot s is free
+      if (!__all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * s, (step / STAGES) & 1, a.err, KID_GEMM, 6))) break;
+      if (FP4 && j >= N_LORA) {
+        const int t = pid + (step / total) * npairs;
+        const int mt = t % a.Mt;
+        const int kt = j - N_LORA;
+        const int kbv = min(4, kblocks - 4 * kt);
+        const bool rows_ok = (2 * mt + static_cast<int>(crank)) * BM < a.M;
+        const uint32_t sft = smem_u32(a_tile(s)) + SF_OFF + lane * 16;
+        uint32_t sa[8], sb[16];
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int kb = 2 * h + e;
+          uint4 va = make_uint4(0, 0, 0, 0), v0 = va, v1 = va;
+          if (kb < kbv) {
+            if (rows_ok) va = ld_shared_u32x4(sft + kb * SF_BLOCK);
+            v0 = ld_shared_u32x4(sft + (4 + kb) * SF_BLOCK);
+            v1 = ld_shared_u32x4(sft + (8 + kb) * SF_BLOCK);
+          }
+          sa[4 * e + 0] = va.x; sa[4 * e + 1] = va.y; sa[4 * e + 2] = va.z; sa[4 * e + 3] = va.w;
+          sb[8 * e + 0] = v0.x; sb[8 * e + 1] = v0.y; sb[8 * e + 2] = v0.z; sb[8 * e + 3] = v0.w;
+          sb[8 * e + 4] = v1.x; sb[8 * e + 5] = v1.y; sb[8 * e + 6] = v1.z; sb[8 * e + 7] = v1.w;
+        }
         // slot columns: SFA k-block kb at 4 kb, SFB k-block kb at 16 + 8 kb (rows 0-127, then 128-255)
         const uint32_t tsf = tbase + lane_base + SF_COL0 + SF_COLS * s;
-        tmem_st8(tsf + 8 * h, b.sa);
-        tmem_st16(tsf + 16 + 16 * h, b.sb);
+        tmem_st8(tsf + 8 * h, sa);
+        tmem_st16(tsf + 16 + 16 * h, sb);
         tmem_wait_st();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_remote(full_lead + 8 * s);
-      return true;
-    };
-    Lines b0, b1, b2;
-    load(0, b0);
-    load(1, b1);
-    for (int step = 0; step < nsteps; step += 3) {
-      load(step + 2, b2);
-      if (!put(step, b0) || step + 1 >= nsteps) break;
-      load(step + 3, b0);
-      if (!put(step + 1, b1) || step + 2 >= nsteps) break;
-      load(step + 4, b1);
-      if (!put(step + 2, b2)) break;
     }
   } else {
     // ------------------------------------------------------------ output stage
@@ -360,8 +367,37 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int row0 = mt * BMP + static_cast<int>(crank) * BM;
       const int m = row0 + row;
       if constexpr (!ADD_Y) {
-        // the group's previous TMA stores have finished reading the staging tile, and its
-        // threads are done with the previous bias values
+        // The group owns one staging box (128 rows x 64 columns, 16-byte chunk k of row r at
+        // k ^ (r % 8)) and fills it twice per tile: columns 0-63 of its half, then 64-127.
+        // The accumulator is released as soon as all four 32-column chunks are in registers.
+        uint8_t *rowp = ystage + half * (BM * 128) + row * 128;
+        auto convert_store = [&](const uint32_t(&v32)[32], int colh) {
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int ch = ((colh & 63) >> 3) + q;
+            const float4 b0 = *reinterpret_cast<const float4 *>(bias_s + half * 128 + colh + 8 * q);
+            const float4 b1 = *reinterpret_cast<const float4 *>(bias_s + half * 128 + colh + 8 * q + 4);
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(v32[8 * q + e]);
+            const uint32_t p0 = pack_bf16x2(fmaf(a.alpha, v[0], b0.x), fmaf(a.alpha, v[1], b0.y));
+            const uint32_t p1 = pack_bf16x2(fmaf(a.alpha, v[2], b0.z), fmaf(a.alpha, v[3], b0.w));
+            const uint32_t p2 = pack_bf16x2(fmaf(a.alpha, v[4], b1.x), fmaf(a.alpha, v[5], b1.y));
+            const uint32_t p3 = pack_bf16x2(fmaf(a.alpha, v[6], b1.z), fmaf(a.alpha, v[7], b1.w));
+            *reinterpret_cast<uint4 *>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(p0, p1, p2, p3);
+          }
+        };
+        auto store_box = [&](int colh) {
+          fence_proxy_async_smem();
+          named_bar_sync(1 + half, 128);
+          if (et == 0) {
+            if (row0 < a.M && n0 + half * 128 + colh < a.N)
+              tma_store_2d(&tm_y, smem_u32(ystage + half * (BM * 128)), n0 + half * 128 + colh, row0);
+            bulk_commit();
+          }
+        };
+        // the group's previous TMA store has finished reading the box, and its threads are done
+        // with the previous bias values
         if (et == 0) bulk_wait_read0();
         {
           const int e = half * 128 + et;
@@ -370,55 +406,35 @@ __global__ void __launch_bounds__(THREADS, 1)
         named_bar_sync(1 + half, 128);
         if (ok) ok = mbar_wait_parked(bar_accfull, tcount & 1, a.err, KID_GEMM, 4);
         ok = __all_sync(0xffffffffu, ok);
+        uint32_t r0[32], r1[32];
         if (ok) {
           tc_fence_after();
-          uint32_t r0[32], r1[32];
           tmem_ld32(taddr, r0);
+          tmem_ld32(taddr + 32, r1);
           tmem_wait_ld_dep(r0);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t(&cur)[32] = (c & 1) ? r1 : r0;
-            uint32_t(&nxt)[32] = (c & 1) ? r0 : r1;
-            if (c + 1 < 4) {
-              tmem_ld32(taddr + (c + 1) * 32, nxt);
-            } else {
-              // every column of this warp's rows has been read: release the accumulator
-              tc_fence_before();
-              __syncwarp();
-              if (lane == 0) mbar_arrive_remote(accempty_lead);
-            }
-            // box (col0 / 64) holds 128 rows of 128 bytes, 16-byte chunk k of row r at k ^ (r % 8)
-            const int col0 = half * 128 + c * 32;
-            uint8_t *rowp = ystage + (col0 >> 6) * (BM * 128) + row * 128;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const int ch = ((col0 & 63) >> 3) + q;
-              const float4 b0 = *reinterpret_cast<const float4 *>(bias_s + col0 + 8 * q);
-              const float4 b1 = *reinterpret_cast<const float4 *>(bias_s + col0 + 8 * q + 4);
-              float v[8];
-#pragma unroll
-              for (int e = 0; e < 8; ++e) v[e] = __uint_as_float(cur[8 * q + e]);
-              const uint32_t p0 = pack_bf16x2(fmaf(a.alpha, v[0], b0.x), fmaf(a.alpha, v[1], b0.y));
-              const uint32_t p1 = pack_bf16x2(fmaf(a.alpha, v[2], b0.z), fmaf(a.alpha, v[3], b0.w));
-              const uint32_t p2 = pack_bf16x2(fmaf(a.alpha, v[4], b1.x), fmaf(a.alpha, v[5], b1.y));
-              const uint32_t p3 = pack_bf16x2(fmaf(a.alpha, v[6], b1.z), fmaf(a.alpha, v[7], b1.w));
-              *reinterpret_cast<uint4 *>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(p0, p1, p2, p3);
-            }
-            if (c + 1 < 4) tmem_wait_ld_dep(nxt);
-          }
+          tmem_wait_ld_dep(r1);
+          convert_store(r0, 0);
+          convert_store(r1, 32);
+          tmem_ld32(taddr + 64, r0);
+          tmem_ld32(taddr + 96, r1);
         }
-        fence_proxy_async_smem();
+        store_box(0);
+        if (ok) {
+          tmem_wait_ld_dep(r0);
+          tmem_wait_ld_dep(r1);
+          // every column of this warp's rows has been read: release the accumulator
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_remote(accempty_lead);
+        }
+        // the first store has finished reading the box
+        if (et == 0) bulk_wait_read0();
         named_bar_sync(1 + half, 128);
-        if (et == 0) {
-          if (row0 < a.M) {
-            for (int b = 0; b < 2; ++b) {
-              const int box = half * 2 + b;
-              if (n0 + 64 * box < a.N)
-                tma_store_2d(&tm_y, smem_u32(ystage + box * (BM * 128)), n0 + 64 * box, row0);
-            }
-          }
-          bulk_commit();
+        if (ok) {
+          convert_store(r0, 64);
+          convert_store(r1, 96);
         }
+        store_box(64);
       } else {
         // Unfused up-projection: Y = bf16(Y + alpha * acc), one 32-column chunk at a time.
         if (ok) ok = mbar_wait_parked(bar_accfull, tcount & 1, a.err, KID_GEMM, 4);
