@@ -80,9 +80,16 @@ constexpr uint32_t SMEM = DATA_BYTES + YST_BYTES + BIAS_BYTES + BAR_BYTES + 1024
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = 256;  // one scale slot per stage follows the accumulator
 constexpr uint32_t SF_COLS = 48;   // per slot: 4 k-blocks x (4 SFA + 8 SFB) columns
-constexpr int SF_WARP0 = 2;
-constexpr int EPI_WARP0 = 10;
-constexpr int THREADS = 576;
+// 20 warps = 5 warpgroups (registers are reallocated per warpgroup): warp 0 producer, warp 1
+// MMA issuer, warps 2..7 and 16..17 scale writers (two per tensor-memory sub-partition), warps
+// 8..15 output stage (warpgroups 2 and 3), warps 18..19 idle.
+constexpr int EPI_WARP0 = 8;
+constexpr int THREADS = 640;
+// Registers per thread after reallocation: the output warpgroups hold a row's whole 128-column
+// accumulator slice (4 x 32 fp32) before releasing it; the others need few.
+constexpr uint32_t EPI_REGS = 168;
+constexpr uint32_t OTHER_REGS = 48;
+constexpr uint32_t REG_POOL_NEEDED = 32u * (8u * EPI_REGS + 12u * OTHER_REGS);  // per CTA
 // Arrivals the MMA issuer waits for, besides the producer's: one per scale-writer warp and one
 // per output warp, from both CTAs of the pair.
 constexpr uint32_t SF_WARPS = 8;
@@ -175,183 +182,13 @@ __global__ void __launch_bounds__(THREADS, 1)
   grid_dep_wait();
   grid_dep_launch();
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
-      if (FP4) {
-        tma_prefetch_desc(&tm_xq);
-        tma_prefetch_desc(&tm_wq);
-      }
-      if (RANK) {
-        tma_prefetch_desc(&tm_la);
-        tma_prefetch_desc(&tm_l2);
-      }
-      uint32_t it = 0;
-      bool ok = true;
-      for (int t = pid; t < tiles && ok; t += npairs) {
-        const int mt = t % a.Mt;
-        const int nt = t / a.Mt;
-        const int row0 = mt * BMP + static_cast<int>(crank) * BM;  // this CTA's rows of X
-        const int wrow0 = nt * BN + static_cast<int>(crank) * BNH;  // this CTA's rows of W
-        for (int j = 0; j < total; ++j, ++it) {
-          const int s = it % STAGES;
-          // spin rather than park: a parked thread wakes measurably later, and this round trip
-          // (slot released -> loads issued -> stage full) is the kernel's critical path
-          if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1, a.err, KID_GEMM, 1)) {
-            ok = false;
-            break;
-          }
-          const uint32_t fb = bar_full + 8 * s;
-          const uint32_t fb_lead = map_shared_rank(fb, 0);
-          const uint32_t at = smem_u32(a_tile(s));
-          const uint32_t bt = smem_u32(b_tile(s));
-          if (j < N_LORA) {
-            mbar_arrive(bar_sf + 8 * s);  // no scales for a low-rank step; the phase still advances
-            if (crank == 0) mbar_arrive_expect_tx(fb, 2 * (2 * LORA_A_BYTES + LORA_B_BYTES));
-            tma_load_2d_pair(at, &tm_la, j * KC, row0, fb_lead);
-            tma_load_2d_pair(at + LORA_LO_OFF, &tm_la, RANK + j * KC, row0, fb_lead);
-            tma_load_2d_pair(bt, &tm_l2, j * KC, wrow0, fb_lead);
-          } else {
-            const int kt = j - N_LORA;
-            const int kbv = min(4, kblocks - 4 * kt);
-            const int mb = 2 * mt + static_cast<int>(crank);  // this CTA's 128-row block of X
-            const bool rows_ok = mb * BM < a.M;               // activation scales cover ceil(M / 128) blocks
-            const uint32_t sfb = bar_sf + 8 * s;
-            const uint32_t blk = static_cast<uint32_t>(kbv) * SF_BLOCK;
-            mbar_arrive_expect_tx(sfb, (rows_ok ? 3u : 2u) * blk);
-            if (rows_ok)
-              bulk_load(at + SF_OFF, a.xs + (static_cast<size_t>(mb) * kblocks + 4 * kt) * SF_BLOCK, blk, sfb);
-            bulk_load(at + SF_OFF + 4 * SF_BLOCK, a.ws + (static_cast<size_t>(2 * nt) * kblocks + 4 * kt) * SF_BLOCK,
-                      blk, sfb);
-            bulk_load(at + SF_OFF + 8 * SF_BLOCK,
-                      a.ws + (static_cast<size_t>(2 * nt + 1) * kblocks + 4 * kt) * SF_BLOCK, blk, sfb);
-            if (crank == 0) mbar_arrive_expect_tx(fb, 2 * (A_BYTES + B_BYTES));
-            tma_load_2d_pair(at, &tm_xq, kt * 128, row0, fb_lead);
-            tma_load_2d_pair(bt, &tm_wq, kt * 128, wrow0, fb_lead);
-          }
-        }
-      }
-      // The MMA issuer's last commits to this CTA's empty barriers have landed before it exits.
-      for (uint32_t i = it > STAGES ? it - STAGES : 0; ok && i < it; ++i)
-        ok = mbar_wait(bar_empty + 8 * (i % STAGES), (i / STAGES) & 1, a.err, KID_GEMM, 7);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (even CTA)
-    // The whole warp runs the loops, so the descriptor arithmetic stays warp-uniform (no
-    // per-instruction register moves); one elected lane issues the MMAs and their commits.
-    if (crank == 0) {
-      // kind::mxf4nvf4: A, B e2m1 (bits 7-9, 10-12 = 1), K-major, N = 256 (bits 17-22),
-      // scale type ue4m3 (bit 23 = 0), M = 256 across the pair (bits 24-28), scale ids 0, K = 64.
-      const uint32_t idesc_fp4 = (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BMP) >> 4) << 24);
-      // kind::f16: D fp32, A, B bf16, N = 256, M = 256 across the pair.
-      const uint32_t idesc_bf16 =
-          (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BMP) >> 4) << 24);
-      uint32_t it = 0;
-      uint32_t tcount = 0;
-      bool ok = true;
-      for (int t = pid; t < tiles && ok; t += npairs, ++tcount) {
-        if (tcount > 0 && !__all_sync(0xffffffffu, mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 2))) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        for (int j = 0; j < total; ++j, ++it) {
-          const int s = it % STAGES;
-          const uint32_t par = (it / STAGES) & 1;
-          if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, par, a.err, KID_GEMM, 3))) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t st = smem_u32(a_tile(s));
-          if (j < N_LORA) {
-            const uint64_t ad = umma_desc(st, 16, 8 * LORA_ROW, LORA_SWZ);
-            const uint64_t ald = umma_desc(st + LORA_LO_OFF, 16, 8 * LORA_ROW, LORA_SWZ);
-            const uint64_t bd = umma_desc(st + A_BYTES, 16, 8 * LORA_ROW, LORA_SWZ);
-            if (elect_one()) {
-#pragma unroll
-              for (int k = 0; k < KC / 16; ++k) {
-                mma_bf16_pair(tbase, ad + 2u * k, bd + 2u * k, idesc_bf16, (j | k) != 0 ? 1u : 0u);
-                mma_bf16_pair(tbase, ald + 2u * k, bd + 2u * k, idesc_bf16, 1u);
-              }
-              tc_commit_pair_mc(bar_empty + 8 * s, 0x3);
-            }
-          } else {
-            const int kt = j - N_LORA;
-            const int kbv = min(4, kblocks - 4 * kt);
-            const uint32_t tsf = tbase + SF_COL0 + SF_COLS * s;
-            const uint64_t ad = umma_desc(st, 16, 1024, 2);
-            const uint64_t bd = umma_desc(st + A_BYTES, 16, 1024, 2);
-            if (elect_one()) {
-              for (int kb = 0; kb < kbv; ++kb)
-                mma_nvfp4_pair(tbase, ad + 2u * kb, bd + 2u * kb, idesc_fp4, tsf + 4 * kb, tsf + 16 + 8 * kb,
-                               (j | kb) != 0 ? 1u : 0u);
-              tc_commit_pair_mc(bar_empty + 8 * s, 0x3);
-            }
-          }
-          __syncwarp();
-        }
-        if (!ok) break;
-        if (elect_one()) tc_commit_pair_mc(bar_accfull, 0x3);
-        __syncwarp();
-      }
-      // both CTAs' output stages have released the last accumulator
-      if (ok && tcount > 0) mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 8);
-    }
-  } else if (warp < EPI_WARP0) {
-    // ------------------------------------------------------------ scale-factor writers
-    // Warp (q, h) writes tensor-memory lanes 32 q .. 32 q + 31 for k-blocks 2 h and 2 h + 1 of
-    // every step: lane i moves the 16-byte line i of the CTA's activation block (4 columns) and of
-    // the tile's two weight blocks (8 columns) of each k-block from the stage's scale region into
-    // the step's slot. Every step (low-rank ones too) is announced on the even CTA's full
-    // barrier, once per warp.
-    const int h = (warp - SF_WARP0) >> 2;
-    const uint32_t full_lead = map_shared_rank(bar_full, 0);
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const int my_tiles = tiles > pid ? (tiles - 1 - pid) / npairs + 1 : 0;
-    const int nsteps = my_tiles * total;
-    for (int step = 0; step < nsteps; ++step) {
-      const int s = step % STAGES;
-      const int j = step % total;
-      // sffull of this step: its scale blocks are in shared memory and slot s is free
-      if (!__all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * s, (step / STAGES) & 1, a.err, KID_GEMM, 6))) break;
-      if (FP4 && j >= N_LORA) {
-        const int t = pid + (step / total) * npairs;
-        const int mt = t % a.Mt;
-        const int kt = j - N_LORA;
-        const int kbv = min(4, kblocks - 4 * kt);
-        const bool rows_ok = (2 * mt + static_cast<int>(crank)) * BM < a.M;
-        const uint32_t sft = smem_u32(a_tile(s)) + SF_OFF + lane * 16;
-        uint32_t sa[8], sb[16];
-#pragma unroll
-        for (int e = 0; e < 2; ++e) {
-          const int kb = 2 * h + e;
-          uint4 va = make_uint4(0, 0, 0, 0), v0 = va, v1 = va;
-          if (kb < kbv) {
-            if (rows_ok) va = ld_shared_u32x4(sft + kb * SF_BLOCK);
-            v0 = ld_shared_u32x4(sft + (4 + kb) * SF_BLOCK);
-            v1 = ld_shared_u32x4(sft + (8 + kb) * SF_BLOCK);
-          }
-          sa[4 * e + 0] = va.x; sa[4 * e + 1] = va.y; sa[4 * e + 2] = va.z; sa[4 * e + 3] = va.w;
-          sb[8 * e + 0] = v0.x; sb[8 * e + 1] = v0.y; sb[8 * e + 2] = v0.z; sb[8 * e + 3] = v0.w;
-          sb[8 * e + 4] = v1.x; sb[8 * e + 5] = v1.y; sb[8 * e + 6] = v1.z; sb[8 * e + 7] = v1.w;
-        }
-        // slot columns: SFA k-block kb at 4 kb, SFB k-block kb at 16 + 8 kb (rows 0-127, then 128-255)
-        const uint32_t tsf = tbase + lane_base + SF_COL0 + SF_COLS * s;
-        tmem_st8(tsf + 8 * h, sa);
-        tmem_st16(tsf + 16 + 16 * h, sb);
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_remote(full_lead + 8 * s);
-    }
-  } else {
+  if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 8) {
+    setmaxnreg_inc<EPI_REGS>();
     // ------------------------------------------------------------ output stage
     // Two groups of four warps (named barriers 1 and 2), one per 128-column half of the tile;
-    // the warps of a group cover the four 32-lane sub-partitions. Thread (row, half) drains
-    // columns 128 half .. 128 half + 127 of its row in four 32-column chunks, the load of chunk
-    // c + 1 in flight while chunk c is converted.
+    // the warps of a group cover the four 32-lane sub-partitions. Thread (row, half) loads
+    // columns 128 half .. 128 half + 127 of its row (four 32-column chunks) into registers,
+    // releases the accumulator to the next tile's MMAs, then converts and stores them.
     const int half = (warp - EPI_WARP0) >> 2;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
@@ -406,33 +243,31 @@ __global__ void __launch_bounds__(THREADS, 1)
         named_bar_sync(1 + half, 128);
         if (ok) ok = mbar_wait_parked(bar_accfull, tcount & 1, a.err, KID_GEMM, 4);
         ok = __all_sync(0xffffffffu, ok);
-        uint32_t r0[32], r1[32];
+        uint32_t r0[32], r1[32], r2[32], r3[32];
         if (ok) {
           tc_fence_after();
           tmem_ld32(taddr, r0);
           tmem_ld32(taddr + 32, r1);
+          tmem_ld32(taddr + 64, r2);
+          tmem_ld32(taddr + 96, r3);
           tmem_wait_ld_dep(r0);
           tmem_wait_ld_dep(r1);
-          convert_store(r0, 0);
-          convert_store(r1, 32);
-          tmem_ld32(taddr + 64, r0);
-          tmem_ld32(taddr + 96, r1);
-        }
-        store_box(0);
-        if (ok) {
-          tmem_wait_ld_dep(r0);
-          tmem_wait_ld_dep(r1);
-          // every column of this warp's rows has been read: release the accumulator
+          tmem_wait_ld_dep(r2);
+          tmem_wait_ld_dep(r3);
+          // every column of this warp's rows is in registers: release the accumulator
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_remote(accempty_lead);
+          convert_store(r0, 0);
+          convert_store(r1, 32);
         }
+        store_box(0);
         // the first store has finished reading the box
         if (et == 0) bulk_wait_read0();
         named_bar_sync(1 + half, 128);
         if (ok) {
-          convert_store(r0, 64);
-          convert_store(r1, 96);
+          convert_store(r2, 64);
+          convert_store(r3, 96);
         }
         store_box(64);
       } else {
@@ -469,6 +304,180 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     }
     if (!ADD_Y && et == 0) bulk_wait0();  // stores complete before the CTA exits
+  } else {
+    setmaxnreg_dec<OTHER_REGS>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer (both CTAs)
+      if (lane == 0) {
+        if (FP4) {
+          tma_prefetch_desc(&tm_xq);
+          tma_prefetch_desc(&tm_wq);
+        }
+        if (RANK) {
+          tma_prefetch_desc(&tm_la);
+          tma_prefetch_desc(&tm_l2);
+        }
+        uint32_t it = 0;
+        bool ok = true;
+        for (int t = pid; t < tiles && ok; t += npairs) {
+          const int mt = t % a.Mt;
+          const int nt = t / a.Mt;
+          const int row0 = mt * BMP + static_cast<int>(crank) * BM;  // this CTA's rows of X
+          const int wrow0 = nt * BN + static_cast<int>(crank) * BNH;  // this CTA's rows of W
+          for (int j = 0; j < total; ++j, ++it) {
+            const int s = it % STAGES;
+            // spin rather than park: a parked thread wakes measurably later, and this round trip
+            // (slot released -> loads issued -> stage full) is the kernel's critical path
+            if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1, a.err, KID_GEMM, 1)) {
+              ok = false;
+              break;
+            }
+            const uint32_t fb = bar_full + 8 * s;
+            const uint32_t fb_lead = map_shared_rank(fb, 0);
+            const uint32_t at = smem_u32(a_tile(s));
+            const uint32_t bt = smem_u32(b_tile(s));
+            if (j < N_LORA) {
+              mbar_arrive(bar_sf + 8 * s);  // no scales for a low-rank step; the phase still advances
+              if (crank == 0) mbar_arrive_expect_tx(fb, 2 * (2 * LORA_A_BYTES + LORA_B_BYTES));
+              tma_load_2d_pair(at, &tm_la, j * KC, row0, fb_lead);
+              tma_load_2d_pair(at + LORA_LO_OFF, &tm_la, RANK + j * KC, row0, fb_lead);
+              tma_load_2d_pair(bt, &tm_l2, j * KC, wrow0, fb_lead);
+            } else {
+              const int kt = j - N_LORA;
+              const int kbv = min(4, kblocks - 4 * kt);
+              const int mb = 2 * mt + static_cast<int>(crank);  // this CTA's 128-row block of X
+              const bool rows_ok = mb * BM < a.M;               // activation scales cover ceil(M / 128) blocks
+              const uint32_t sfb = bar_sf + 8 * s;
+              const uint32_t blk = static_cast<uint32_t>(kbv) * SF_BLOCK;
+              mbar_arrive_expect_tx(sfb, (rows_ok ? 3u : 2u) * blk);
+              if (rows_ok)
+                bulk_load(at + SF_OFF, a.xs + (static_cast<size_t>(mb) * kblocks + 4 * kt) * SF_BLOCK, blk, sfb);
+              bulk_load(at + SF_OFF + 4 * SF_BLOCK, a.ws + (static_cast<size_t>(2 * nt) * kblocks + 4 * kt) * SF_BLOCK,
+                        blk, sfb);
+              bulk_load(at + SF_OFF + 8 * SF_BLOCK,
+                        a.ws + (static_cast<size_t>(2 * nt + 1) * kblocks + 4 * kt) * SF_BLOCK, blk, sfb);
+              if (crank == 0) mbar_arrive_expect_tx(fb, 2 * (A_BYTES + B_BYTES));
+              tma_load_2d_pair(at, &tm_xq, kt * 128, row0, fb_lead);
+              tma_load_2d_pair(bt, &tm_wq, kt * 128, wrow0, fb_lead);
+            }
+          }
+        }
+        // The MMA issuer's last commits to this CTA's empty barriers have landed before it exits.
+        for (uint32_t i = it > STAGES ? it - STAGES : 0; ok && i < it; ++i)
+          ok = mbar_wait(bar_empty + 8 * (i % STAGES), (i / STAGES) & 1, a.err, KID_GEMM, 7);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer (even CTA)
+      // The whole warp runs the loops, so the descriptor arithmetic stays warp-uniform (no
+      // per-instruction register moves); one elected lane issues the MMAs and their commits.
+      if (crank == 0) {
+        // kind::mxf4nvf4: A, B e2m1 (bits 7-9, 10-12 = 1), K-major, N = 256 (bits 17-22),
+        // scale type ue4m3 (bit 23 = 0), M = 256 across the pair (bits 24-28), scale ids 0, K = 64.
+        const uint32_t idesc_fp4 = (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BMP) >> 4) << 24);
+        // kind::f16: D fp32, A, B bf16, N = 256, M = 256 across the pair.
+        const uint32_t idesc_bf16 =
+            (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t(BN) >> 3) << 17) | ((uint32_t(BMP) >> 4) << 24);
+        uint32_t it = 0;
+        uint32_t tcount = 0;
+        bool ok = true;
+        for (int t = pid; t < tiles && ok; t += npairs, ++tcount) {
+          if (tcount > 0 && !__all_sync(0xffffffffu, mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 2))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          for (int j = 0; j < total; ++j, ++it) {
+            const int s = it % STAGES;
+            const uint32_t par = (it / STAGES) & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, par, a.err, KID_GEMM, 3))) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t st = smem_u32(a_tile(s));
+            if (j < N_LORA) {
+              const uint64_t ad = umma_desc(st, 16, 8 * LORA_ROW, LORA_SWZ);
+              const uint64_t ald = umma_desc(st + LORA_LO_OFF, 16, 8 * LORA_ROW, LORA_SWZ);
+              const uint64_t bd = umma_desc(st + A_BYTES, 16, 8 * LORA_ROW, LORA_SWZ);
+              if (elect_one()) {
+  #pragma unroll
+                for (int k = 0; k < KC / 16; ++k) {
+                  mma_bf16_pair(tbase, ad + 2u * k, bd + 2u * k, idesc_bf16, (j | k) != 0 ? 1u : 0u);
+                  mma_bf16_pair(tbase, ald + 2u * k, bd + 2u * k, idesc_bf16, 1u);
+                }
+                tc_commit_pair_mc(bar_empty + 8 * s, 0x3);
+              }
+            } else {
+              const int kt = j - N_LORA;
+              const int kbv = min(4, kblocks - 4 * kt);
+              const uint32_t tsf = tbase + SF_COL0 + SF_COLS * s;
+              const uint64_t ad = umma_desc(st, 16, 1024, 2);
+              const uint64_t bd = umma_desc(st + A_BYTES, 16, 1024, 2);
+              if (elect_one()) {
+                for (int kb = 0; kb < kbv; ++kb)
+                  mma_nvfp4_pair(tbase, ad + 2u * kb, bd + 2u * kb, idesc_fp4, tsf + 4 * kb, tsf + 16 + 8 * kb,
+                                 (j | kb) != 0 ? 1u : 0u);
+                tc_commit_pair_mc(bar_empty + 8 * s, 0x3);
+              }
+            }
+            __syncwarp();
+          }
+          if (!ok) break;
+          if (elect_one()) tc_commit_pair_mc(bar_accfull, 0x3);
+          __syncwarp();
+        }
+        // both CTAs' output stages have released the last accumulator
+        if (ok && tcount > 0) mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 8);
+      }
+    } else if ((warp >= 2 && warp < EPI_WARP0) || warp == 16 || warp == 17) {
+      // ------------------------------------------------------------ scale-factor writers
+      // Warp (q, h) writes tensor-memory lanes 32 q .. 32 q + 31 for k-blocks 2 h and 2 h + 1 of
+      // every step: lane i moves the 16-byte line i of the CTA's activation block (4 columns) and of
+      // the tile's two weight blocks (8 columns) of each k-block from the stage's scale region into
+      // the step's slot. Every step (low-rank ones too) is announced on the even CTA's full
+      // barrier, once per warp.
+      const int h = (warp >= 2 && warp < 6) ? 0 : 1;  // warps 2..5 and 6, 7, 16, 17 each cover the four sub-partitions
+      const uint32_t full_lead = map_shared_rank(bar_full, 0);
+      const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+      const int my_tiles = tiles > pid ? (tiles - 1 - pid) / npairs + 1 : 0;
+      const int nsteps = my_tiles * total;
+      for (int step = 0; step < nsteps; ++step) {
+        const int s = step % STAGES;
+        const int j = step % total;
+        // sffull of this step: its scale blocks are in shared memory and slot s is free
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * s, (step / STAGES) & 1, a.err, KID_GEMM, 6))) break;
+        if (FP4 && j >= N_LORA) {
+          const int t = pid + (step / total) * npairs;
+          const int mt = t % a.Mt;
+          const int kt = j - N_LORA;
+          const int kbv = min(4, kblocks - 4 * kt);
+          const bool rows_ok = (2 * mt + static_cast<int>(crank)) * BM < a.M;
+          const uint32_t sft = smem_u32(a_tile(s)) + SF_OFF + lane * 16;
+          uint32_t sa[8], sb[16];
+  #pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const int kb = 2 * h + e;
+            uint4 va = make_uint4(0, 0, 0, 0), v0 = va, v1 = va;
+            if (kb < kbv) {
+              if (rows_ok) va = ld_shared_u32x4(sft + kb * SF_BLOCK);
+              v0 = ld_shared_u32x4(sft + (4 + kb) * SF_BLOCK);
+              v1 = ld_shared_u32x4(sft + (8 + kb) * SF_BLOCK);
+            }
+            sa[4 * e + 0] = va.x; sa[4 * e + 1] = va.y; sa[4 * e + 2] = va.z; sa[4 * e + 3] = va.w;
+            sb[8 * e + 0] = v0.x; sb[8 * e + 1] = v0.y; sb[8 * e + 2] = v0.z; sb[8 * e + 3] = v0.w;
+            sb[8 * e + 4] = v1.x; sb[8 * e + 5] = v1.y; sb[8 * e + 6] = v1.z; sb[8 * e + 7] = v1.w;
+          }
+          // slot columns: SFA k-block kb at 4 kb, SFB k-block kb at 16 + 8 kb (rows 0-127, then 128-255)
+          const uint32_t tsf = tbase + lane_base + SF_COL0 + SF_COLS * s;
+          tmem_st8(tsf + 8 * h, sa);
+          tmem_st16(tsf + 16 + 16 * h, sb);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_remote(full_lead + 8 * s);
+      }
+    }
   }
 
   __syncthreads();
@@ -492,6 +501,15 @@ int pair_slots(cudaError_t *err) {
   }
   if (cache[dev] > 0) return cache[dev];
   auto kern = k2_gemm_w4a4_lora_up<RANK, FP4, ADD_Y>;
+  // setmaxnreg.inc would wait forever for registers the block was not launched with: the split
+  // must fit the pool of the compiled kernel (registers per thread x threads).
+  cudaFuncAttributes fa;
+  if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess ||
+      static_cast<uint32_t>(fa.numRegs) * THREADS < REG_POOL_NEEDED ||
+      static_cast<uint32_t>(fa.numRegs) > EPI_REGS || static_cast<uint32_t>(fa.numRegs) < OTHER_REGS) {
+    *err = cudaErrorLaunchOutOfResources;
+    return 0;
+  }
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
   if (e != cudaSuccess) {
     *err = e;
