@@ -26,8 +26,8 @@
 // Scale factors reach tensor memory through shared memory and registers. With each 4-bit step
 // the producer bulk-copies three 2 KiB scale blocks into the stage (the CTA's activation block
 // and the tile's two weight blocks, four k-blocks each), signalled on a per-stage sffull barrier;
-// eight warps per CTA, two per 32-lane sub-partition, each owning two of a step's four k-blocks,
-// read the lines and write them with tcgen05.st in the replicated layout the block-scaled MMA
+// eight warps per CTA in two groups of four (one warp per 32-lane sub-partition), the groups taking
+// alternate steps, read the lines and write them with tcgen05.st in the replicated layout the block-scaled MMA
 // reads (lane i of every sub-partition holds rows i, i+32, i+64, i+96 of a block, one 32-bit
 // column each). tcgen05.st moves them several times faster than the tensor-memory copy unit,
 // which has to replicate every 512-byte block four times; staging the blocks with the stage
@@ -36,10 +36,11 @@
 // A CTA holds the activation scales of its own 128 rows and the weight scales of all 256 rows of
 // the tile, since its half of the MMA multiplies its rows by the whole of B.
 //
-// Warp roles (576 threads per CTA): warp 0 TMA producer; warp 1 tensor-memory owner and, in the
-// even CTA, MMA issuer; warps 2..9 scale-factor writers;
-// warps 10..17 output stage (warp w reaches lanes 32 (w % 4).. and drains columns
-// 128 ((w - 10) / 4)..). The output stage drains the accumulator into a swizzled bf16 box in
+// Warp roles (640 threads per CTA): warp 0 TMA producer; warp 1 tensor-memory owner and, in the
+// even CTA, MMA issuer; warps 2..5 (even steps) and 6, 7, 16, 17 (odd steps) scale-factor
+// writers; warps 8..15 output stage (warp w reaches lanes 32 (w % 4).. and drains columns
+// 128 ((w - 8) / 4)..), which take 168 registers a thread from the other warpgroups
+// (setmaxnreg); warps 18, 19 idle. The output stage drains the accumulator into a swizzled bf16 box in
 // shared memory (one box of 64 columns per half, filled twice per tile), releases the
 // accumulator once all its chunks are in registers, and writes the boxes with TMA stores (which
 // clip the M / N edges).
@@ -90,13 +91,13 @@ constexpr int THREADS = 640;
 constexpr uint32_t EPI_REGS = 168;
 constexpr uint32_t OTHER_REGS = 48;
 constexpr uint32_t REG_POOL_NEEDED = 32u * (8u * EPI_REGS + 12u * OTHER_REGS);  // per CTA
-// Arrivals the MMA issuer waits for, besides the producer's: one per scale-writer warp and one
-// per output warp, from both CTAs of the pair.
-constexpr uint32_t SF_WARPS = 8;
+// Arrivals the MMA issuer waits for, besides the producer's: per step one per writer warp of the
+// step's group (four per CTA), per tile one per output warp, from both CTAs of the pair.
+constexpr uint32_t SF_GROUP_WARPS = 4;
 constexpr uint32_t EPI_WARPS = 8;
-constexpr uint32_t FULL_COUNT = 1 + 2 * SF_WARPS;
+constexpr uint32_t FULL_COUNT = 1 + 2 * SF_GROUP_WARPS;
 constexpr uint32_t ACCEMPTY_COUNT = 2 * EPI_WARPS;
-constexpr int N_BARS = 3 * STAGES + 2;
+constexpr int N_BARS = 4 * STAGES + 2;
 static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1 KiB alignment of 128B-swizzled tiles");
 static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "scale slots exceed the tensor memory");
 static_assert(SMEM <= 232448, "shared memory per CTA");
@@ -142,8 +143,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   const uint32_t bar_empty = bar_full + 8 * STAGES;
   const uint32_t bar_accfull = bar_empty + 8 * STAGES;
   const uint32_t bar_accempty = bar_accfull + 8;
-  // sffull[s]: the stage's scale blocks have landed in this CTA (and, by the producer's order,
-  // the MMAs that last read slot s are done)
+  // sffull[s][p] (p = parity of the step): the stage's scale blocks have landed in this CTA (and,
+  // by the producer's order, the MMAs that last read slot s are done). Even and odd steps have
+  // barriers of their own, so each writer group waits on phases ten steps apart.
   const uint32_t bar_sf = bar_accempty + 8;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + N_BARS);
 
@@ -167,7 +169,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     }
     mbar_init(bar_accfull, 1);
     mbar_init(bar_accempty, ACCEMPTY_COUNT);
-    for (int s = 0; s < STAGES; ++s) mbar_init(bar_sf + 8 * s, 1);
+    for (int s = 0; s < 2 * STAGES; ++s) mbar_init(bar_sf + 8 * s, 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -337,7 +339,7 @@ __global__ void __launch_bounds__(THREADS, 1)
             const uint32_t at = smem_u32(a_tile(s));
             const uint32_t bt = smem_u32(b_tile(s));
             if (j < N_LORA) {
-              mbar_arrive(bar_sf + 8 * s);  // no scales for a low-rank step; the phase still advances
+              mbar_arrive(bar_sf + 8 * (2 * s + (it & 1)));  // no scales for a low-rank step; the phase still advances
               if (crank == 0) mbar_arrive_expect_tx(fb, 2 * (2 * LORA_A_BYTES + LORA_B_BYTES));
               tma_load_2d_pair(at, &tm_la, j * KC, row0, fb_lead);
               tma_load_2d_pair(at + LORA_LO_OFF, &tm_la, RANK + j * KC, row0, fb_lead);
@@ -347,7 +349,7 @@ __global__ void __launch_bounds__(THREADS, 1)
               const int kbv = min(4, kblocks - 4 * kt);
               const int mb = 2 * mt + static_cast<int>(crank);  // this CTA's 128-row block of X
               const bool rows_ok = mb * BM < a.M;               // activation scales cover ceil(M / 128) blocks
-              const uint32_t sfb = bar_sf + 8 * s;
+              const uint32_t sfb = bar_sf + 8 * (2 * s + (it & 1));
               const uint32_t blk = static_cast<uint32_t>(kbv) * SF_BLOCK;
               mbar_arrive_expect_tx(sfb, (rows_ok ? 3u : 2u) * blk);
               if (rows_ok)
@@ -431,21 +433,23 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
     } else if ((warp >= 2 && warp < EPI_WARP0) || warp == 16 || warp == 17) {
       // ------------------------------------------------------------ scale-factor writers
-      // Warp (q, h) writes tensor-memory lanes 32 q .. 32 q + 31 for k-blocks 2 h and 2 h + 1 of
-      // every step: lane i moves the 16-byte line i of the CTA's activation block (4 columns) and of
-      // the tile's two weight blocks (8 columns) of each k-block from the stage's scale region into
-      // the step's slot. Every step (low-rank ones too) is announced on the even CTA's full
-      // barrier, once per warp.
-      const int h = (warp >= 2 && warp < 6) ? 0 : 1;  // warps 2..5 and 6, 7, 16, 17 each cover the four sub-partitions
+      // Warp (q, h) writes tensor-memory lanes 32 q .. 32 q + 31 for the steps of parity h (two
+      // groups, so each warp's shared-memory reads, which queue behind the MMA operand reads and
+      // the TMA fills, have two steps of time): lane i moves the 16-byte line i of the CTA's
+      // activation block (4 columns) and of the tile's two weight blocks (8 columns) of each
+      // k-block from the stage's scale region into the step's slot. Every step (low-rank ones
+      // too) is announced on the even CTA's full barrier by the four warps of its group.
+      const int h = (warp >= 2 && warp < 6) ? 0 : 1;  // warps 2..5 take the even steps, 6, 7, 16, 17 the odd ones
       const uint32_t full_lead = map_shared_rank(bar_full, 0);
       const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
       const int my_tiles = tiles > pid ? (tiles - 1 - pid) / npairs + 1 : 0;
       const int nsteps = my_tiles * total;
-      for (int step = 0; step < nsteps; ++step) {
+      for (int step = h; step < nsteps; step += 2) {
         const int s = step % STAGES;
         const int j = step % total;
         // sffull of this step: its scale blocks are in shared memory and slot s is free
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * s, (step / STAGES) & 1, a.err, KID_GEMM, 6))) break;
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * (2 * s + h), (step / (2 * STAGES)) & 1, a.err, KID_GEMM, 6)))
+          break;
         if (FP4 && j >= N_LORA) {
           const int t = pid + (step / total) * npairs;
           const int mt = t % a.Mt;
@@ -453,10 +457,13 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int kbv = min(4, kblocks - 4 * kt);
           const bool rows_ok = (2 * mt + static_cast<int>(crank)) * BM < a.M;
           const uint32_t sft = smem_u32(a_tile(s)) + SF_OFF + lane * 16;
+          const uint32_t tsf = tbase + lane_base + SF_COL0 + SF_COLS * s;
+  #pragma unroll
+          for (int hh = 0; hh < 2; ++hh) {
           uint32_t sa[8], sb[16];
   #pragma unroll
           for (int e = 0; e < 2; ++e) {
-            const int kb = 2 * h + e;
+            const int kb = 2 * hh + e;
             uint4 va = make_uint4(0, 0, 0, 0), v0 = va, v1 = va;
             if (kb < kbv) {
               if (rows_ok) va = ld_shared_u32x4(sft + kb * SF_BLOCK);
@@ -468,9 +475,9 @@ __global__ void __launch_bounds__(THREADS, 1)
             sb[8 * e + 4] = v1.x; sb[8 * e + 5] = v1.y; sb[8 * e + 6] = v1.z; sb[8 * e + 7] = v1.w;
           }
           // slot columns: SFA k-block kb at 4 kb, SFB k-block kb at 16 + 8 kb (rows 0-127, then 128-255)
-          const uint32_t tsf = tbase + lane_base + SF_COL0 + SF_COLS * s;
-          tmem_st8(tsf + 8 * h, sa);
-          tmem_st16(tsf + 16 + 16 * h, sb);
+          tmem_st8(tsf + 8 * hh, sa);
+          tmem_st16(tsf + 16 + 16 * hh, sb);
+          }
           tmem_wait_st();
         }
         tc_fence_before();
