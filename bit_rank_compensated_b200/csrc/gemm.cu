@@ -23,18 +23,22 @@
 // All steps accumulate into one fp32 accumulator. lora_act arrives pre-divided by
 // alpha = s_x s_w, so the output stage computes Y = bf16(alpha * acc + bias) for every element.
 //
-// Scale factors reach tensor memory through shared memory and registers. With each 4-bit step
-// the producer bulk-copies three 2 KiB scale blocks into the stage (the CTA's activation block
-// and the tile's two weight blocks, four k-blocks each), signalled on a per-stage sffull barrier;
-// eight warps per CTA in two groups of four (one warp per 32-lane sub-partition), the groups taking
-// alternate steps, read the lines and write them with tcgen05.st in the replicated layout the block-scaled MMA
-// reads (lane i of every sub-partition holds rows i, i+32, i+64, i+96 of a block, one 32-bit
-// column each). tcgen05.st moves them several times faster than the tensor-memory copy unit,
-// which has to replicate every 512-byte block four times; staging the blocks with the stage
-// gives them the ring's whole latency tolerance (loaded from L2 by the writers themselves, two
-// steps ahead, they set the kernel's pace: a scratch copy without those loads ran 35% faster).
-// A CTA holds the activation scales of its own 128 rows and the weight scales of all 256 rows of
-// the tile, since its half of the MMA multiplies its rows by the whole of B.
+// Scale factors reach tensor memory from shared memory. With each 4-bit step the producer
+// bulk-copies three 2 KiB scale blocks into the stage (the CTA's activation block and the tile's
+// two weight blocks, four k-blocks each), signalled on a per-stage sffull barrier. The MMA
+// issuer copies the activation blocks with tcgen05.cp (one 32x128b.warpx4 copy per k-block, in
+// both CTAs, in order with and overlapping the MMAs: four per step keep the copy unit, ~90
+// cycles a block, inside the step's 512 MMA cycles). The eight weight blocks of a step would
+// overrun the copy unit, so eight warps per CTA in two groups of four (one warp per 32-lane
+// sub-partition, the groups taking alternate steps) read their lines and write them with
+// tcgen05.st. Both paths produce the replicated layout the block-scaled MMA reads (lane i of
+// every sub-partition holds rows i, i+32, i+64, i+96 of a block, one 32-bit column each).
+// Staging the blocks with the stage gives them the ring's whole latency tolerance (loaded from
+// L2 by the writers themselves, two steps ahead, they set the kernel's pace). A CTA holds the
+// activation scales of its own 128 rows and the weight scales of all 256 rows of the tile, since
+// its half of the MMA multiplies its rows by the whole of B (writing only the half of the weight
+// scales that matches the CTA's B rows, or writing them in the even CTA only, fails the
+// bit-exact layout tests).
 //
 // Warp roles (640 threads per CTA): warp 0 TMA producer; warp 1 tensor-memory owner and, in the
 // even CTA, MMA issuer; warps 2..5 (even steps) and 6, 7, 16, 17 (odd steps) scale-factor
@@ -416,9 +420,13 @@ __global__ void __launch_bounds__(THREADS, 1)
               const uint64_t ad = umma_desc(st, 16, 1024, 2);
               const uint64_t bd = umma_desc(st + A_BYTES, 16, 1024, 2);
               if (elect_one()) {
-                for (int kb = 0; kb < kbv; ++kb)
+                // activation scales: the copy unit replicates each CTA's 512-byte block into its
+                // four sub-partitions, in order with (and overlapping) the MMAs
+                for (int kb = 0; kb < kbv; ++kb) {
+                  tmem_cp_32x128b_x4_pair(tsf + 4 * kb, umma_desc(st + SF_OFF + SF_BLOCK * kb, 0, 128, 0));
                   mma_nvfp4_pair(tbase, ad + 2u * kb, bd + 2u * kb, idesc_fp4, tsf + 4 * kb, tsf + 16 + 8 * kb,
                                  (j | kb) != 0 ? 1u : 0u);
+                }
                 tc_commit_pair_mc(bar_empty + 8 * s, 0x3);
               }
             }
@@ -435,10 +443,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ------------------------------------------------------------ scale-factor writers
       // Warp (q, h) writes tensor-memory lanes 32 q .. 32 q + 31 for the steps of parity h (two
       // groups, so each warp's shared-memory reads, which queue behind the MMA operand reads and
-      // the TMA fills, have two steps of time): lane i moves the 16-byte line i of the CTA's
-      // activation block (4 columns) and of the tile's two weight blocks (8 columns) of each
-      // k-block from the stage's scale region into the step's slot. Every step (low-rank ones
-      // too) is announced on the even CTA's full barrier by the four warps of its group.
+      // the TMA fills, have two steps of time): lane i moves the 16-byte line i of the tile's two
+      // weight blocks (8 columns) of each k-block from the stage's scale region into the step's
+      // slot. Every step (low-rank ones too) is announced on the even CTA's full barrier by the
+      // four warps of its group.
       const int h = (warp >= 2 && warp < 6) ? 0 : 1;  // warps 2..5 take the even steps, 6, 7, 16, 17 the odd ones
       const uint32_t full_lead = map_shared_rank(bar_full, 0);
       const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -451,32 +459,27 @@ __global__ void __launch_bounds__(THREADS, 1)
         if (!__all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * (2 * s + h), (step / (2 * STAGES)) & 1, a.err, KID_GEMM, 6)))
           break;
         if (FP4 && j >= N_LORA) {
-          const int t = pid + (step / total) * npairs;
-          const int mt = t % a.Mt;
           const int kt = j - N_LORA;
           const int kbv = min(4, kblocks - 4 * kt);
-          const bool rows_ok = (2 * mt + static_cast<int>(crank)) * BM < a.M;
           const uint32_t sft = smem_u32(a_tile(s)) + SF_OFF + lane * 16;
           const uint32_t tsf = tbase + lane_base + SF_COL0 + SF_COLS * s;
   #pragma unroll
           for (int hh = 0; hh < 2; ++hh) {
-          uint32_t sa[8], sb[16];
+            uint32_t sb[16];
   #pragma unroll
-          for (int e = 0; e < 2; ++e) {
-            const int kb = 2 * hh + e;
-            uint4 va = make_uint4(0, 0, 0, 0), v0 = va, v1 = va;
-            if (kb < kbv) {
-              if (rows_ok) va = ld_shared_u32x4(sft + kb * SF_BLOCK);
-              v0 = ld_shared_u32x4(sft + (4 + kb) * SF_BLOCK);
-              v1 = ld_shared_u32x4(sft + (8 + kb) * SF_BLOCK);
+            for (int e = 0; e < 2; ++e) {
+              const int kb = 2 * hh + e;
+              uint4 v0 = make_uint4(0, 0, 0, 0), v1 = v0;
+              if (kb < kbv) {
+                v0 = ld_shared_u32x4(sft + (4 + kb) * SF_BLOCK);
+                v1 = ld_shared_u32x4(sft + (8 + kb) * SF_BLOCK);
+              }
+              sb[8 * e + 0] = v0.x; sb[8 * e + 1] = v0.y; sb[8 * e + 2] = v0.z; sb[8 * e + 3] = v0.w;
+              sb[8 * e + 4] = v1.x; sb[8 * e + 5] = v1.y; sb[8 * e + 6] = v1.z; sb[8 * e + 7] = v1.w;
             }
-            sa[4 * e + 0] = va.x; sa[4 * e + 1] = va.y; sa[4 * e + 2] = va.z; sa[4 * e + 3] = va.w;
-            sb[8 * e + 0] = v0.x; sb[8 * e + 1] = v0.y; sb[8 * e + 2] = v0.z; sb[8 * e + 3] = v0.w;
-            sb[8 * e + 4] = v1.x; sb[8 * e + 5] = v1.y; sb[8 * e + 6] = v1.z; sb[8 * e + 7] = v1.w;
-          }
-          // slot columns: SFA k-block kb at 4 kb, SFB k-block kb at 16 + 8 kb (rows 0-127, then 128-255)
-          tmem_st8(tsf + 8 * hh, sa);
-          tmem_st16(tsf + 16 + 16 * hh, sb);
+            // slot columns: SFB k-block kb at 16 + 8 kb (rows 0-127, then 128-255); the SFA
+            // columns (4 kb) are filled by the MMA issuer's copies
+            tmem_st16(tsf + 16 + 16 * hh, sb);
           }
           tmem_wait_st();
         }
