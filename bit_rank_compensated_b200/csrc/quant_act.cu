@@ -18,7 +18,7 @@
 // The down-projection is stored pre-divided by alpha = s_x s_w as an unevaluated sum of two
 // bf16 values (hi + lo), so the fp32 result reaches K2 without a 16-bit rounding.
 //
-// Warp roles (576 threads):
+// Warp roles (576 threads, 704 where the reduction has warps of its own):
 //   warp 0       TMA producer: per chunk of a stage the X tile (rows x 64 bf16, 128B swizzle),
 //                the L1s tile (rank x 64 bf16, 128B swizzle) and the chunk's inv_lambda values.
 //   warp 1       owns the tensor-memory accumulator (rows x rank fp32) and issues the bf16
@@ -29,6 +29,10 @@
 //                Each quarter-warp reads eight consecutive rows of one group (conflict-free
 //                under the 128B swizzle) and one broadcast copy of the group's 16 inv_lambda
 //                values, which serve both of the lane's rows.
+//   warps 18..21 (ranks up to 64) split-K reduction: one warp per tensor-memory quadrant reads
+//                its accumulator rows once the last MMAs are committed, sends the partials of
+//                rows another CTA owns with st.async, sums its own rows and stores lora_act,
+//                while the quantizers are still on their last stages.
 #include "common.cuh"
 #include "internal.h"
 #include "nvfp4.cuh"
@@ -42,7 +46,6 @@ struct QCfg {
   static constexpr int QWARPS = 16;
   static constexpr int WARPS_PER_CHUNK = ROWS / 16;
   static constexpr int SUB = QWARPS / WARPS_PER_CHUNK;  // 64-column chunks per stage
-  static constexpr int THREADS = 64 + 32 * QWARPS;
   static constexpr uint32_t X_BYTES = ROWS * 128u;  // per chunk
   static constexpr uint32_t L1_BYTES = RANK * 128u;
   static constexpr uint32_t IL_BYTES = QUANT ? 64u * 4u : 0u;
@@ -54,14 +57,25 @@ struct QCfg {
   // (16-byte accesses spread over banks)
   static constexpr uint32_t RED_STRIDE = RANK + 4;
   static constexpr uint32_t RED_BYTES = RED_STRIDE * (ROWS + 8) * 4u;
-  static constexpr uint32_t DATA_BYTES =
-      (STAGES * STAGE_BYTES > RED_BYTES) ? STAGES * STAGE_BYTES : RED_BYTES;
   static constexpr uint32_t BAR_BYTES = 256;
+  // Where the split-K slots fit beside the stages, they get a region of their own and four more
+  // warps (one per tensor-memory quadrant) reduce as soon as the accumulator is complete, while
+  // the quantizers finish their last stages; otherwise (rank 128) the slots reuse the stage
+  // memory once it is idle and the quantizer warps reduce.
+  static constexpr uint32_t STAGE_TOTAL = STAGES * STAGE_BYTES;
+  static constexpr bool RED_SEPARATE = RANK > 0 && STAGE_TOTAL + RED_BYTES + BAR_BYTES + 1024u <= 232448u;
+  static constexpr int RED_WARPS = RED_SEPARATE ? 4 : 0;
+  static constexpr int RED_WARP0 = 2 + QWARPS;
+  static constexpr int THREADS = 64 + 32 * QWARPS + 32 * RED_WARPS;
+  static constexpr uint32_t RED_OFF = RED_SEPARATE ? STAGE_TOTAL : 0u;
+  static constexpr uint32_t DATA_BYTES =
+      RED_SEPARATE ? STAGE_TOTAL + RED_BYTES : (STAGE_TOTAL > RED_BYTES ? STAGE_TOTAL : RED_BYTES);
   static constexpr uint32_t SMEM = DATA_BYTES + BAR_BYTES + 1024;  // + alignment slack
   static constexpr uint32_t TMEM_COLS = RANK <= 32 ? 32u : static_cast<uint32_t>(RANK);
   // arrivals that free a stage: one per quantizer warp, one MMA commit
   static constexpr uint32_t EMPTY_COUNT = (QUANT ? QWARPS : 0) + (RANK ? 1 : 0);
   static_assert(ROWS == 64 || ROWS == 128, "tensor-core M");
+  static_assert(RED_OFF % 1024 == 0, "reduction slots start on a stage boundary");
   static_assert(STAGES >= 2, "pipeline needs two stages");
   static_assert(2 * STAGES + 3 <= static_cast<int>(BAR_BYTES / 8), "barrier area");
 };
@@ -157,6 +171,9 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = RANK ? *tmem_holder : 0u;
+  // With separate reduction slots every thread arrives on the cluster barrier now: a CTA's slots
+  // and recv barrier are ready for the other CTAs' partials from the start.
+  if constexpr (C::RED_SEPARATE) cluster_arrive();
   // The prologue above overlaps the previous kernel of the stream; global memory only after it.
   grid_dep_wait();
   grid_dep_launch();
@@ -212,7 +229,7 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
       if (elect_one()) tc_commit(bar_acc);
       __syncwarp();
     }
-  } else if (QUANT) {
+  } else if (QUANT && warp < C::RED_WARP0) {
     // ------------------------------------------------------------ quantizers
     const int qw = warp - 2;
     const int u = qw / C::WARPS_PER_CHUNK;  // chunk of the stage
@@ -285,8 +302,88 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
     // soon as this CTA's quantizer warps and MMAs are done with it.
     constexpr uint32_t RS = C::RED_STRIDE;
     const uint32_t slot_bytes = static_cast<uint32_t>(rows_per) * RS * 4u;
-    const uint32_t red_base = smem_u32(smem);
-    if (warp >= 2) {
+    uint8_t *red = smem + C::RED_OFF;
+    const uint32_t red_base = smem_u32(red);
+    // rows own_r0 .. own_r1 - 1: sum the slots in rank order, four columns per thread, and store
+    // lora_act (threads t0, t0 + nthr, ...)
+    auto sum_store = [&](int t0, int nthr) {
+      constexpr int QUADS = RANK / 4;
+      for (int idx = t0; idx < (own_r1 - own_r0) * QUADS; idx += nthr) {
+        const int lr = idx / QUADS;
+        const int c = 4 * (idx % QUADS);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int src = 0; src < nsplit; ++src) {
+          const float4 v =
+              *reinterpret_cast<const float4 *>(red + src * slot_bytes + static_cast<uint32_t>(lr * RS + c) * 4u);
+          acc.x += v.x;
+          acc.y += v.y;
+          acc.z += v.z;
+          acc.w += v.w;
+        }
+        const int m = m0 + own_r0 + lr;
+        if (m < a.M) {
+          // lora_act row = [hi(0..RANK-1) | lo(0..RANK-1)], v ~ hi + lo with hi = bf16(v),
+          // lo = bf16(v - hi): the pair carries ~16 significant bits of the fp32 value.
+          const float v0 = __fmul_rn(acc.x, a.inv_alpha), v1 = __fmul_rn(acc.y, a.inv_alpha);
+          const float v2 = __fmul_rn(acc.z, a.inv_alpha), v3 = __fmul_rn(acc.w, a.inv_alpha);
+          const uint32_t h01 = pack_bf16x2(v0, v1), h23 = pack_bf16x2(v2, v3);
+          const uint32_t l01 = pack_bf16x2(__fsub_rn(v0, bf16_lo(h01)), __fsub_rn(v1, bf16_hi(h01)));
+          const uint32_t l23 = pack_bf16x2(__fsub_rn(v2, bf16_lo(h23)), __fsub_rn(v3, bf16_hi(h23)));
+          uint16_t *out = a.lora_act + static_cast<size_t>(m) * (2 * RANK) + c;
+          *reinterpret_cast<uint2 *>(out) = make_uint2(h01, h23);
+          *reinterpret_cast<uint2 *>(out + RANK) = make_uint2(l01, l23);
+        }
+      }
+    };
+    // this CTA's partial of accumulator row `row` (vals: RANK fp32) into the owner's slot
+    auto send_row = [&](int row, const uint32_t *vals, int c0, int nc, bool ok) {
+      const int owner = row / rows_per;
+      const uint32_t off =
+          static_cast<uint32_t>(split) * slot_bytes + static_cast<uint32_t>((row - owner * rows_per) * RS + c0) * 4u;
+      if (owner == split) {
+        for (int j = 0; j < nc; j += 4)
+          *reinterpret_cast<float4 *>(red + off + 4 * j) =
+              ok ? make_float4(__uint_as_float(vals[j]), __uint_as_float(vals[j + 1]), __uint_as_float(vals[j + 2]),
+                               __uint_as_float(vals[j + 3]))
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+      } else {
+        const uint32_t dst = map_shared_rank(red_base + off, owner);
+        const uint32_t rbar = map_shared_rank(bar_recv, owner);
+        for (int j = 0; j < nc; j += 4)
+          st_async_f32x4(dst + 4 * j,
+                         ok ? make_float4(__uint_as_float(vals[j]), __uint_as_float(vals[j + 1]),
+                                          __uint_as_float(vals[j + 2]), __uint_as_float(vals[j + 3]))
+                            : make_float4(0.f, 0.f, 0.f, 0.f),
+                         rbar);
+      }
+    };
+    if constexpr (C::RED_SEPARATE) {
+      if (warp >= C::RED_WARP0) {
+        // Warp w reads the accumulator rows of tensor-memory quadrant w % 4, all RANK columns.
+        const int quad = warp & 3;
+        const bool row_ok = C::ROWS == 128 || lane < 16;
+        const int row = C::ROWS == 128 ? quad * 32 + lane : quad * 16 + (lane & 15);
+        const bool ok = mbar_wait_parked(bar_acc, 0, a.err, KID_QUANT, 5) && n_local > 0;
+        tc_fence_after();
+        const uint32_t taddr = tbase + (static_cast<uint32_t>(quad * 32) << 16);
+        uint32_t r[RANK];
+        if constexpr (RANK == 16) {
+          tmem_ld16(taddr, *reinterpret_cast<uint32_t(*)[16]>(r));
+        } else {
+#pragma unroll
+          for (int c = 0; c < RANK / 32; ++c) tmem_ld32(taddr + 32 * c, *reinterpret_cast<uint32_t(*)[32]>(r + 32 * c));
+        }
+        tmem_wait_ld();
+        tc_fence_before();
+        cluster_wait();  // every CTA of the cluster has initialised its recv barrier
+        if (row_ok) send_row(row, r, 0, RANK, ok);
+        named_bar_sync(2, 32 * C::RED_WARPS);
+        mbar_wait_parked(bar_recv, 0, a.err, KID_QUANT, 6);
+        sum_store(static_cast<int>(threadIdx.x) - 32 * C::RED_WARP0, 32 * C::RED_WARPS);
+      } else {
+        cluster_wait();
+      }
+    } else if (warp >= 2) {
       // A warp reads the 32 tensor-memory lanes of its quadrant (warp % 4). Accumulator row r
       // sits in lane r for M = 128 and in lane 32 (r / 16) + r % 16 for M = 64 (the upper 16
       // lanes of each quadrant then hold nothing).
@@ -312,59 +409,10 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
       }
       tc_fence_before();
       cluster_wait();
-      if (row_ok && (RANK != 16 || grp == 0)) {
-        const int owner = row / rows_per;
-        const uint32_t off = static_cast<uint32_t>(split) * slot_bytes +
-                             static_cast<uint32_t>((row - owner * rows_per) * RS + cb) * 4u;
-        if (owner == split) {
-#pragma unroll
-          for (int j = 0; j < CPG; j += 4)
-            *reinterpret_cast<float4 *>(smem + off + 4 * j) =
-                ok ? make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                                 __uint_as_float(r[j + 3]))
-                   : make_float4(0.f, 0.f, 0.f, 0.f);
-        } else {
-          const uint32_t dst = map_shared_rank(red_base + off, owner);
-          const uint32_t rbar = map_shared_rank(bar_recv, owner);
-#pragma unroll
-          for (int j = 0; j < CPG; j += 4)
-            st_async_f32x4(dst + 4 * j,
-                           ok ? make_float4(__uint_as_float(r[j]), __uint_as_float(r[j + 1]), __uint_as_float(r[j + 2]),
-                                            __uint_as_float(r[j + 3]))
-                              : make_float4(0.f, 0.f, 0.f, 0.f),
-                           rbar);
-        }
-      }
+      if (row_ok && (RANK != 16 || grp == 0)) send_row(row, r, cb, CPG, ok);
       named_bar_sync(1, 32 * C::QWARPS);
       mbar_wait_parked(bar_recv, 0, a.err, KID_QUANT, 6);
-      // rows own_r0 .. own_r1 - 1: sum the slots in rank order, four columns per thread
-      constexpr int QUADS = RANK / 4;
-      for (int idx = threadIdx.x - 64; idx < (own_r1 - own_r0) * QUADS; idx += 32 * C::QWARPS) {
-        const int lr = idx / QUADS;
-        const int c = 4 * (idx % QUADS);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int src = 0; src < nsplit; ++src) {
-          const float4 v =
-              *reinterpret_cast<const float4 *>(smem + src * slot_bytes + static_cast<uint32_t>(lr * RS + c) * 4u);
-          acc.x += v.x;
-          acc.y += v.y;
-          acc.z += v.z;
-          acc.w += v.w;
-        }
-        const int m = m0 + own_r0 + lr;
-        if (m < a.M) {
-          // lora_act row = [hi(0..RANK-1) | lo(0..RANK-1)], v ~ hi + lo with hi = bf16(v),
-          // lo = bf16(v - hi): the pair carries ~16 significant bits of the fp32 value.
-          const float v0 = __fmul_rn(acc.x, a.inv_alpha), v1 = __fmul_rn(acc.y, a.inv_alpha);
-          const float v2 = __fmul_rn(acc.z, a.inv_alpha), v3 = __fmul_rn(acc.w, a.inv_alpha);
-          const uint32_t h01 = pack_bf16x2(v0, v1), h23 = pack_bf16x2(v2, v3);
-          const uint32_t l01 = pack_bf16x2(__fsub_rn(v0, bf16_lo(h01)), __fsub_rn(v1, bf16_hi(h01)));
-          const uint32_t l23 = pack_bf16x2(__fsub_rn(v2, bf16_lo(h23)), __fsub_rn(v3, bf16_hi(h23)));
-          uint16_t *out = a.lora_act + static_cast<size_t>(m) * (2 * RANK) + c;
-          *reinterpret_cast<uint2 *>(out) = make_uint2(h01, h23);
-          *reinterpret_cast<uint2 *>(out + RANK) = make_uint2(l01, l23);
-        }
-      }
+      sum_store(static_cast<int>(threadIdx.x) - 64, 32 * C::QWARPS);
     } else {
       cluster_arrive();
       cluster_wait();
