@@ -406,6 +406,11 @@ __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol
 // needed. Every thread of every CTA of the cluster executes both.
 __device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// Arrive without release semantics: enough when the only writes the other CTAs rely on are
+// mbarrier initialisations published by fence.mbarrier_init.release.cluster.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
 // 16-byte store into a CTA of the cluster (addr, bar: shared::cluster addresses of that CTA) that
 // counts its bytes against the transaction count of the mbarrier bar there.
 __device__ __forceinline__ void st_async_f32x4(uint32_t addr, float4 v, uint32_t bar) {

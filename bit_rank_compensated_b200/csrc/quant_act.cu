@@ -172,8 +172,9 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
   tc_fence_after();
   const uint32_t tbase = RANK ? *tmem_holder : 0u;
   // With separate reduction slots every thread arrives on the cluster barrier now: a CTA's slots
-  // and recv barrier are ready for the other CTAs' partials from the start.
-  if constexpr (C::RED_SEPARATE) cluster_arrive();
+  // and recv barrier (initialised and published with fence.mbarrier_init above) are ready for
+  // the other CTAs' partials from the start.
+  if constexpr (C::RED_SEPARATE) cluster_arrive_relaxed();
   // The prologue above overlaps the previous kernel of the stream; global memory only after it.
   grid_dep_wait();
   grid_dep_launch();
