@@ -320,3 +320,56 @@ def layer_forward(Xv, layer: Layer):
 def calibration_absmax(Xv):
     """a_x[j] = max_m |X[m, j]| (exact)."""
     return np.abs(np.asarray(Xv, dtype=np.float64)).max(axis=0)
+
+
+# --------------------------------------------------------------------------- fused QKV output stage
+# "Nunchaku Lite in Diffusers", section on quantized models with structural rewrites
+# ("نماذج الكم مع إعادة الكتابة الهيكلية"): FLUX.1-dev's Q, K and V projections are
+# concatenated along the output dimension, in that order, into one to_qkv layer, and the
+# engine's fused operator consumes that projection together with the Q/K normalization
+# (norm_q, norm_k) and the rotary embedding (apply_rotary_emb on Q and K), which the default
+# path runs as separate steps after splitting the output into heads.
+# Readings (the page names the steps, not their formulas):
+#   * Y = [Q | K | V], each section `heads` heads of `head_dim` columns, head h of a section
+#     in columns h*head_dim .. (h+1)*head_dim - 1;
+#   * norm_q / norm_k are RMS normalizations over a head's head_dim values with a learned
+#     per-column weight: u = y w / sqrt(mean(y^2) + eps);
+#   * the rotary embedding turns each pair of columns (2i, 2i + 1) of a Q or K head by the
+#     angle theta[m, i] of token m and pair i, given as the table (cos theta, sin theta);
+#   * V passes through unchanged;
+#   * in the fused operator the normalization reads the layer output before its 16-bit
+#     rounding.
+def rms_norm_heads(Yh, weight, eps: float):
+    """u = y * w / sqrt(mean(y^2) + eps) over the last axis (one head), fp64."""
+    Yh = np.asarray(Yh, dtype=np.float64)
+    ms = np.mean(Yh * Yh, axis=-1, keepdims=True)
+    return Yh / np.sqrt(ms + eps) * np.asarray(weight, dtype=np.float64)
+
+
+def rotary_pairs(U, cos, sin):
+    """Turn the pairs (U[..., 2i], U[..., 2i+1]) by the angle whose cosine and sine are
+    cos[m, i], sin[m, i]; U is (M, heads, head_dim), cos / sin are (M, head_dim / 2)."""
+    U = np.asarray(U, dtype=np.float64)
+    x0 = U[..., 0::2]
+    x1 = U[..., 1::2]
+    c = np.asarray(cos, dtype=np.float64)[:, None, :]
+    s = np.asarray(sin, dtype=np.float64)[:, None, :]
+    out = np.empty_like(U)
+    out[..., 0::2] = x0 * c - x1 * s
+    out[..., 1::2] = x1 * c + x0 * s
+    return out
+
+
+def qk_norm_rope(Y, heads: int, head_dim: int, norm_q_weight, norm_k_weight, cos, sin, eps: float):
+    """Output stage of the fused QKV projection: per-head RMS normalization and rotary
+    embedding of the Q and K sections of Y = [Q | K | V]; V unchanged. fp64."""
+    Y = np.asarray(Y, dtype=np.float64)
+    M, N = Y.shape
+    width = heads * head_dim
+    assert N == 3 * width and head_dim % 2 == 0
+    Z = Y.copy()
+    for sec, w in ((0, norm_q_weight), (1, norm_k_weight)):
+        block = Y[:, sec * width:(sec + 1) * width].reshape(M, heads, head_dim)
+        U = rms_norm_heads(block, w, eps)
+        Z[:, sec * width:(sec + 1) * width] = rotary_pairs(U, cos, sin).reshape(M, width)
+    return Z

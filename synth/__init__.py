@@ -24,6 +24,12 @@ Draw order: outlier channel indices, outlier factors, activations, weights, bias
 
 Activations are generated in fp64, cast to fp32 and rounded to bf16 (round to nearest
 even) for storage; W and b are stored as fp32.
+
+Inputs of the fused QKV output stage (per-head Q/K normalization and rotary embedding):
+``rope_table`` gives FLUX-like token positions (text tokens first at position 0, then image
+tokens on a 64-wide latent grid, three position axes of 16, 56 and 56 head columns, base
+10000) as a (cos, sin) table per token and column pair, angles in fp64 rounded to fp32;
+``qk_norm_weights`` draws the two normalization weight vectors ~ N(1, 0.1^2).
 """
 from __future__ import annotations
 
@@ -39,6 +45,8 @@ __all__ = [
     "make_inputs",
     "f32_to_bf16_bits",
     "bf16_bits_to_f32",
+    "rope_table",
+    "qk_norm_weights",
 ]
 
 
@@ -130,3 +138,34 @@ def make_inputs(shape: LayerShape, seed: int = 0, M: int | None = None):
 
     Xb = f32_to_bf16_bits(X.astype(np.float32))
     return Xb, W.astype(np.float32), b.astype(np.float32), np.sort(ch)
+
+
+def rope_table(M: int, head_dim: int = 128, n_text: int | None = None, grid_w: int = 64,
+               axes=(16, 56, 56), theta: float = 10000.0) -> np.ndarray:
+    """(cos, sin) of the rotary angle per token and head-column pair: float32 [M, head_dim/2, 2].
+
+    Token m < n_text is a text token (every position coordinate 0); token n_text + j is the
+    image token at row j // grid_w, column j % grid_w of the latent grid, with coordinates
+    (0, row, column) on the three axes. Axis a of width d_a contributes d_a / 2 pairs with
+    frequencies theta^(-2k / d_a), k = 0 .. d_a/2 - 1; the angle is coordinate x frequency.
+    ``n_text`` defaults to the FLUX proportion of 512 text tokens per 4608.
+    """
+    assert sum(axes) == head_dim and all(d % 2 == 0 for d in axes)
+    if n_text is None:
+        n_text = (M * 512) // 4608
+    m = np.arange(M)
+    j = np.maximum(m - n_text, 0)
+    img = m >= n_text
+    coords = np.stack([np.zeros(M), np.where(img, j // grid_w, 0), np.where(img, j % grid_w, 0)], axis=1)
+    angles = []
+    for a, d in enumerate(axes):
+        freq = theta ** (-np.arange(0, d, 2, dtype=np.float64) / d)
+        angles.append(coords[:, a:a + 1].astype(np.float64) * freq[None, :])
+    ang = np.concatenate(angles, axis=1)
+    return np.stack([np.cos(ang), np.sin(ang)], axis=-1).astype(np.float32)
+
+
+def qk_norm_weights(head_dim: int = 128, seed: int = 0):
+    """Weights of the Q and K normalizations, float32 [head_dim] each, ~ N(1, 0.1^2)."""
+    rng = np.random.Generator(np.random.PCG64(seed + 1000))
+    return (rng.normal(1.0, 0.1, head_dim).astype(np.float32), rng.normal(1.0, 0.1, head_dim).astype(np.float32))
