@@ -238,15 +238,26 @@ def time_graphs(stream, graphs):
     return [evs[k].elapsed_time(evs[k + 1]) for k in range(len(graphs))]
 
 
-SUITE = ["qkv", "mlp_up", "mlp_down", "sweep_m256", "sweep_m1024", "sweep_m4096", "sweep_m16384",
+SUITE = ["qkv", "qkv_qknorm_rope", "mlp_up", "mlp_down", "sweep_m256", "sweep_m1024", "sweep_m4096", "sweep_m16384",
          "sweep_r0", "sweep_r16", "sweep_r32", "sweep_r64", "sweep_r128"]
+HEAD_DIM = 128
 
 
-def time_layer(shape, steps, warmup, dev, stream, unfused=False, nb=3):
+def qk_stage_bytes(M, N):
+    """Algorithmic HBM bytes of the unfused Q/K normalization + rotary step: read and rewrite the
+    bf16 Q and K sections (2/3 of Y), read the (cos, sin) table (M x 64 x 2 fp32)."""
+    return 2.0 * (2.0 * M * (2 * N // 3)) + M * (HEAD_DIM // 2) * 8.0
+
+
+def time_layer(shape, steps, warmup, dev, stream, unfused=False, nb=3, stage="plain"):
     """Mean device time (ms) per step of the layer on one GPU over `nb` rotating buffer sets:
-    fused K1 + K2, or the unfused four-kernel path. Returns (step_ms, k1_ms, k2_ms)."""
+    fused K1 + K2, or the unfused four-kernel path. stage = "qknr": K2 with the fused QKV output
+    stage (Q/K normalization and rotary embedding); "qknr_unfused": plain K2 followed by the
+    separate normalization + rotary step. Returns (step_ms, k1_ms, k2_ms); for "qknr_unfused"
+    k2_ms covers K2 and the separate step."""
     import torch
     from bit_rank_compensated_b200 import svdq
+    from synth import qk_norm_weights, rope_table
 
     M, K, N, r = shape.M, shape.K, shape.N, shape.rank
     Xb, W, b, _ = make_inputs(shape, seed=0)
@@ -256,14 +267,29 @@ def time_layer(shape, steps, warmup, dev, stream, unfused=False, nb=3):
     Xs = [X0] + [X0.clone() for _ in range(nb - 1)]
     bufs = [svdq.alloc_activations(M, L, dev) for _ in range(nb)]
     Ys = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(nb)]
+    heads = N // (3 * HEAD_DIM)
+    if stage != "plain":
+        wq, wk = (torch.from_numpy(w).to(dev) for w in qk_norm_weights(HEAD_DIM))
+        ropes = [torch.from_numpy(rope_table(M, HEAD_DIM)).to(dev) for _ in range(nb)]
+
+    def k2_part(j):
+        xq, xs, la = bufs[j]
+        if stage == "qknr":
+            return lambda st: svdq.gemm_w4a4_lora_up_qk_norm_rope(xq, xs, la, M, L, heads, wq, wk, ropes[j], 1e-6,
+                                                                  Ys[j], st)
+        if stage == "qknr_unfused":
+            def both(st):
+                svdq.gemm_w4a4_lora_up(xq, xs, la, M, L, Ys[j], st)
+                svdq.qk_norm_rope(Ys[j], heads, wq, wk, ropes[j], 1e-6, st)
+            return both
+        return lambda st: svdq.gemm_w4a4_lora_up(xq, xs, la, M, L, Ys[j], st)
 
     def step_on(j):
         # part 0: K1 (or the whole unfused path), part 1: K2 (None when unfused)
         xq, xs, la = bufs[j]
         if unfused:
             return (lambda st: svdq.unfused_forward(Xs[j], L, bufs[j], Ys[j], st)), None
-        return ((lambda st: svdq.quant_act_lora_down(Xs[j], L, xq, xs, la, st)),
-                (lambda st: svdq.gemm_w4a4_lora_up(xq, xs, la, M, L, Ys[j], st)))
+        return (lambda st: svdq.quant_act_lora_down(Xs[j], L, xq, xs, la, st)), k2_part(j)
 
     def step(i):
         a, b = step_on(i % nb)
@@ -304,19 +330,37 @@ def run_suite(args):
     hbm_gbs, bf16_tf, peak_kind = read_peaks()
     fp4_peak = bf16_tf * FP4_OVER_BF16
     r0_ms = None
+    plain_k2 = {}
     for name in args.suite.split(","):
-        shape = CONFIGS[name]
+        qknr = name.endswith("_qknorm_rope")
+        shape = CONFIGS[name[:-len("_qknorm_rope")] if qknr else name]
         M, K, N, r = shape.M, shape.K, shape.N, shape.rank
-        step_ms, k1_ms, k2_ms = time_layer(shape, args.steps, args.warmup, dev, stream)
+        step_ms, k1_ms, k2_ms = time_layer(shape, args.steps, args.warmup, dev, stream,
+                                           stage="qknr" if qknr else "plain")
         line = {"metric": METRIC, "value": layer_flops(M, K, N, r) / (step_ms * 1e-3) / 1e12, "unit": "TFLOPS",
                 "n_gpus": 1, "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
                 "higher_is_better": True, "dtype": "nvfp4", "data": "synthetic",
-                "config": {"workload": workload_name(shape), "M": M, "K": K, "N": N, "rank": r},
+                "config": {"workload": workload_name(shape) + (", fused Q/K RMS norm + rotary output stage"
+                                                               if qknr else ""), "M": M, "K": K, "N": N, "rank": r},
                 "k1": {"us": k1_ms * 1e3, "gbs": k1_bytes(M, K, r) / (k1_ms * 1e-3) / 1e9,
                        "frac_hbm": k1_bytes(M, K, r) / (k1_ms * 1e-3) / 1e9 / hbm_gbs},
                 "k2": {"us": k2_ms * 1e3, "tflops": k2_flops(M, K, N, r) / (k2_ms * 1e-3) / 1e12,
                        "frac_fp4": k2_flops(M, K, N, r) / (k2_ms * 1e-3) / 1e12 / fp4_peak},
                 "tokens_per_s": M / (step_ms * 1e-3), "peaks": peak_kind}
+        if not qknr:
+            plain_k2[shape.name] = k2_ms
+        else:
+            if shape.name not in plain_k2:
+                plain_k2[shape.name] = time_layer(shape, args.steps, args.warmup, dev, stream)[2]
+            unf_ms, _, unf_k2 = time_layer(shape, args.steps, args.warmup, dev, stream, stage="qknr_unfused")
+            # the separate step alone: the unfused K2 + step minus the plain K2
+            sep_ms = unf_k2 - plain_k2[shape.name]
+            line["qknorm_rope"] = {
+                "fused_stage_overhead_vs_plain_k2": k2_ms / plain_k2[shape.name] - 1.0,
+                "unfused_step_ms": unf_ms, "unfused_over_fused": unf_ms / step_ms,
+                "separate_step_us": sep_ms * 1e3,
+                "separate_step_gbs": qk_stage_bytes(M, N) / (sep_ms * 1e-3) / 1e9 if sep_ms > 0 else None,
+                "separate_step_frac_hbm": qk_stage_bytes(M, N) / (sep_ms * 1e-3) / 1e9 / hbm_gbs if sep_ms > 0 else None}
         if name.startswith("sweep_r"):
             if r == 0:
                 r0_ms = step_ms

@@ -150,8 +150,14 @@ svdq_status run_quant(const uint16_t *X, int M, const svdq_layer *L, uint8_t *xq
   return launch_quant_act(q) == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 
+struct QkNormRope {
+  int heads;
+  const float *norm_q, *norm_k, *rope;
+  float eps;
+};
+
 svdq_status run_gemm(const uint8_t *xq, const uint8_t *xs, const uint16_t *la, int M, const svdq_layer *L,
-                     uint16_t *Y, bool fp4, bool add_y, bool lora, void *stream) {
+                     uint16_t *Y, bool fp4, bool add_y, bool lora, void *stream, const QkNormRope *qk = nullptr) {
   DeviceState *d = nullptr;
   svdq_status st = device_check(&d);
   if (st != SVDQ_OK) return st;
@@ -200,6 +206,14 @@ svdq_status run_gemm(const uint8_t *xq, const uint8_t *xs, const uint16_t *la, i
   g.alpha = alpha_of(L);
   g.fp4 = fp4;
   g.add_y = add_y;
+  if (qk) {
+    g.qk_norm_rope = true;
+    g.norm_q = qk->norm_q;
+    g.norm_k = qk->norm_k;
+    g.rope = qk->rope;
+    g.qk_width = qk->heads * 128;
+    g.eps = qk->eps;
+  }
   g.num_sms = d->num_sms;
   g.err = d->err;
   g.stream = static_cast<cudaStream_t>(stream);
@@ -352,6 +366,42 @@ svdq_status svdq_quant_act_lora_down(const uint16_t *X, int M, const svdq_layer 
 svdq_status svdq_gemm_w4a4_lora_up(const uint8_t *xq, const uint8_t *xs, const uint16_t *lora_act, int M,
                                    const svdq_layer *layer, uint16_t *Y, void *stream) {
   return run_gemm(xq, xs, lora_act, M, layer, Y, true, false, true, stream);
+}
+
+namespace {
+svdq_status check_qk_args(int N, int heads, int head_dim, const float *wq, const float *wk, const float *rope,
+                          float eps) {
+  if (heads <= 0 || head_dim != 128 || N != 3 * heads * 128 || !wq || !wk || !rope || !(eps >= 0.0f))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(wq) || !aligned16(wk) || !aligned16(rope)) return SVDQ_ERR_MISALIGNED;
+  return SVDQ_OK;
+}
+}  // namespace
+
+svdq_status svdq_gemm_w4a4_lora_up_qk_norm_rope(const uint8_t *xq, const uint8_t *xs, const uint16_t *lora_act,
+                                                int M, const svdq_layer *layer, int heads, int head_dim,
+                                                const float *norm_q_weight, const float *norm_k_weight,
+                                                const float *rope, float eps, uint16_t *Y, void *stream) {
+  if (!layer) return SVDQ_ERR_INVALID_ARG;
+  svdq_status st = check_qk_args(layer->N, heads, head_dim, norm_q_weight, norm_k_weight, rope, eps);
+  if (st != SVDQ_OK) return st;
+  const QkNormRope qk{heads, norm_q_weight, norm_k_weight, rope, eps};
+  return run_gemm(xq, xs, lora_act, M, layer, Y, true, false, true, stream, &qk);
+}
+
+svdq_status svdq_qk_norm_rope(uint16_t *Y, int M, int heads, int head_dim, const float *norm_q_weight,
+                              const float *norm_k_weight, const float *rope, float eps, void *stream) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  if (!Y || M <= 0 || heads <= 0) return SVDQ_ERR_INVALID_ARG;
+  st = check_qk_args(3 * heads * head_dim, heads, head_dim, norm_q_weight, norm_k_weight, rope, eps);
+  if (st != SVDQ_OK) return st;
+  if (!aligned16(Y)) return SVDQ_ERR_MISALIGNED;
+  return launch_qk_norm_rope(Y, M, heads, norm_q_weight, norm_k_weight, rope, eps, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? SVDQ_OK
+             : SVDQ_ERR_CUDA;
 }
 
 svdq_status svdq_linear_forward(const uint16_t *X, int M, const svdq_layer *layer, uint8_t *xq, uint8_t *xs,

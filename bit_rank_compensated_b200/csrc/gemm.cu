@@ -80,8 +80,10 @@ constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SF_STAGE_BYTES;  // 38 KiB
 constexpr uint32_t DATA_BYTES = STAGES * STAGE_BYTES;
 constexpr uint32_t YST_BYTES = BM * 64 * 2 * 2;  // bf16 output staging: one box of 128 rows x 64 columns per half
 constexpr uint32_t BIAS_BYTES = BN * 4;
+constexpr uint32_t NORMW_BYTES = 2 * 2 * 128 * 4;  // fused QKV output stage only
 constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM = DATA_BYTES + YST_BYTES + BIAS_BYTES + BAR_BYTES + 1024;
+constexpr uint32_t SMEM_QKNR = SMEM + NORMW_BYTES;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = 256;  // one scale slot per stage follows the accumulator
 constexpr uint32_t SF_COLS = 48;   // per slot: 4 k-blocks x (4 SFA + 8 SFB) columns
@@ -104,7 +106,7 @@ constexpr uint32_t ACCEMPTY_COUNT = 2 * EPI_WARPS;
 constexpr int N_BARS = 4 * STAGES + 2;
 static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1 KiB alignment of 128B-swizzled tiles");
 static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "scale slots exceed the tensor memory");
-static_assert(SMEM <= 232448, "shared memory per CTA");
+static_assert(SMEM_QKNR <= 232448, "shared memory per CTA");
 static_assert(N_BARS * 8 + 4 <= BAR_BYTES, "barrier area");
 
 struct GArgs {
@@ -116,9 +118,15 @@ struct GArgs {
   int Mt, Nt;  // pair tiles along M (256 rows) and N (256 rows of W)
   float alpha;
   uint32_t *err;
+  // fused QKV output stage (QKNR): Y = [Q | K | V], qk_width = heads x 128 columns per section
+  const float *norm_q;  // [128]
+  const float *norm_k;  // [128]
+  const float *rope;    // [M][64][2]: (cos, sin) per token and column pair
+  int qk_width;
+  float eps;
 };
 
-template <int RANK, bool FP4, bool ADD_Y>
+template <int RANK, bool FP4, bool ADD_Y, bool QKNR>
 __global__ void __launch_bounds__(THREADS, 1)
     k2_gemm_w4a4_lora_up(const __grid_constant__ CUtensorMap tm_xq, const __grid_constant__ CUtensorMap tm_wq,
                          const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_l2,
@@ -136,9 +144,12 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  static_assert(!(QKNR && ADD_Y), "the normalized output stage writes Y once");
   uint8_t *ystage = smem + DATA_BYTES;
   float *bias_s = reinterpret_cast<float *>(ystage + YST_BYTES);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(ystage + YST_BYTES + BIAS_BYTES);
+  // QKNR: each output group's copy of the Q and K normalization weights, [half][section][128]
+  float *normw_s = reinterpret_cast<float *>(ystage + YST_BYTES + BIAS_BYTES);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ystage + YST_BYTES + BIAS_BYTES + (QKNR ? NORMW_BYTES : 0u));
   // full[s] (used in the even CTA): stage s is loaded in both CTAs and both CTAs' scales for it
   // are in tensor memory; empty[s]: the MMAs reading stage s are done (both CTAs); accfull: the
   // accumulator is complete (both CTAs); accempty (used in the even CTA): both CTAs' output
@@ -230,6 +241,46 @@ __global__ void __launch_bounds__(THREADS, 1)
             *reinterpret_cast<uint4 *>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(p0, p1, p2, p3);
           }
         };
+        // Fused QKV output stage: the half's 128 columns are one head. For a Q or K head,
+        // u = v w / sqrt(mean(v^2) + eps) with v = alpha acc + bias (fp32, before any 16-bit
+        // rounding), then each column pair (2i, 2i + 1) turns by the token's angle for pair i.
+        auto bias_sumsq = [&](uint32_t(&v32)[32], int colh) {
+          float sq[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float v = fmaf(a.alpha, __uint_as_float(v32[e]), bias_s[half * 128 + colh + e]);
+            v32[e] = __float_as_uint(v);
+            sq[e & 3] = fmaf(v, v, sq[e & 3]);
+          }
+          return (sq[0] + sq[1]) + (sq[2] + sq[3]);
+        };
+        auto qk_store = [&](const uint32_t(&v32)[32], int colh, int sec, float inv) {
+          const float *w = normw_s + (half * 2 + sec) * 128 + colh;
+          const float4 *rp = reinterpret_cast<const float4 *>(a.rope) + static_cast<size_t>(m < a.M ? m : 0) * 32 +
+                             (colh >> 2);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int ch = ((colh & 63) >> 3) + q;
+            float4 cs0 = make_float4(1.f, 0.f, 1.f, 0.f), cs1 = cs0;  // rows beyond M: no rotation
+            if (m < a.M) {
+              cs0 = __ldg(rp + 2 * q);
+              cs1 = __ldg(rp + 2 * q + 1);
+            }
+            const float4 w0 = *reinterpret_cast<const float4 *>(w + 8 * q);
+            const float4 w1 = *reinterpret_cast<const float4 *>(w + 8 * q + 4);
+            const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+            const float cs[8] = {cs0.x, cs0.y, cs0.z, cs0.w, cs1.x, cs1.y, cs1.z, cs1.w};
+            uint32_t p[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const float u0 = __fmul_rn(__fmul_rn(__uint_as_float(v32[8 * q + 2 * i]), inv), wv[2 * i]);
+              const float u1 = __fmul_rn(__fmul_rn(__uint_as_float(v32[8 * q + 2 * i + 1]), inv), wv[2 * i + 1]);
+              const float c = cs[2 * i], sn = cs[2 * i + 1];
+              p[i] = pack_bf16x2(fmaf(u0, c, -__fmul_rn(u1, sn)), fmaf(u1, c, __fmul_rn(u0, sn)));
+            }
+            *reinterpret_cast<uint4 *>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(p[0], p[1], p[2], p[3]);
+          }
+        };
         auto store_box = [&](int colh) {
           fence_proxy_async_smem();
           named_bar_sync(1 + half, 128);
@@ -245,8 +296,15 @@ __global__ void __launch_bounds__(THREADS, 1)
         {
           const int e = half * 128 + et;
           bias_s[e] = (a.bias && n0 + e < a.N) ? __ldg(a.bias + n0 + e) : 0.0f;
+          if (QKNR && tcount == 0) {
+            normw_s[(half * 2 + 0) * 128 + et] = __ldg(a.norm_q + et);
+            normw_s[(half * 2 + 1) * 128 + et] = __ldg(a.norm_k + et);
+          }
         }
         named_bar_sync(1 + half, 128);
+        // section of this half's head: 0 Q, 1 K (normalized and rotated), 2 V
+        const int sec = QKNR ? (n0 + half * 128) / a.qk_width : 2;
+        float inv = 0.0f;
         if (ok) ok = mbar_wait_parked(bar_accfull, tcount & 1, a.err, KID_GEMM, 4);
         ok = __all_sync(0xffffffffu, ok);
         uint32_t r0[32], r1[32], r2[32], r3[32];
@@ -264,16 +322,28 @@ __global__ void __launch_bounds__(THREADS, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive_remote(accempty_lead);
-          convert_store(r0, 0);
-          convert_store(r1, 32);
+          if (QKNR && sec < 2) {
+            const float ss = (bias_sumsq(r0, 0) + bias_sumsq(r1, 32)) + (bias_sumsq(r2, 64) + bias_sumsq(r3, 96));
+            inv = __frsqrt_rn(__fadd_rn(__fmul_rn(ss, 1.0f / 128.0f), a.eps));
+            qk_store(r0, 0, sec, inv);
+            qk_store(r1, 32, sec, inv);
+          } else {
+            convert_store(r0, 0);
+            convert_store(r1, 32);
+          }
         }
         store_box(0);
         // the first store has finished reading the box
         if (et == 0) bulk_wait_read0();
         named_bar_sync(1 + half, 128);
         if (ok) {
-          convert_store(r2, 64);
-          convert_store(r3, 96);
+          if (QKNR && sec < 2) {
+            qk_store(r2, 64, sec, inv);
+            qk_store(r3, 96, sec, inv);
+          } else {
+            convert_store(r2, 64);
+            convert_store(r3, 96);
+          }
         }
         store_box(64);
       } else {
@@ -500,7 +570,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 }
 
 // Pairs that can be resident at once (clusters of two, one CTA per SM), per device.
-template <int RANK, bool FP4, bool ADD_Y>
+template <int RANK, bool FP4, bool ADD_Y, bool QKNR>
 int pair_slots(cudaError_t *err) {
   static int cache[64] = {0};
   int dev = 0;
@@ -510,7 +580,8 @@ int pair_slots(cudaError_t *err) {
     return 0;
   }
   if (cache[dev] > 0) return cache[dev];
-  auto kern = k2_gemm_w4a4_lora_up<RANK, FP4, ADD_Y>;
+  auto kern = k2_gemm_w4a4_lora_up<RANK, FP4, ADD_Y, QKNR>;
+  constexpr uint32_t smem = QKNR ? SMEM_QKNR : SMEM;
   // setmaxnreg.inc would wait forever for registers the block was not launched with: the split
   // must fit the pool of the compiled kernel (registers per thread x threads).
   cudaFuncAttributes fa;
@@ -520,7 +591,7 @@ int pair_slots(cudaError_t *err) {
     *err = cudaErrorLaunchOutOfResources;
     return 0;
   }
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) {
     *err = e;
     return 0;
@@ -528,7 +599,7 @@ int pair_slots(cudaError_t *err) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2, 1, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);
-  cfg.dynamicSmemBytes = SMEM;
+  cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
@@ -546,18 +617,19 @@ int pair_slots(cudaError_t *err) {
   return n;
 }
 
-template <int RANK, bool FP4, bool ADD_Y>
+template <int RANK, bool FP4, bool ADD_Y, bool QKNR>
 cudaError_t launch_t(const GemmLaunch &g) {
   cudaError_t e = cudaSuccess;
-  const int slots = pair_slots<RANK, FP4, ADD_Y>(&e);
+  const int slots = pair_slots<RANK, FP4, ADD_Y, QKNR>(&e);
   if (slots <= 0) return e;
-  GArgs a{g.xs, g.ws, g.bias, g.Y, g.M, g.N, g.K, (g.M + BMP - 1) / BMP, (g.N + BN - 1) / BN, g.alpha, g.err};
+  GArgs a{g.xs,  g.ws, g.bias, g.Y, g.M, g.N, g.K, (g.M + BMP - 1) / BMP, (g.N + BN - 1) / BN, g.alpha, g.err,
+          g.norm_q, g.norm_k, g.rope, g.qk_width, g.eps};
   const int tiles = a.Mt * a.Nt;
   const int pairs = tiles < slots ? tiles : slots;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(2 * pairs, 1, 1);
   cfg.blockDim = dim3(THREADS, 1, 1);
-  cfg.dynamicSmemBytes = SMEM;
+  cfg.dynamicSmemBytes = QKNR ? SMEM_QKNR : SMEM;
   cfg.stream = g.stream;
   cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -568,27 +640,35 @@ cudaError_t launch_t(const GemmLaunch &g) {
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, k2_gemm_w4a4_lora_up<RANK, FP4, ADD_Y>, g.tm_xq, g.tm_wq, g.tm_la, g.tm_l2,
+  return cudaLaunchKernelEx(&cfg, k2_gemm_w4a4_lora_up<RANK, FP4, ADD_Y, QKNR>, g.tm_xq, g.tm_wq, g.tm_la, g.tm_l2,
                             g.tm_y, a);
 }
 
 }  // namespace
 
 cudaError_t launch_gemm(const GemmLaunch &g) {
-  if (g.fp4 && !g.add_y) {
+  if (g.fp4 && !g.add_y && g.qk_norm_rope) {
     switch (g.rank) {
-      case 0: return launch_t<0, true, false>(g);
-      case 16: return launch_t<16, true, false>(g);
-      case 32: return launch_t<32, true, false>(g);
-      case 64: return launch_t<64, true, false>(g);
-      case 128: return launch_t<128, true, false>(g);
+      case 0: return launch_t<0, true, false, true>(g);
+      case 16: return launch_t<16, true, false, true>(g);
+      case 32: return launch_t<32, true, false, true>(g);
+      case 64: return launch_t<64, true, false, true>(g);
+      case 128: return launch_t<128, true, false, true>(g);
+    }
+  } else if (g.fp4 && !g.add_y) {
+    switch (g.rank) {
+      case 0: return launch_t<0, true, false, false>(g);
+      case 16: return launch_t<16, true, false, false>(g);
+      case 32: return launch_t<32, true, false, false>(g);
+      case 64: return launch_t<64, true, false, false>(g);
+      case 128: return launch_t<128, true, false, false>(g);
     }
   } else if (!g.fp4 && g.add_y) {
     switch (g.rank) {
-      case 16: return launch_t<16, false, true>(g);
-      case 32: return launch_t<32, false, true>(g);
-      case 64: return launch_t<64, false, true>(g);
-      case 128: return launch_t<128, false, true>(g);
+      case 16: return launch_t<16, false, true, false>(g);
+      case 32: return launch_t<32, false, true, false>(g);
+      case 64: return launch_t<64, false, true, false>(g);
+      case 128: return launch_t<128, false, true, false>(g);
     }
   }
   return cudaErrorInvalidValue;

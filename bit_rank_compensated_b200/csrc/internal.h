@@ -45,11 +45,22 @@ struct GemmLaunch {
   float alpha;
   bool fp4;    // run the block-scaled 4-bit product
   bool add_y;  // Y = bf16(Y + alpha * acc) instead of bf16(alpha * acc + bias)
+  // Fused QKV output stage: per-head RMS normalization and rotary embedding of the Q and K
+  // sections of Y = [Q | K | V] (head_dim 128, qk_width = heads x 128 columns per section).
+  bool qk_norm_rope;
+  const float *norm_q, *norm_k;  // [128] each
+  const float *rope;             // [M][64][2] (cos, sin)
+  int qk_width;
+  float eps;
   int num_sms;
   uint32_t *err;
   cudaStream_t stream;
 };
 cudaError_t launch_gemm(const GemmLaunch &g);
+
+// Unfused per-head Q/K normalization and rotary embedding of a bf16 Y = [Q | K | V], in place.
+cudaError_t launch_qk_norm_rope(uint16_t *Y, int M, int heads, const float *norm_q, const float *norm_k,
+                                const float *rope, float eps, cudaStream_t st);
 
 // Failure-path self-test (selftest.cu): bounded waits on an mbarrier nobody signals.
 cudaError_t launch_selftest_wait(uint32_t *err, uint64_t limit_ns, cudaStream_t st);

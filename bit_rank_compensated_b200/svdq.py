@@ -28,7 +28,8 @@ EXPORTED = (
     "svdq_prepare_workspace_bytes", "svdq_prepare_weights", "svdq_quantize_rows", "svdq_quant_act_lora_down",
     "svdq_gemm_w4a4_lora_up", "svdq_linear_forward", "svdq_linear_forward_host", "svdq_baseline_lora_down",
     "svdq_baseline_quantize", "svdq_baseline_gemm_w4a4", "svdq_baseline_lora_up", "svdq_last_device_error",
-    "svdq_smoothing_factors_noalloc", "svdq_selftest_wait_timeout",
+    "svdq_smoothing_factors_noalloc", "svdq_selftest_wait_timeout", "svdq_gemm_w4a4_lora_up_qk_norm_rope",
+    "svdq_qk_norm_rope",
 )
 
 
@@ -81,6 +82,8 @@ def load() -> ctypes.CDLL:
         "svdq_last_device_error": ([P, ctypes.POINTER(ctypes.c_uint32)], I),
         "svdq_selftest_wait_timeout": ([ctypes.c_uint32, P], I),
         "svdq_smoothing_factors_noalloc": ([P, P, I, I, P, P, P, P], I),
+        "svdq_gemm_w4a4_lora_up_qk_norm_rope": ([P, P, P, I, LP, I, I, P, P, P, F, P, P], I),
+        "svdq_qk_norm_rope": ([P, I, I, I, P, P, P, F, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -244,6 +247,25 @@ def gemm_w4a4_lora_up(xq, xs, lora_act, M: int, layer: Layer, Y=None, stream=Non
         Y = torch.empty(M, layer.N, dtype=torch.bfloat16, device=xq.device)
     _check("svdq_gemm_w4a4_lora_up", load().svdq_gemm_w4a4_lora_up(
         _ptr(xq), _ptr(xs), _ptr(lora_act), M, ctypes.byref(layer.s), _ptr(Y), _stream(stream)))
+    return Y
+
+
+def gemm_w4a4_lora_up_qk_norm_rope(xq, xs, lora_act, M: int, layer: Layer, heads: int, norm_q, norm_k, rope,
+                                   eps: float = 1e-6, Y=None, stream=None, head_dim: int = 128):
+    """K2 with the fused QKV output stage: Y = [Q | K | V], Q and K heads RMS-normalized with
+    norm_q / norm_k (fp32 [head_dim]) and turned by the (cos, sin) table rope (fp32 [M, 64, 2])."""
+    if Y is None:
+        Y = torch.empty(M, layer.N, dtype=torch.bfloat16, device=xq.device)
+    _check("svdq_gemm_w4a4_lora_up_qk_norm_rope", load().svdq_gemm_w4a4_lora_up_qk_norm_rope(
+        _ptr(xq), _ptr(xs), _ptr(lora_act), M, ctypes.byref(layer.s), heads, head_dim, _ptr(norm_q), _ptr(norm_k),
+        _ptr(rope), float(eps), _ptr(Y), _stream(stream)))
+    return Y
+
+
+def qk_norm_rope(Y, heads: int, norm_q, norm_k, rope, eps: float = 1e-6, stream=None, head_dim: int = 128):
+    """Unfused step: normalizes and rotates the Q and K sections of a bf16 Y in place."""
+    _check("svdq_qk_norm_rope", load().svdq_qk_norm_rope(
+        _ptr(Y), Y.shape[0], heads, head_dim, _ptr(norm_q), _ptr(norm_k), _ptr(rope), float(eps), _stream(stream)))
     return Y
 
 

@@ -171,6 +171,35 @@ SVDQ_API svdq_status svdq_quant_act_lora_down(const uint16_t *X, int M, const sv
 SVDQ_API svdq_status svdq_gemm_w4a4_lora_up(const uint8_t *xq, const uint8_t *xs, const uint16_t *lora_act,
                                    int M, const svdq_layer *layer, uint16_t *Y, void *stream);
 
+/* K2 with the output stage of the fused QKV projection ("Nunchaku Lite in Diffusers", section on
+ * quantized models with structural rewrites: the engine's operator takes the concatenated
+ * to_qkv projection together with the Q/K normalizations norm_q, norm_k and the rotary
+ * embedding, which the default path runs as separate steps):
+ *   Y = [Q | K | V] along N, each section heads x head_dim columns (head_dim must be 128, so
+ *   layer->N == 3 * heads * 128); v = alpha * acc + bias as in svdq_gemm_w4a4_lora_up (fp32);
+ *   for every head of Q and K:  u = v * w / sqrt(mean(v^2) + eps)  (w = norm_q_weight for Q,
+ *   norm_k_weight for K), then each column pair (2i, 2i + 1) of the head turns by token m's
+ *   angle for pair i:  (u0, u1) -> (u0 cos - u1 sin, u1 cos + u0 sin);  V: bf16(v) unchanged.
+ *   The normalization reads the fp32 values before any 16-bit rounding; Y is written once.
+ *   norm_q_weight, norm_k_weight  device, 128 fp32 each.
+ *   rope                          device, M x 64 x 2 fp32: (cos, sin) per token and pair.
+ *   eps                           > 0 or 0 (added to the mean square).
+ * Errors: SVDQ_ERR_INVALID_ARG for head_dim != 128 or N != 3 * heads * 128; otherwise as
+ * svdq_gemm_w4a4_lora_up. Asynchronous on stream. */
+SVDQ_API svdq_status svdq_gemm_w4a4_lora_up_qk_norm_rope(const uint8_t *xq, const uint8_t *xs,
+                                                         const uint16_t *lora_act, int M,
+                                                         const svdq_layer *layer, int heads, int head_dim,
+                                                         const float *norm_q_weight, const float *norm_k_weight,
+                                                         const float *rope, float eps, uint16_t *Y,
+                                                         void *stream);
+
+/* Unfused baseline of the step above: the per-head normalization and rotary embedding of the
+ * Q and K sections of a bf16 Y = [Q | K | V] that a plain projection has already written
+ * (M x 3 * heads * 128, modified in place; it reads the 16-bit values back and rewrites them).
+ * Same weights, table and eps as svdq_gemm_w4a4_lora_up_qk_norm_rope. Asynchronous on stream. */
+SVDQ_API svdq_status svdq_qk_norm_rope(uint16_t *Y, int M, int heads, int head_dim, const float *norm_q_weight,
+                                       const float *norm_k_weight, const float *rope, float eps, void *stream);
+
 /* K1 then K2 on the same stream (the layer's forward pass). Buffers as above. */
 SVDQ_API svdq_status svdq_linear_forward(const uint16_t *X, int M, const svdq_layer *layer,
                                 uint8_t *xq, uint8_t *xs, uint16_t *lora_act,
