@@ -210,9 +210,12 @@ svdq_status run_gemm(const uint8_t *xq, const uint8_t *xs, const uint16_t *la, i
     g.qk_norm_rope = true;
     g.norm_q = qk->norm_q;
     g.norm_k = qk->norm_k;
-    g.rope = qk->rope;
     g.qk_width = qk->heads * 128;
     g.eps = qk->eps;
+    // rotary table [M][64 pairs][cos, sin] as M rows of 128 fp32, staged 32 floats x 128 rows per box
+    if (!make_map(&g.tm_rope, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, qk->rope, 128, M, 512, 32, 128,
+                  CU_TENSOR_MAP_SWIZZLE_128B))
+      return SVDQ_ERR_CUDA;
   }
   g.num_sms = d->num_sms;
   g.err = d->err;

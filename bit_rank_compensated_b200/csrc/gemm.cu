@@ -64,6 +64,27 @@
 namespace svdq {
 namespace {
 
+// Two fp32 values in one 64-bit register, for the packed f32x2 arithmetic of the fused QKV
+// output stage (each lane of a packed op rounds like its scalar counterpart).
+__device__ __forceinline__ uint64_t pk2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void upk2(uint64_t v, float &lo, float &hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t mul2_rn(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t fma2_rn(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+
 constexpr int BM = 128;      // rows of X per CTA
 constexpr int BMP = 2 * BM;  // rows of X per pair tile
 constexpr int BN = 256;      // rows of W per pair tile
@@ -80,10 +101,16 @@ constexpr uint32_t STAGE_BYTES = A_BYTES + B_BYTES + SF_STAGE_BYTES;  // 38 KiB
 constexpr uint32_t DATA_BYTES = STAGES * STAGE_BYTES;
 constexpr uint32_t YST_BYTES = BM * 64 * 2 * 2;  // bf16 output staging: one box of 128 rows x 64 columns per half
 constexpr uint32_t BIAS_BYTES = BN * 4;
-constexpr uint32_t NORMW_BYTES = 2 * 2 * 128 * 4;  // fused QKV output stage only
 constexpr uint32_t BAR_BYTES = 256;
 constexpr uint32_t SMEM = DATA_BYTES + YST_BYTES + BIAS_BYTES + BAR_BYTES + 1024;
-constexpr uint32_t SMEM_QKNR = SMEM + NORMW_BYTES;
+// Fused QKV output stage (QKNR): four ring stages instead of five make room for the rotary
+// table rows of the tile (128 rows x 32 column pairs x (cos, sin) fp32, 32 KiB, one half of the
+// head's pairs at a time) and the two normalization weight vectors.
+constexpr int STAGES_QKNR = 4;
+constexpr uint32_t ROPE_BYTES = 128 * 32 * 2 * 4;
+constexpr uint32_t NORMW_BYTES = 2 * 2 * 128 * 4;
+constexpr uint32_t SMEM_QKNR =
+    STAGES_QKNR * STAGE_BYTES + ROPE_BYTES + YST_BYTES + BIAS_BYTES + NORMW_BYTES + BAR_BYTES + 1024;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint32_t SF_COL0 = 256;  // one scale slot per stage follows the accumulator
 constexpr uint32_t SF_COLS = 48;   // per slot: 4 k-blocks x (4 SFA + 8 SFB) columns
@@ -103,7 +130,7 @@ constexpr uint32_t SF_GROUP_WARPS = 4;
 constexpr uint32_t EPI_WARPS = 8;
 constexpr uint32_t FULL_COUNT = 1 + 2 * SF_GROUP_WARPS;
 constexpr uint32_t ACCEMPTY_COUNT = 2 * EPI_WARPS;
-constexpr int N_BARS = 4 * STAGES + 2;
+constexpr int N_BARS = 4 * STAGES + 2 + 2;  // + rope_full, rope_empty (QKNR)
 static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1 KiB alignment of 128B-swizzled tiles");
 static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "scale slots exceed the tensor memory");
 static_assert(SMEM_QKNR <= 232448, "shared memory per CTA");
@@ -121,7 +148,6 @@ struct GArgs {
   // fused QKV output stage (QKNR): Y = [Q | K | V], qk_width = heads x 128 columns per section
   const float *norm_q;  // [128]
   const float *norm_k;  // [128]
-  const float *rope;    // [M][64][2]: (cos, sin) per token and column pair
   int qk_width;
   float eps;
 };
@@ -130,7 +156,8 @@ template <int RANK, bool FP4, bool ADD_Y, bool QKNR>
 __global__ void __launch_bounds__(THREADS, 1)
     k2_gemm_w4a4_lora_up(const __grid_constant__ CUtensorMap tm_xq, const __grid_constant__ CUtensorMap tm_wq,
                          const __grid_constant__ CUtensorMap tm_la, const __grid_constant__ CUtensorMap tm_l2,
-                         const __grid_constant__ CUtensorMap tm_y, GArgs a) {
+                         const __grid_constant__ CUtensorMap tm_y, const __grid_constant__ CUtensorMap tm_rope,
+                         GArgs a) {
   // Low-rank steps: kc columns of lora_act (hi and lo planes) and of L2t per step.
   constexpr int KC = RANK == 0 ? 32 : (RANK < 32 ? RANK : 32);
   constexpr int N_LORA = RANK == 0 ? 0 : RANK / KC;
@@ -145,7 +172,15 @@ __global__ void __launch_bounds__(THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   static_assert(!(QKNR && ADD_Y), "the normalized output stage writes Y once");
-  uint8_t *ystage = smem + DATA_BYTES;
+  // Ring stages; a writer group meets the same (stage, step parity) pair again after
+  // SF_PERIOD steps (2 ST for an odd stage count, ST for an even one).
+  constexpr int ST = QKNR ? STAGES_QKNR : STAGES;
+  constexpr int SF_PERIOD = (ST % 2) ? 2 * ST : ST;
+  static_assert(ST <= STAGES, "barrier area is sized for STAGES");
+  // QKNR: the rotary rows of the tile (two 16 KiB boxes of 128 rows x 32 floats, 128B swizzle),
+  // filled twice per tile (column pairs 0-31, then 32-63)
+  uint8_t *rope_s = smem + ST * STAGE_BYTES;
+  uint8_t *ystage = rope_s + (QKNR ? ROPE_BYTES : 0u);
   float *bias_s = reinterpret_cast<float *>(ystage + YST_BYTES);
   // QKNR: each output group's copy of the Q and K normalization weights, [half][section][128]
   float *normw_s = reinterpret_cast<float *>(ystage + YST_BYTES + BIAS_BYTES);
@@ -162,6 +197,10 @@ __global__ void __launch_bounds__(THREADS, 1)
   // by the producer's order, the MMAs that last read slot s are done). Even and odd steps have
   // barriers of their own, so each writer group waits on phases ten steps apart.
   const uint32_t bar_sf = bar_accempty + 8;
+  // QKNR: rope_full (the pass's rotary rows have landed), rope_empty (the eight output warps of
+  // this CTA are done reading them)
+  const uint32_t bar_rope_full = bar_sf + 8 * 2 * STAGES;
+  const uint32_t bar_rope_empty = bar_rope_full + 8;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + N_BARS);
 
   const int warp = threadIdx.x >> 5;
@@ -185,6 +224,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     mbar_init(bar_accfull, 1);
     mbar_init(bar_accempty, ACCEMPTY_COUNT);
     for (int s = 0; s < 2 * STAGES; ++s) mbar_init(bar_sf + 8 * s, 1);
+    if (QKNR) {
+      mbar_init(bar_rope_full, 1);
+      mbar_init(bar_rope_empty, EPI_WARPS);
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -245,40 +288,72 @@ __global__ void __launch_bounds__(THREADS, 1)
         // u = v w / sqrt(mean(v^2) + eps) with v = alpha acc + bias (fp32, before any 16-bit
         // rounding), then each column pair (2i, 2i + 1) turns by the token's angle for pair i.
         auto bias_sumsq = [&](uint32_t(&v32)[32], int colh) {
-          float sq[4] = {0.f, 0.f, 0.f, 0.f};
+          const uint64_t al2 = pk2(a.alpha, a.alpha);
+          uint64_t sq0 = 0, sq1 = 0;  // packed (+0, +0)
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float v = fmaf(a.alpha, __uint_as_float(v32[e]), bias_s[half * 128 + colh + e]);
-            v32[e] = __float_as_uint(v);
-            sq[e & 3] = fmaf(v, v, sq[e & 3]);
+          for (int e = 0; e < 16; ++e) {
+            const float2 b = *reinterpret_cast<const float2 *>(bias_s + half * 128 + colh + 2 * e);
+            const uint64_t v = fma2_rn(al2, pk2(__uint_as_float(v32[2 * e]), __uint_as_float(v32[2 * e + 1])),
+                                       pk2(b.x, b.y));
+            float lo, hi;
+            upk2(v, lo, hi);
+            v32[2 * e] = __float_as_uint(lo);
+            v32[2 * e + 1] = __float_as_uint(hi);
+            if (e & 1) sq1 = fma2_rn(v, v, sq1);
+            else sq0 = fma2_rn(v, v, sq0);
           }
-          return (sq[0] + sq[1]) + (sq[2] + sq[3]);
+          float a0, a1, b0, b1;
+          upk2(sq0, a0, a1);
+          upk2(sq1, b0, b1);
+          return (a0 + a1) + (b0 + b1);
         };
+        // The pair's (cos, sin) of the token come from the staged rotary rows: box (colh & 63) / 32
+        // of the current pass holds pairs 16 ((colh & 63) / 32) .. + 15 of each row, 16-byte
+        // chunk k of row r at k ^ (r % 8).
+        const uint32_t rope_row = smem_u32(rope_s) + row * 128;
         auto qk_store = [&](const uint32_t(&v32)[32], int colh, int sec, float inv) {
           const float *w = normw_s + (half * 2 + sec) * 128 + colh;
-          const float4 *rp = reinterpret_cast<const float4 *>(a.rope) + static_cast<size_t>(m < a.M ? m : 0) * 32 +
-                             (colh >> 2);
+          const uint32_t rb = rope_row + ((colh & 63) >> 5) * (ROPE_BYTES / 2);
+          const uint64_t inv2 = pk2(inv, inv);
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
             const int ch = ((colh & 63) >> 3) + q;
-            float4 cs0 = make_float4(1.f, 0.f, 1.f, 0.f), cs1 = cs0;  // rows beyond M: no rotation
-            if (m < a.M) {
-              cs0 = __ldg(rp + 2 * q);
-              cs1 = __ldg(rp + 2 * q + 1);
-            }
+            const uint4 c0 = ld_shared_u32x4(rb + (((2 * q) ^ (row & 7)) << 4));
+            const uint4 c1 = ld_shared_u32x4(rb + (((2 * q + 1) ^ (row & 7)) << 4));
             const float4 w0 = *reinterpret_cast<const float4 *>(w + 8 * q);
             const float4 w1 = *reinterpret_cast<const float4 *>(w + 8 * q + 4);
             const float wv[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
-            const float cs[8] = {cs0.x, cs0.y, cs0.z, cs0.w, cs1.x, cs1.y, cs1.z, cs1.w};
+            const uint32_t cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
             uint32_t p[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              const float u0 = __fmul_rn(__fmul_rn(__uint_as_float(v32[8 * q + 2 * i]), inv), wv[2 * i]);
-              const float u1 = __fmul_rn(__fmul_rn(__uint_as_float(v32[8 * q + 2 * i + 1]), inv), wv[2 * i + 1]);
-              const float c = cs[2 * i], sn = cs[2 * i + 1];
-              p[i] = pack_bf16x2(fmaf(u0, c, -__fmul_rn(u1, sn)), fmaf(u1, c, __fmul_rn(u0, sn)));
+              // (u0, u1) = (v0, v1) inv w;  z = (u0 c - u1 s, u1 c + u0 s)
+              const uint64_t u = mul2_rn(mul2_rn(pk2(__uint_as_float(v32[8 * q + 2 * i]),
+                                                     __uint_as_float(v32[8 * q + 2 * i + 1])), inv2),
+                                         pk2(wv[2 * i], wv[2 * i + 1]));
+              const float c = __uint_as_float(cs[2 * i]), sn = __uint_as_float(cs[2 * i + 1]);
+              float u0, u1;
+              upk2(u, u0, u1);
+              const uint64_t z = fma2_rn(pk2(u1, u0), pk2(-sn, sn), mul2_rn(u, pk2(c, c)));
+              float z0, z1;
+              upk2(z, z0, z1);
+              p[i] = pack_bf16x2(z0, z1);
             }
             *reinterpret_cast<uint4 *>(rowp + ((ch ^ (row & 7)) << 4)) = make_uint4(p[0], p[1], p[2], p[3]);
+          }
+        };
+        // A pass of rotary rows: every output warp waits for it (so that no early arrival on
+        // rope_empty can let the filler start the next pass over rows still being read) and
+        // reports once it is done with it. Pass A (pairs 0-31) has phase parity 0, pass B 1.
+        // Tiles whose two heads both lie in V get no rotary passes (the filler skips them too).
+        const bool rope_tile = QKNR && n0 < 2 * a.qk_width;
+        auto rope_wait = [&](uint32_t parity) {
+          if (rope_tile && ok) ok = __all_sync(0xffffffffu, mbar_wait_parked(bar_rope_full, parity, a.err, KID_GEMM, 10));
+        };
+        auto rope_done = [&]() {
+          if (rope_tile && ok) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_rope_empty);
           }
         };
         auto store_box = [&](int colh) {
@@ -305,6 +380,9 @@ __global__ void __launch_bounds__(THREADS, 1)
         // section of this half's head: 0 Q, 1 K (normalized and rotated), 2 V
         const int sec = QKNR ? (n0 + half * 128) / a.qk_width : 2;
         float inv = 0.0f;
+        // pass A of the tile's rotary rows is loaded while the tile's MMAs run: wait for it
+        // before the accumulator's 128 columns take up the registers
+        rope_wait(0);
         if (ok) ok = mbar_wait_parked(bar_accfull, tcount & 1, a.err, KID_GEMM, 4);
         ok = __all_sync(0xffffffffu, ok);
         uint32_t r0[32], r1[32], r2[32], r3[32];
@@ -331,19 +409,24 @@ __global__ void __launch_bounds__(THREADS, 1)
             convert_store(r0, 0);
             convert_store(r1, 32);
           }
+          rope_done();
         }
         store_box(0);
         // the first store has finished reading the box
         if (et == 0) bulk_wait_read0();
         named_bar_sync(1 + half, 128);
         if (ok) {
+          rope_wait(1);
           if (QKNR && sec < 2) {
-            qk_store(r2, 64, sec, inv);
-            qk_store(r3, 96, sec, inv);
+            if (ok) {
+              qk_store(r2, 64, sec, inv);
+              qk_store(r3, 96, sec, inv);
+            }
           } else {
             convert_store(r2, 64);
             convert_store(r3, 96);
           }
+          rope_done();
         }
         store_box(64);
       } else {
@@ -401,10 +484,10 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int row0 = mt * BMP + static_cast<int>(crank) * BM;  // this CTA's rows of X
           const int wrow0 = nt * BN + static_cast<int>(crank) * BNH;  // this CTA's rows of W
           for (int j = 0; j < total; ++j, ++it) {
-            const int s = it % STAGES;
+            const int s = it % ST;
             // spin rather than park: a parked thread wakes measurably later, and this round trip
             // (slot released -> loads issued -> stage full) is the kernel's critical path
-            if (it >= STAGES && !mbar_wait(bar_empty + 8 * s, ((it / STAGES) - 1) & 1, a.err, KID_GEMM, 1)) {
+            if (it >= ST && !mbar_wait(bar_empty + 8 * s, ((it / ST) - 1) & 1, a.err, KID_GEMM, 1)) {
               ok = false;
               break;
             }
@@ -439,8 +522,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
         }
         // The MMA issuer's last commits to this CTA's empty barriers have landed before it exits.
-        for (uint32_t i = it > STAGES ? it - STAGES : 0; ok && i < it; ++i)
-          ok = mbar_wait(bar_empty + 8 * (i % STAGES), (i / STAGES) & 1, a.err, KID_GEMM, 7);
+        for (uint32_t i = it > ST ? it - ST : 0; ok && i < it; ++i)
+          ok = mbar_wait(bar_empty + 8 * (i % ST), (i / ST) & 1, a.err, KID_GEMM, 7);
       }
     } else if (warp == 1) {
       // ------------------------------------------------------------ MMA issuer (even CTA)
@@ -463,8 +546,8 @@ __global__ void __launch_bounds__(THREADS, 1)
           }
           tc_fence_after();
           for (int j = 0; j < total; ++j, ++it) {
-            const int s = it % STAGES;
-            const uint32_t par = (it / STAGES) & 1;
+            const int s = it % ST;
+            const uint32_t par = (it / ST) & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(bar_full + 8 * s, par, a.err, KID_GEMM, 3))) {
               ok = false;
               break;
@@ -509,6 +592,33 @@ __global__ void __launch_bounds__(THREADS, 1)
         // both CTAs' output stages have released the last accumulator
         if (ok && tcount > 0) mbar_wait(bar_accempty, (tcount - 1) & 1, a.err, KID_GEMM, 8);
       }
+    } else if (QKNR && warp == 18) {
+      // ------------------------------------------------------------ rotary-row filler (QKNR)
+      // Per tile two passes over this CTA's 128 rows of the (cos, sin) table: pairs 0-31 for
+      // the output stage's first box of columns, then pairs 32-63. A pass reuses the buffer once
+      // the eight output warps have read the previous one; the first pass of a tile is loaded
+      // while the tile's MMAs run. Rows beyond M are filled with zeros by the copy (never stored).
+      if (lane == 0) {
+        tma_prefetch_desc(&tm_rope);
+        const uint32_t rs = smem_u32(rope_s);
+        uint32_t pass = 0;
+        bool ok = true;
+        for (int t = pid; t < tiles && ok; t += npairs) {
+          const int row0 = (t % a.Mt) * BMP + static_cast<int>(crank) * BM;
+          if ((t / a.Mt) * BN >= 2 * a.qk_width) continue;  // both heads in V: no rotation
+          for (int ph = 0; ph < 2; ++ph, ++pass) {
+            if (pass > 0 && !mbar_wait(bar_rope_empty, (pass - 1) & 1, a.err, KID_GEMM, 9)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(bar_rope_full, ROPE_BYTES);
+            tma_load_2d(rs, &tm_rope, 64 * ph, row0, bar_rope_full);
+            tma_load_2d(rs + ROPE_BYTES / 2, &tm_rope, 64 * ph + 32, row0, bar_rope_full);
+          }
+        }
+        // the last pass has landed before the CTA can exit
+        if (pass > 0) mbar_wait(bar_rope_full, (pass - 1) & 1, a.err, KID_GEMM, 11);
+      }
     } else if ((warp >= 2 && warp < EPI_WARP0) || warp == 16 || warp == 17) {
       // ------------------------------------------------------------ scale-factor writers
       // Warp (q, h) writes tensor-memory lanes 32 q .. 32 q + 31 for the steps of parity h (two
@@ -523,10 +633,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int my_tiles = tiles > pid ? (tiles - 1 - pid) / npairs + 1 : 0;
       const int nsteps = my_tiles * total;
       for (int step = h; step < nsteps; step += 2) {
-        const int s = step % STAGES;
+        const int s = step % ST;
         const int j = step % total;
         // sffull of this step: its scale blocks are in shared memory and slot s is free
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * (2 * s + h), (step / (2 * STAGES)) & 1, a.err, KID_GEMM, 6)))
+        if (!__all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * (2 * s + h), (step / SF_PERIOD) & 1, a.err, KID_GEMM, 6)))
           break;
         if (FP4 && j >= N_LORA) {
           const int kt = j - N_LORA;
@@ -622,8 +732,8 @@ cudaError_t launch_t(const GemmLaunch &g) {
   cudaError_t e = cudaSuccess;
   const int slots = pair_slots<RANK, FP4, ADD_Y, QKNR>(&e);
   if (slots <= 0) return e;
-  GArgs a{g.xs,  g.ws, g.bias, g.Y, g.M, g.N, g.K, (g.M + BMP - 1) / BMP, (g.N + BN - 1) / BN, g.alpha, g.err,
-          g.norm_q, g.norm_k, g.rope, g.qk_width, g.eps};
+  GArgs a{g.xs,     g.ws,     g.bias,       g.Y,  g.M, g.N, g.K, (g.M + BMP - 1) / BMP, (g.N + BN - 1) / BN,
+          g.alpha, g.err, g.norm_q, g.norm_k, g.qk_width, g.eps};
   const int tiles = a.Mt * a.Nt;
   const int pairs = tiles < slots ? tiles : slots;
   cudaLaunchConfig_t cfg = {};
@@ -641,7 +751,7 @@ cudaError_t launch_t(const GemmLaunch &g) {
   cfg.attrs = attr;
   cfg.numAttrs = 2;
   return cudaLaunchKernelEx(&cfg, k2_gemm_w4a4_lora_up<RANK, FP4, ADD_Y, QKNR>, g.tm_xq, g.tm_wq, g.tm_la, g.tm_l2,
-                            g.tm_y, a);
+                            g.tm_y, QKNR ? g.tm_rope : g.tm_y, a);
 }
 
 }  // namespace

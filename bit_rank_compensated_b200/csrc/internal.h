@@ -37,6 +37,7 @@ struct GemmLaunch {
   CUtensorMap tm_la;  // lora_act, bf16 [M, 2 rank] (hi | lo planes), box kc x 128
   CUtensorMap tm_l2;  // L2t, bf16 [N, rank], box kc x 128 (half a pair tile)
   CUtensorMap tm_y;   // Y, bf16 [M, N], box 64 x 128, 128B swizzle (output stores)
+  CUtensorMap tm_rope;  // rotary table, fp32 [M, 128], box 32 x 128, 128B swizzle (QKNR only)
   const uint8_t *xs;  // activation scales (block layout, ceil(M / 128) row blocks)
   const uint8_t *ws;  // weight scales (block layout, rows padded to 256)
   const float *bias;
@@ -49,7 +50,6 @@ struct GemmLaunch {
   // sections of Y = [Q | K | V] (head_dim 128, qk_width = heads x 128 columns per section).
   bool qk_norm_rope;
   const float *norm_q, *norm_k;  // [128] each
-  const float *rope;             // [M][64][2] (cos, sin)
   int qk_width;
   float eps;
   int num_sms;
