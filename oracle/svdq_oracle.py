@@ -373,3 +373,54 @@ def qk_norm_rope(Y, heads: int, head_dim: int, norm_q_weight, norm_k_weight, cos
         U = rms_norm_heads(block, w, eps)
         Z[:, sec * width:(sec + 1) * width] = rotary_pairs(U, cos, sin).reshape(M, width)
     return Z
+
+
+# --------------------------------------------------------------------------- awq_w4a16
+# "Nunchaku Lite in Diffusers": the second kernel family, awq_w4a16 (4-bit weights, 16-bit
+# activations), serves the adaptive-normalization / modulation projections (FLUX's
+# adaLN_modulation), which are memory-bound and precision-sensitive; its quantization_config
+# entry fixes precision int4 and group_size 64.
+# Readings (the page gives no formulas):
+#   * groups of 64 consecutive input channels of a weight row share one scale and one zero
+#     point (AWQ's asymmetric storage): W_hat[n, k] = (q[n, k] - z[n, g]) * s[n, g], q and z in
+#     0 .. 15, s stored as fp16;
+#   * the codes come from round-to-nearest on the group's range, decided in fp32:
+#       range = fp32(max - min), raised to fp32(1e-5) when smaller;
+#       s = fp16(fp32(range / 15));
+#       z = clamp(rint(fp32(-min / s)), 0, 15);   q = clamp(rint(fp32(w / s)) + z, 0, 15)
+#     (rint: nearest, ties to even).  AWQ's activation-aware search for per-channel scales is a
+#     calibration procedure the pages do not describe; it would change W before this step.
+#   * Y = X W_hat^T + b with 16-bit X and the output rounded to bf16 once.
+AWQ_GROUP = 64
+
+
+def f16(x):
+    """Round fp64 values to fp16 (nearest, ties to even); return them as fp64."""
+    return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
+def awq_quantize(W, group: int = AWQ_GROUP):
+    """Int4 codes q (N, K) uint8, fp16 scales s (N, K/group) as fp64, zeros z (N, K/group) uint8."""
+    W = np.asarray(W, dtype=np.float64)
+    N, K = W.shape
+    G = W.reshape(N, K // group, group)
+    mx = G.max(axis=2)
+    mn = G.min(axis=2)
+    rng = f32(mx - mn)
+    rng = np.where(rng < f32(1e-5), f32(1e-5), rng)
+    s = f16(f32(rng / 15.0))
+    z = np.clip(np.rint(f32(-mn / s)), 0, 15)
+    q = np.clip(np.rint(f32(G / s[:, :, None])) + z[:, :, None], 0, 15)
+    return q.reshape(N, K).astype(np.uint8), s, z.astype(np.uint8)
+
+
+def awq_dequantize(q, s, z, group: int = AWQ_GROUP):
+    N, K = q.shape
+    qg = q.reshape(N, K // group, group).astype(np.float64)
+    return ((qg - z[:, :, None].astype(np.float64)) * s[:, :, None]).reshape(N, K)
+
+
+def awq_linear(Xv, q, s, z, bias=None, group: int = AWQ_GROUP):
+    """Y = X W_hat^T + b in fp64 (W_hat the dequantized int4 weight)."""
+    Y = np.asarray(Xv, dtype=np.float64) @ awq_dequantize(q, s, z, group).T
+    return Y if bias is None else Y + np.asarray(bias, dtype=np.float64)[None, :]

@@ -30,6 +30,10 @@ Inputs of the fused QKV output stage (per-head Q/K normalization and rotary embe
 tokens on a 64-wide latent grid, three position axes of 16, 56 and 56 head columns, base
 10000) as a (cos, sin) table per token and column pair, angles in fp64 rounded to fp32;
 ``qk_norm_weights`` draws the two normalization weight vectors ~ N(1, 0.1^2).
+
+Inputs of the 4-bit-weight modulation projection (awq_w4a16): FLUX's adaptive-normalization
+linear reads SiLU of the conditioning embedding, so X = SiLU(Z), Z ~ N(0, 1), rounded to bf16;
+W ~ N(0, 0.02^2) fp32, b ~ N(0, 0.01^2) (``make_modulation_inputs``).
 """
 from __future__ import annotations
 
@@ -47,6 +51,7 @@ __all__ = [
     "bf16_bits_to_f32",
     "rope_table",
     "qk_norm_weights",
+    "make_modulation_inputs",
 ]
 
 
@@ -169,3 +174,13 @@ def qk_norm_weights(head_dim: int = 128, seed: int = 0):
     """Weights of the Q and K normalizations, float32 [head_dim] each, ~ N(1, 0.1^2)."""
     rng = np.random.Generator(np.random.PCG64(seed + 1000))
     return (rng.normal(1.0, 0.1, head_dim).astype(np.float32), rng.normal(1.0, 0.1, head_dim).astype(np.float32))
+
+
+def make_modulation_inputs(M: int, K: int, N: int, seed: int = 0):
+    """(X_bf16_bits [M, K] uint16, W [N, K] float32, b [N] float32) for a modulation projection."""
+    rng = np.random.Generator(np.random.PCG64(seed + 2000))
+    Z = rng.standard_normal((M, K))
+    X = Z / (1.0 + np.exp(-Z))
+    W = rng.normal(0.0, 0.02, (N, K))
+    b = rng.normal(0.0, 0.01, N)
+    return f32_to_bf16_bits(X.astype(np.float32)), W.astype(np.float32), b.astype(np.float32)
