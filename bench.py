@@ -238,7 +238,43 @@ def time_graphs(stream, graphs):
     return [evs[k].elapsed_time(evs[k + 1]) for k in range(len(graphs))]
 
 
-SUITE = ["qkv", "qkv_qknorm_rope", "mlp_up", "mlp_down", "sweep_m256", "sweep_m1024", "sweep_m4096", "sweep_m16384",
+AWQ_WORKLOADS = {"awq_mod": (1, 3072, 18432), "awq_mod_m2": (2, 3072, 18432)}
+
+
+def awq_bytes(M, K, N):
+    """Algorithmic HBM bytes of the 4-bit-weight GEMV: int4 codes, fp16 scales and zero points
+    (3 bytes per group of 64; the packed layout carries 4, counted as 3), bf16 X and Y, fp32 bias."""
+    return N * K / 2.0 + N * (K / 64) * 3.0 + 2.0 * M * K + 2.0 * M * N + 4.0 * N
+
+
+def time_awq(M, K, N, steps, warmup, dev, stream, nb=5):
+    """Mean device time (ms) of svdq_awq_gemv_w4a16 over K back-to-back launches (one graph),
+    rotating over `nb` weight sets (more bytes than the L2 holds)."""
+    import torch
+    from bit_rank_compensated_b200 import svdq
+    from synth import make_modulation_inputs
+
+    Xb, W, b = make_modulation_inputs(M, K, N)
+    X = torch.from_numpy(Xb.view(np.int16)).to(dev).view(torch.bfloat16)
+    bias = torch.from_numpy(b).to(dev)
+    sets = [svdq.AwqLinear.from_float(torch.from_numpy(W).to(dev), bias) for _ in range(nb)]
+    Ys = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(nb)]
+
+    def launch(i):
+        return [lambda st: svdq.awq_gemv_w4a16(X, sets[i % nb], Ys[i % nb], st)]
+
+    for i in range(warmup):
+        launch(i)[0](stream)
+    torch.cuda.synchronize()
+    g = capture_sequence(steps, launch)
+    g.replay()
+    torch.cuda.synchronize()
+    (total,) = time_graphs(stream, [g])
+    assert svdq.last_device_error() == 0
+    return total / steps
+
+
+SUITE = ["qkv", "qkv_qknorm_rope", "awq_mod", "awq_mod_m2", "mlp_up", "mlp_down", "sweep_m256", "sweep_m1024", "sweep_m4096", "sweep_m16384",
          "sweep_r0", "sweep_r16", "sweep_r32", "sweep_r64", "sweep_r128"]
 HEAD_DIM = 128
 
@@ -332,6 +368,21 @@ def run_suite(args):
     r0_ms = None
     plain_k2 = {}
     for name in args.suite.split(","):
+        if name in AWQ_WORKLOADS:
+            M, K, N = AWQ_WORKLOADS[name]
+            ms = time_awq(M, K, N, args.steps, args.warmup, dev, stream)
+            gbs = awq_bytes(M, K, N) / (ms * 1e-3) / 1e9
+            print(json.dumps({
+                "metric": "awq_w4a16 modulation GEMV HBM GB/s", "value": gbs, "unit": "GB/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "dtype": "int4 x bf16 -> fp32", "data": "synthetic",
+                "config": {"workload": f"{name}: awq_w4a16 GEMV M={M} K={K} N={N} (FLUX double-block modulation)",
+                           "M": M, "K": K, "N": N},
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
+                             "bytes_per_launch": awq_bytes(M, K, N)},
+                "peaks": peak_kind}), flush=True)
+            torch.cuda.empty_cache()
+            continue
         qknr = name.endswith("_qknorm_rope")
         shape = CONFIGS[name[:-len("_qknorm_rope")] if qknr else name]
         M, K, N, r = shape.M, shape.K, shape.N, shape.rank

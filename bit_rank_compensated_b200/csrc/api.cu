@@ -407,6 +407,51 @@ svdq_status svdq_qk_norm_rope(uint16_t *Y, int M, int heads, int head_dim, const
              : SVDQ_ERR_CUDA;
 }
 
+svdq_status svdq_awq_quantize_weights(const float *W, int N, int K, uint8_t *wq, uint16_t *scales, uint8_t *zeros,
+                                      void *stream) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  if (!W || !wq || !scales || !zeros || N <= 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(wq)) return SVDQ_ERR_MISALIGNED;
+  return launch_awq_quantize(W, N, K, wq, scales, zeros, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SVDQ_OK
+             : SVDQ_ERR_CUDA;
+}
+
+size_t svdq_awq_packed_weight_bytes(int N, int K) {
+  return (N > 0 && K > 0 && K % 64 == 0) ? awq_packed_weight_bytes(N, K) : 0;
+}
+
+size_t svdq_awq_packed_sz_bytes(int N, int K) { return (N > 0 && K > 0 && K % 64 == 0) ? awq_packed_sz_bytes(N, K) : 0; }
+
+svdq_status svdq_awq_pack_weights(const uint8_t *wq, const uint16_t *scales, const uint8_t *zeros, int N, int K,
+                                  uint8_t *wq_packed, uint8_t *sz_packed, void *stream) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  if (!wq || !scales || !zeros || !wq_packed || !sz_packed || N <= 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(wq_packed) || !aligned16(sz_packed)) return SVDQ_ERR_MISALIGNED;
+  return launch_awq_pack(wq, scales, zeros, N, K, wq_packed, sz_packed, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
+             ? SVDQ_OK
+             : SVDQ_ERR_CUDA;
+}
+
+svdq_status svdq_awq_gemv_w4a16(const uint16_t *X, int M, const uint8_t *wq_packed, const uint8_t *sz_packed,
+                                const float *bias, int N, int K, uint16_t *Y, void *stream) {
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
+  if (!X || !wq_packed || !sz_packed || !Y || N <= 0 || K <= 0 || K % 64 || M <= 0 || M > awq_max_tokens() ||
+      awq_smem_bytes(M, K) > 227u * 1024u)
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(wq_packed) || !aligned16(sz_packed)) return SVDQ_ERR_MISALIGNED;
+  return launch_awq_gemv(X, M, wq_packed, sz_packed, bias, N, K, Y, static_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? SVDQ_OK
+             : SVDQ_ERR_CUDA;
+}
+
 svdq_status svdq_linear_forward(const uint16_t *X, int M, const svdq_layer *layer, uint8_t *xq, uint8_t *xs,
                                 uint16_t *lora_act, uint16_t *Y, void *stream) {
   svdq_status st = svdq_quant_act_lora_down(X, M, layer, xq, xs, lora_act, stream);

@@ -62,6 +62,18 @@ cudaError_t launch_gemm(const GemmLaunch &g);
 cudaError_t launch_qk_norm_rope(uint16_t *Y, int M, int heads, const float *norm_q, const float *norm_k,
                                 const float *rope, float eps, cudaStream_t st);
 
+// awq_w4a16 (awq.cu): int4 weights in groups of 64 with fp16 scales and zero points.
+int awq_max_tokens();
+size_t awq_smem_bytes(int M, int K);
+size_t awq_packed_weight_bytes(int N, int K);
+size_t awq_packed_sz_bytes(int N, int K);
+cudaError_t launch_awq_quantize(const float *W, int N, int K, uint8_t *wq, uint16_t *scales, uint8_t *zeros,
+                                cudaStream_t st);
+cudaError_t launch_awq_pack(const uint8_t *wq, const uint16_t *scales, const uint8_t *zeros, int N, int K, uint8_t *wt,
+                            uint8_t *szt, cudaStream_t st);
+cudaError_t launch_awq_gemv(const uint16_t *X, int M, const uint8_t *wt, const uint8_t *szt, const float *bias, int N,
+                            int K, uint16_t *Y, cudaStream_t st);
+
 // Failure-path self-test (selftest.cu): bounded waits on an mbarrier nobody signals.
 cudaError_t launch_selftest_wait(uint32_t *err, uint64_t limit_ns, cudaStream_t st);
 

@@ -29,7 +29,8 @@ EXPORTED = (
     "svdq_gemm_w4a4_lora_up", "svdq_linear_forward", "svdq_linear_forward_host", "svdq_baseline_lora_down",
     "svdq_baseline_quantize", "svdq_baseline_gemm_w4a4", "svdq_baseline_lora_up", "svdq_last_device_error",
     "svdq_smoothing_factors_noalloc", "svdq_selftest_wait_timeout", "svdq_gemm_w4a4_lora_up_qk_norm_rope",
-    "svdq_qk_norm_rope",
+    "svdq_qk_norm_rope", "svdq_awq_quantize_weights", "svdq_awq_gemv_w4a16", "svdq_awq_pack_weights",
+    "svdq_awq_packed_weight_bytes", "svdq_awq_packed_sz_bytes",
 )
 
 
@@ -84,6 +85,11 @@ def load() -> ctypes.CDLL:
         "svdq_smoothing_factors_noalloc": ([P, P, I, I, P, P, P, P], I),
         "svdq_gemm_w4a4_lora_up_qk_norm_rope": ([P, P, P, I, LP, I, I, P, P, P, F, P, P], I),
         "svdq_qk_norm_rope": ([P, I, I, I, P, P, P, F, P], I),
+        "svdq_awq_quantize_weights": ([P, I, I, P, P, P, P], I),
+        "svdq_awq_gemv_w4a16": ([P, I, P, P, P, I, I, P, P], I),
+        "svdq_awq_pack_weights": ([P, P, P, I, I, P, P, P], I),
+        "svdq_awq_packed_weight_bytes": ([I, I], S),
+        "svdq_awq_packed_sz_bytes": ([I, I], S),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -266,6 +272,51 @@ def qk_norm_rope(Y, heads: int, norm_q, norm_k, rope, eps: float = 1e-6, stream=
     """Unfused step: normalizes and rotates the Q and K sections of a bf16 Y in place."""
     _check("svdq_qk_norm_rope", load().svdq_qk_norm_rope(
         _ptr(Y), Y.shape[0], heads, head_dim, _ptr(norm_q), _ptr(norm_k), _ptr(rope), float(eps), _stream(stream)))
+    return Y
+
+
+def awq_quantize_weights(W: torch.Tensor, stream=None):
+    """int4 codes (N x K/2 uint8), fp16 scales (N x K/64), zero points (N x K/64 uint8) of W (fp32)."""
+    N, K = W.shape
+    wq = torch.empty(N, K // 2, dtype=torch.uint8, device=W.device)
+    scales = torch.empty(N, K // 64, dtype=torch.float16, device=W.device)
+    zeros = torch.empty(N, K // 64, dtype=torch.uint8, device=W.device)
+    _check("svdq_awq_quantize_weights", load().svdq_awq_quantize_weights(
+        _ptr(W), N, K, _ptr(wq), _ptr(scales), _ptr(zeros), _stream(stream)))
+    return wq, scales, zeros
+
+
+def awq_pack_weights(wq, scales, zeros, stream=None):
+    """The GEMV's tile layout of quantized weights: (wq_packed, sz_packed) uint8 device buffers."""
+    N, K = wq.shape[0], 2 * wq.shape[1]
+    lib = load()
+    wt = torch.empty(lib.svdq_awq_packed_weight_bytes(N, K), dtype=torch.uint8, device=wq.device)
+    szt = torch.empty(lib.svdq_awq_packed_sz_bytes(N, K), dtype=torch.uint8, device=wq.device)
+    _check("svdq_awq_pack_weights", lib.svdq_awq_pack_weights(
+        _ptr(wq), _ptr(scales), _ptr(zeros), N, K, _ptr(wt), _ptr(szt), _stream(stream)))
+    return wt, szt
+
+
+class AwqLinear:
+    """A packed awq_w4a16 weight (N x K) with its bias, ready for awq_gemv_w4a16."""
+
+    def __init__(self, wq, scales, zeros, bias=None, stream=None):
+        self.N, self.K = wq.shape[0], 2 * wq.shape[1]
+        self.wt, self.szt = awq_pack_weights(wq, scales, zeros, stream)
+        self.bias = bias
+
+    @classmethod
+    def from_float(cls, W: torch.Tensor, bias=None, stream=None):
+        return cls(*awq_quantize_weights(W, stream), bias=bias, stream=stream)
+
+
+def awq_gemv_w4a16(X: torch.Tensor, lin: "AwqLinear", Y=None, stream=None):
+    """Y = bf16(X W_hat^T + bias) for a bf16 X of 1..8 rows."""
+    M, K = X.shape
+    if Y is None:
+        Y = torch.empty(M, lin.N, dtype=torch.bfloat16, device=X.device)
+    _check("svdq_awq_gemv_w4a16", load().svdq_awq_gemv_w4a16(
+        _ptr(X), M, _ptr(lin.wt), _ptr(lin.szt), _ptr(lin.bias), lin.N, K, _ptr(Y), _stream(stream)))
     return Y
 
 

@@ -200,6 +200,40 @@ SVDQ_API svdq_status svdq_gemm_w4a4_lora_up_qk_norm_rope(const uint8_t *xq, cons
 SVDQ_API svdq_status svdq_qk_norm_rope(uint16_t *Y, int M, int heads, int head_dim, const float *norm_q_weight,
                                        const float *norm_k_weight, const float *rope, float eps, void *stream);
 
+/* awq_w4a16 — the second kernel family ("Nunchaku Lite in Diffusers": 4-bit weights with 16-bit
+ * activations for the adaptive-normalization / modulation projections, memory-bound and
+ * precision-sensitive; quantization_config: int4, group_size 64).
+ * Storage: wq N x K/2 bytes (element 2i of a row in the low nibble of byte i), scales N x K/64
+ * fp16, zeros N x K/64 bytes; W_hat[n, k] = (q[n, k] - z[n, k/64]) * s[n, k/64]. K % 64 == 0.
+ *
+ * svdq_awq_quantize_weights: round-to-nearest per group of 64, decided in fp32:
+ *   range = max - min (at least 1e-5), s = fp16(range / 15), z = clamp(rint(-min / s), 0, 15),
+ *   q = clamp(rint(w / s) + z, 0, 15)  (rint: ties to even; divisions correctly rounded).
+ *   W device N x K fp32 (16-byte aligned), |W| below ~4.9e5 (fp16 scale range).
+ *   wq, scales, zeros device outputs (wq 16-byte aligned). Asynchronous on stream.
+ *
+ * svdq_awq_pack_weights: rearranges wq, scales and zeros (as above) into the layout the GEMV
+ *   streams: per 16 rows x 64 columns a 512-byte tile of codes in tensor-core operand order and
+ *   64 bytes of scales and zero points (rows padded to a multiple of 16 with zeros).
+ *   wq_packed  device, svdq_awq_packed_weight_bytes(N, K) bytes, 16-byte aligned.
+ *   sz_packed  device, svdq_awq_packed_sz_bytes(N, K) bytes, 16-byte aligned.
+ *   Done once per layer. Asynchronous on stream.
+ *
+ * svdq_awq_gemv_w4a16: Y[m, n] = bf16(sum_k X[m, k] W_hat[n, k] + bias[n]) for 1 <= M <= 8 tokens;
+ *   the tensor cores sum exact products (128 + q) x in fp32 per group of 64, and the scale and
+ *   zero point are applied per group in fp32: s (D - (128 + z) sum x). X device M x K bf16 (16-byte aligned); wq_packed, sz_packed from
+ *   svdq_awq_pack_weights; bias device N fp32 or NULL; Y device M x N bf16. K <= 13568 (the
+ *   staged activations take K/64 KiB of shared memory); otherwise SVDQ_ERR_INVALID_ARG.
+ *   Asynchronous on stream. */
+SVDQ_API svdq_status svdq_awq_quantize_weights(const float *W, int N, int K, uint8_t *wq, uint16_t *scales,
+                                               uint8_t *zeros, void *stream);
+SVDQ_API size_t svdq_awq_packed_weight_bytes(int N, int K);
+SVDQ_API size_t svdq_awq_packed_sz_bytes(int N, int K);
+SVDQ_API svdq_status svdq_awq_pack_weights(const uint8_t *wq, const uint16_t *scales, const uint8_t *zeros, int N,
+                                           int K, uint8_t *wq_packed, uint8_t *sz_packed, void *stream);
+SVDQ_API svdq_status svdq_awq_gemv_w4a16(const uint16_t *X, int M, const uint8_t *wq_packed, const uint8_t *sz_packed,
+                                         const float *bias, int N, int K, uint16_t *Y, void *stream);
+
 /* K1 then K2 on the same stream (the layer's forward pass). Buffers as above. */
 SVDQ_API svdq_status svdq_linear_forward(const uint16_t *X, int M, const svdq_layer *layer,
                                 uint8_t *xq, uint8_t *xs, uint16_t *lora_act,
