@@ -103,8 +103,10 @@ def _oracle_linear(lib, M, N, K, seed, with_bias=True):
     return Xb, lin, Y_ref
 
 
+# K = 128 and 256 give 2 and 4 groups per row, so 2 and 4 warps share a row block (the other
+# shapes use 1 or 8)
 @pytest.mark.parametrize("M,N,K", [(1, 18432, 3072), (2, 9216, 3072), (3, 333, 576), (5, 64, 1024), (8, 130, 6144),
-                                   (1, 1, 64), (7, 4100, 12288)])
+                                   (1, 1, 64), (7, 4100, 12288), (1, 1000, 128), (2, 1000, 256)])
 def test_gemv_matches_oracle(lib, M, N, K):
     Xb, lin, Y_ref = _oracle_linear(lib, M, N, K, seed=M, with_bias=M != 5)
     Y = lib.awq_gemv_w4a16(x_to_device(Xb), lin)
