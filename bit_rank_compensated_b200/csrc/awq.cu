@@ -8,18 +8,15 @@
 //   scales  N x K/64 fp16;   zeros  N x K/64 bytes (0 .. 15);
 //   W_hat[n, k] = (q[n, k] - z[n, k / 64]) * s[n, k / 64].
 //
-// The product is a GEMV for the few tokens a modulation layer sees (M <= 8): bound by reading
-// the 4-bit weights once, so the kernel streams them with 16-byte loads (a warp reads 512
-// contiguous bytes of a row per load) and keeps the per-weight arithmetic to about two
-// instructions:
-//   * a code becomes an fp32 value without a conversion instruction: OR-ing its nibble, left in
-//     place at bit 4j of a 16-bit half word, into the bit pattern of 2^23 gives 2^23 + q 16^j,
-//     and one packed subtraction of 2^23 leaves q 16^j exactly. The activations are stored in
-//     shared memory pre-scaled by 16^-j (exact), so q 16^j x 16^-j = q x;
-//   * the zero point and the scale are applied once per 32 codes:
-//     sum_k (q_k - z) s x_k = s (sum_k q_k x_k - z sum_k x_k), with the 32-element sums of x
-//     computed once per block;
-//   * products and sums are fp32 (packed f32x2), the output is rounded to bf16 once.
+// The product is a GEMV for the few tokens a modulation layer sees (M <= 8), bound by reading the
+// 4-bit weights once. The GEMV streams them from a tile layout (svdq_awq_pack_weights, once per
+// layer) in which a lane's 16 bytes are its operand-A registers of an m16n8k16 bf16 tensor-core
+// MMA for four k-steps, so each 512-byte tile feeds four warp-wide MMAs after one LOP3 per pair of
+// codes (the nibble ORed into the bit pattern of 128.0 gives the exact bf16 integer 128 + q). The
+// tokens are operand B (staged once per block in fragment order); the products (128 + q) x are
+// exact and summed in fp32, and the scale and zero point enter once per group of 64:
+//   sum_k (q_k - z) s x_k = s (sum_k (128 + q_k) x_k - (128 + z) sum_k x_k).
+// The output is rounded to bf16 once.
 #include "common.cuh"
 #include "internal.h"
 
