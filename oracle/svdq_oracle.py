@@ -424,3 +424,31 @@ def awq_linear(Xv, q, s, z, bias=None, group: int = AWQ_GROUP):
     """Y = X W_hat^T + b in fp64 (W_hat the dequantized int4 weight)."""
     Y = np.asarray(Xv, dtype=np.float64) @ awq_dequantize(q, s, z, group).T
     return Y if bias is None else Y + np.asarray(bias, dtype=np.float64)[None, :]
+
+
+# --------------------------------------------------------------------------- MLP pair
+# "Nunchaku Lite in Diffusers" lists fused GELU / MLP kernels among the engine's fusions; FLUX's
+# feed-forward is Linear(3072 -> 12288), GELU (tanh form), Linear(12288 -> 3072), both linears
+# SVDQuant layers. Reading: in the fused pair the intermediate H = GELU(Y1) reaches the second
+# layer's quantizer and low-rank branch without a 16-bit rounding (it stays on chip); in the
+# unfused pair H is written to memory between the layers, as bf16. The second layer is calibrated
+# on H (its smoothing factors come from max |H_j|). The down layer's activation codes are decided
+# by floating point (the GELU), so a fused kernel's parity is judged at the pair's output.
+def gelu_tanh(x):
+    """0.5 x (1 + tanh(sqrt(2 / pi) (x + 0.044715 x^3))), fp64."""
+    x = np.asarray(x, dtype=np.float64)
+    return 0.5 * x * (1.0 + np.tanh(np.sqrt(2.0 / np.pi) * (x + 0.044715 * x ** 3)))
+
+
+def mlp_hidden(Xv, up: Layer, fused: bool = True):
+    """H = GELU(first layer's output), rounded to bf16 when the pair is not fused."""
+    codes, scales, La = quant_act_lora_down(Xv, up)
+    H = gelu_tanh(gemm_w4a4_lora_up(codes, scales, La, up))
+    return H if fused else bf16_round(H)
+
+
+def mlp_pair(Xv, up: Layer, down: Layer, fused: bool = True):
+    """Z = down(GELU(up(X))) with both linears the SVDQuant layer, fp64."""
+    H = mlp_hidden(Xv, up, fused)
+    codes, scales, La = quant_act_lora_down(H, down)
+    return gemm_w4a4_lora_up(codes, scales, La, down)
