@@ -58,3 +58,34 @@ def test_binding_fails_loudly_without_library(tmp_path, monkeypatch):
     monkeypatch.setattr(svdq, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(RuntimeError, match="missing"):
         svdq.load()
+
+
+def _declared_params():
+    """{name: [parameter declarations]} parsed from include/svdq.h."""
+    src = open(os.path.join(ROOT, "include", "svdq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    out = {}
+    for m in re.finditer(r"SVDQ_API\s+[^;(]*?\b(svdq_\w+)\s*\(([^)]*)\)\s*;", src, flags=re.S):
+        params = [p.strip() for p in m.group(2).split(",") if p.strip()]
+        out[m.group(1)] = [] if params == ["void"] else params
+    return out
+
+
+def test_binding_argument_counts_match_the_header(lib):
+    # every declared entry point is bound with as many ctypes arguments as the header has
+    # parameters, and pointer parameters are bound as pointers
+    import ctypes
+
+    decl = _declared_params()
+    assert sorted(decl) == _declared()
+    for name, params in decl.items():
+        f = getattr(lib, name)
+        assert f.argtypes is not None, name
+        assert len(f.argtypes) == len(params), (name, params, f.argtypes)
+        for p, t in zip(params, f.argtypes):
+            if "*" in p:
+                assert t is ctypes.c_void_p or issubclass(t, (ctypes._Pointer, ctypes.c_char_p)), (name, p, t)
+            elif re.match(r"(const\s+)?(int|uint32_t)\b", p):
+                assert t in (ctypes.c_int, ctypes.c_uint32), (name, p, t)
+            elif re.match(r"(const\s+)?float\b", p):
+                assert t is ctypes.c_float, (name, p, t)
