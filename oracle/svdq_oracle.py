@@ -28,6 +28,15 @@ What it computes, in the order the method states it:
    elements along K, and one fp32 tensor scale per tensor.
 4. The layer output Y = Q(X_hat) Q(R)^T + (X L1s) L2 + b.
 
+Beside the layer (each section below states its readings):
+5. The fused QKV projection's output stage: per-head RMS normalization of Q and K and the rotary
+   embedding ("Nunchaku Lite in Diffusers", section on structural rewrites) -- ``qk_norm_rope``.
+6. The awq_w4a16 family: int4 weights in groups of 64 with fp16 scale and zero point times 16-bit
+   activations, for the modulation projections (same page, kernel families and
+   ``quantization_config``) -- ``awq_quantize``, ``awq_linear``.
+7. The FLUX feed-forward pair: SVDQuant linear, GELU (tanh form), SVDQuant linear, with the
+   intermediate kept unrounded when the pair is fused -- ``mlp_pair``.
+
 Every fp32 operation of the method is emulated as "compute in fp64, round once to
 fp32"; for + - * / and sqrt that equals the correctly rounded fp32 result (double
 rounding from 53 to 24 bits is innocuous for these operations).  e4m3 (OCP E4M3FN:
