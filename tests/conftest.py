@@ -9,3 +9,7 @@ if ROOT not in sys.path:
 def pytest_configure(config):
     config.addinivalue_line("markers", "gpu: needs a B200 (sm_100a) GPU and the built CUDA library")
     config.addinivalue_line("markers", "slow: long CPU test")
+    # a planted mistake in the oracle, only when a mutation test asks for one
+    from tests.oracle_mutations import apply_from_env
+
+    apply_from_env()

@@ -348,3 +348,21 @@ def test_tensor_scales_put_the_largest_group_scale_at_e4m3_max():
     _, xs, _ = O.quant_act_lora_down(X, layer)
     assert O.e4m3_decode(xs).max() == 448.0
     assert O.e4m3_decode(layer.w_scales).max() == 448.0
+
+
+def test_smoothed_activations_are_single_fp32_products():
+    # X_hat = fp32(X * inv_lambda): a bf16 input times an fp32 factor, rounded once to fp32
+    # (numpy's float32 multiply is the independent statement); the chosen factors make products
+    # that need more than bf16's 8 significant bits, so a 16-bit rounding of X_hat would show
+    rng = np.random.default_rng(5)
+    K = 64
+    W = rng.normal(0, 0.02, (32, K)).astype(np.float32)
+    layer = O.prepare(W, None, np.abs(rng.normal(size=K)) + 0.5, 0)
+    inv = (1.0 + np.arange(1, K + 1) * 2.0 ** -12).astype(np.float32)
+    layer.inv_lam = inv.astype(np.float64)
+    Xb = f32_to_bf16_bits(rng.normal(size=(3, K)).astype(np.float32))
+    X = bf16_bits_to_f32(Xb)
+    want = (X * inv[None, :]).astype(np.float64)  # float32 x float32 -> float32
+    got = O.smooth_activations(X.astype(np.float64), layer)
+    np.testing.assert_array_equal(got, want)
+    assert np.any(O.bf16_round(want) != want)
