@@ -76,9 +76,60 @@ def _apply(O, name):
             r = np.sqrt(sig)
             return P * r[None, :], sig, Q / r[None, :]  # L1 = P S, L2 = Q^T
         O.svd_split = svd
+    # fused QKV output stage
+    elif name == "rope_turns_backwards":
+        orig = O.rotary_pairs
+        O.rotary_pairs = lambda U, cos, sin: orig(U, cos, -np.asarray(sin))
+    elif name == "rms_without_eps_inside_sqrt":
+        O.rms_norm_heads = lambda Yh, w, eps: np.asarray(Yh, np.float64) / (
+            np.sqrt(np.mean(np.asarray(Yh, np.float64) ** 2, axis=-1, keepdims=True)) + eps) * np.asarray(w, np.float64)
+    elif name == "rope_pairs_split_halves":
+        def rot(U, cos, sin):  # pairs (i, i + D/2) instead of (2i, 2i + 1)
+            U = np.asarray(U, np.float64)
+            h = U.shape[-1] // 2
+            x0, x1 = U[..., :h], U[..., h:]
+            c, sn = np.asarray(cos)[:, None, :], np.asarray(sin)[:, None, :]
+            return np.concatenate([x0 * c - x1 * sn, x1 * c + x0 * sn], axis=-1)
+        O.rotary_pairs = rot
+    # awq_w4a16
+    elif name == "awq_zero_point_added":
+        O.awq_dequantize = lambda q, s, z, group=64: ((q.reshape(q.shape[0], -1, group).astype(np.float64)
+                                                        + z[:, :, None]) * s[:, :, None]).reshape(q.shape)
+    elif name == "awq_scale_not_fp16":
+        O.f16 = lambda x: np.asarray(x, dtype=np.float64)
+    elif name == "awq_ties_away":
+        orig_q = O.awq_quantize
+
+        def aq(W, group=64):
+            saved = np.rint
+            np.rint = lambda x: np.floor(np.asarray(x) + 0.5)
+            try:
+                return orig_q(W, group)
+            finally:
+                np.rint = saved
+        O.awq_quantize = aq
+    # MLP pair
+    elif name == "gelu_erf_form":
+        from math import erf
+        O.gelu_tanh = lambda x: 0.5 * np.asarray(x, np.float64) * (1.0 + np.vectorize(erf)(np.asarray(x, np.float64) / np.sqrt(2.0)))
+    elif name == "mlp_unfused_not_rounded":
+        orig_h = O.mlp_hidden
+        O.mlp_hidden = lambda Xv, up, fused=True: orig_h(Xv, up, True)
     else:
         raise ValueError(name)
 
+
+# mistake -> the pin file that must catch it
+PIN_FILES = {
+    "rope_turns_backwards": "tests/test_oracle_qk_norm_rope.py",
+    "rms_without_eps_inside_sqrt": "tests/test_oracle_qk_norm_rope.py",
+    "rope_pairs_split_halves": "tests/test_oracle_qk_norm_rope.py",
+    "awq_zero_point_added": "tests/test_oracle_awq.py",
+    "awq_scale_not_fp16": "tests/test_oracle_awq.py",
+    "awq_ties_away": "tests/test_oracle_awq.py",
+    "gelu_erf_form": "tests/test_oracle_mlp_pair.py",
+    "mlp_unfused_not_rounded": "tests/test_oracle_mlp_pair.py",
+}
 
 MUTATIONS = ["ties_away_from_zero", "bias_dropped", "branch_sign", "tensor_scale_divisor", "lambda_inverted",
              "no_sign_convention", "e4m3_two_mantissa_bits", "e4m3_max_240", "bf16_smoothed_activations",
