@@ -22,6 +22,11 @@ Metric: layer TFLOPS = (2MNK + 2MNr + 2MKr) / step time, summed over ranks (weak
 every rank runs its own replica on its own batch, no collective on the data path).
 Rank 0 prints one JSON line. ``--impl reference`` times the fp64 CPU oracle instead (the
 only reference implementation of this method available here) on a bounded row sample.
+
+``--suite`` also covers the fused QKV layer with the Q/K normalization + rotary output stage
+(``qkv_qknorm_rope``: against the plain K2 and against plain K2 + the separate step) and the
+awq_w4a16 GEMV on FLUX's double-block modulation shape (``awq_mod``, ``awq_mod_m2``: 1 and 2
+tokens, against the HBM roof).
 """
 from __future__ import annotations
 
