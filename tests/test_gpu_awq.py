@@ -11,6 +11,7 @@ import pytest
 
 from oracle import svdq_oracle as O
 from synth import bf16_bits_to_f32, make_modulation_inputs
+from tests.awq_layout import tile_layout
 from tests.gpu_helpers import Y_TOL, bf16_tensor_to_np, rel_err_floor, x_to_device
 
 pytestmark = pytest.mark.gpu
@@ -50,38 +51,6 @@ def test_quantizer_bit_exact(lib, N, K):
     np.testing.assert_array_equal(zp.cpu().numpy(), z)
 
 
-def _tile_layout(q, s, z):
-    """The GEMV's tile layout written out from its definition (rows padded to 16): word st of
-    lane L = 4 g + t of tile (rb, G), nibble j = 4 h + i, holds
-    q[16 rb + g + 8 (i & 1)][64 G + 16 st + 2 t + 8 (i >> 1) + h]; the tile's 64 side bytes hold,
-    for each g, {s[row g], s[row g + 8]} as fp16, {z[row g], z[row g + 8]}, two zero bytes."""
-    N, K = q.shape
-    Np = (N + 15) // 16 * 16
-    qp = np.zeros((Np, K), np.uint32)
-    qp[:N] = q
-    sp = np.zeros((Np, K // 64), np.float16)
-    sp[:N] = s.astype(np.float16)
-    zp = np.zeros((Np, K // 64), np.uint8)
-    zp[:N] = z
-    wt = np.zeros((Np // 16, K // 64, 32, 4), np.uint32)
-    szt = np.zeros((Np // 16, K // 64, 8, 8), np.uint8)
-    for L in range(32):
-        g, t = L // 4, L % 4
-        for st in range(4):
-            for j in range(8):
-                i, h = j % 4, j // 4
-                rows = np.arange(Np // 16)[:, None] * 16 + g + 8 * (i & 1)
-                ks = np.arange(K // 64)[None, :] * 64 + 16 * st + 2 * t + 8 * (i >> 1) + h
-                wt[:, :, L, st] |= qp[rows, ks] << (4 * j)
-    for g in range(8):
-        r0 = np.arange(Np // 16) * 16 + g
-        szt[:, :, g, 0:2] = sp[r0].view(np.uint8).reshape(Np // 16, K // 64, 2)
-        szt[:, :, g, 2:4] = sp[r0 + 8].view(np.uint8).reshape(Np // 16, K // 64, 2)
-        szt[:, :, g, 4] = zp[r0]
-        szt[:, :, g, 5] = zp[r0 + 8]
-    return wt.reshape(-1).view(np.uint8), szt.reshape(-1)
-
-
 @pytest.mark.parametrize("N,K", [(37, 128), (300, 640)])
 def test_pack_layout(lib, N, K):
     _, W, _ = make_modulation_inputs(1, K, N, seed=N + 1)
@@ -89,7 +58,7 @@ def test_pack_layout(lib, N, K):
     wt, szt = lib.awq_pack_weights(torch.from_numpy(O.pack_codes(q)).cuda(),
                                    torch.from_numpy(s.astype(np.float16)).cuda(), torch.from_numpy(z).cuda())
     torch.cuda.synchronize()
-    want_wt, want_sz = _tile_layout(q, s, z)
+    want_wt, want_sz = tile_layout(q, s, z)
     np.testing.assert_array_equal(wt.cpu().numpy(), want_wt)
     np.testing.assert_array_equal(szt.cpu().numpy(), want_sz)
 

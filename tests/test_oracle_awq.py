@@ -103,3 +103,4 @@ def test_pins_catch_planted_mistakes():
         assert not np.array_equal(bad, W.astype(np.float64))
     assert np.array_equal(good, W.astype(np.float64))
     assert bad2.shape == good.shape
+
