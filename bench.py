@@ -48,6 +48,10 @@ from synth import CONFIGS, make_inputs  # noqa: E402
 
 METRIC = "W4A4+LoRA linear TFLOPS & fraction of B200 FP4 peak; quant-pass HBM GB/s"
 FP4_OVER_BF16 = 9.0 / 2.25  # nominal dense NVFP4 / BF16 tensor throughput ratio on B200
+# Measured on this GPU model with a kind::mxf4nvf4 MMA-only microbenchmark (no operand loads, all
+# SMs): 128 cycles per one-CTA M128 N256 K64 MMA, i.e. 148 x 2 x 128 x 256 x 64 / 128 flops per
+# cycle at 1965 MHz.
+MMA_ONLY_FP4_TFLOPS = 148 * 2 * 128 * 256 * 64 / 128 * 1965e6 / 1e12
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -81,13 +85,20 @@ def k2_flops(M, K, N, r):
     return 2.0 * M * N * K + 2.0 * M * N * r
 
 
-def k2_traffic(workload: str):
-    """DRAM bytes per K2 launch from the committed ncu capture, if it was taken on this exact
-    K2 source (the file records the sha1 of gemm.cu) and workload; otherwise None."""
+def k2_bytes(M, K, N, r):
+    """Algorithmic HBM bytes of K2: codes and scales of X and of R, the hi/lo down-projection,
+    L2, bias, the bf16 output."""
+    return M * K / 2 + M * K / 16 + N * K / 2 + N * K / 16 + 4.0 * M * r + 2.0 * r * N + 4.0 * N + 2.0 * M * N
+
+
+def kernel_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` ("k1" or "k2") from the committed ncu capture of
+    consecutive launches (profiles/<kernel>_traffic.json), if it was taken on the current source
+    of that kernel (the file records its sha1) and this workload; otherwise None."""
     import hashlib
 
-    tr_path = os.path.join(ROOT, "profiles", "k2_traffic.json")
-    src = os.path.join(ROOT, "bit_rank_compensated_b200", "csrc", "gemm.cu")
+    tr_path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.json")
+    src = os.path.join(ROOT, "bit_rank_compensated_b200", "csrc", {"k1": "quant_act.cu", "k2": "gemm.cu"}[kernel])
     if not (os.path.exists(tr_path) and os.path.exists(src)):
         return None
     with open(tr_path) as f:
@@ -109,16 +120,18 @@ def read_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi clock / throttle sampling while the timed region runs."""
+    """nvidia-smi clock / throttle sampling (every 100 ms) around the timed work. mark_start() /
+    mark_end() bracket the loaded period; the summary covers the samples taken inside it."""
 
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
-         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-         "clocks_event_reasons.sw_power_cap")
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
         self.lines = []
+        self.t0 = self.t1 = None
 
     def __enter__(self):
         try:
@@ -130,6 +143,12 @@ class ClockSampler:
             self.proc = None
         return self
 
+    def mark_start(self):
+        self.t0 = time.time()
+
+    def mark_end(self):
+        self.t1 = time.time()
+
     def __exit__(self, *a):
         if self.proc is not None:
             time.sleep(0.2)
@@ -137,54 +156,88 @@ class ClockSampler:
             out, _ = self.proc.communicate(timeout=10)
             self.lines = [l for l in out.splitlines() if l.strip()]
 
+    @staticmethod
+    def _epoch(ts: str):
+        try:
+            return datetime.datetime.strptime(ts.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+        except ValueError:
+            return None
+
     def summary(self):
-        sm, mx, reasons = [], None, set()
+        sm, mx, reasons, n_all = [], None, set(), 0
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for l in self.lines:
             f = [x.strip() for x in l.split(",")]
-            if len(f) < 9:
+            if len(f) < 10:
+                continue
+            n_all += 1
+            t = self._epoch(f[0])
+            if self.t0 is not None and (t is None or t < self.t0 or t > self.t1):
                 continue
             try:
-                sm.append(float(f[1]))
-                mx = float(f[2])
+                sm.append(float(f[2]))
+                mx = float(f[3])
             except ValueError:
                 continue
-            for n, v in zip(names, f[5:9]):
+            for n, v in zip(names, f[6:10]):
                 if v.lower() == "active":
                     reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+        out = {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+               "samples": len(sm), "samples_total": n_all}
+        if self.t0 is not None:
+            out["window_s"] = round(self.t1 - self.t0, 3)
+        return out
 
 
-def cpu_oracle_sample(shape, rows: int, seed: int = 0, budget_s: float = 20.0):
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_oracle_sample(shape, rows: int, seed: int = 0, budget_s: float = 20.0, threads: int | None = None,
+                      layer=None, X=None):
     """Times the fp64 oracle's forward pass (quantize + down-projection + dequantized GEMM +
-    up-projection) on `rows` tokens of the workload; the SVD prepare is timed apart."""
+    up-projection) on `rows`-token slices of the workload for about budget_s seconds; the SVD
+    prepare is timed apart. threads: BLAS thread limit (None: numpy's default pool)."""
     from oracle import svdq_oracle as O
     from synth import bf16_bits_to_f32
 
-    Xb, W, b, _ = make_inputs(shape, seed=seed)
-    X = bf16_bits_to_f32(Xb).astype(np.float64)
-    t0 = time.perf_counter()
-    layer = O.prepare(W, b, O.calibration_absmax(X), shape.rank)
-    t_prep = time.perf_counter() - t0
-    done, t_fwd, reps = 0, 0.0, 0
-    while t_fwd < budget_s and reps < 64:
-        sl = X[(reps * rows) % shape.M:(reps * rows) % shape.M + rows]
+    t_prep = 0.0
+    if layer is None:
+        Xb, W, b, _ = make_inputs(shape, seed=seed)
+        X = bf16_bits_to_f32(Xb).astype(np.float64)
         t0 = time.perf_counter()
-        O.layer_forward(sl, layer)
-        t_fwd += time.perf_counter() - t0
-        done += sl.shape[0]
-        reps += 1
+        layer = O.prepare(W, b, O.calibration_absmax(X), shape.rank)
+        t_prep = time.perf_counter() - t0
     try:
-        from threadpoolctl import threadpool_info
+        from threadpoolctl import threadpool_info, threadpool_limits
+    except Exception:  # pragma: no cover - threadpoolctl is in the image
+        threadpool_info = threadpool_limits = None
+    import contextlib
 
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    except Exception:
-        threads = os.cpu_count()
+    ctx = threadpool_limits(threads) if (threads and threadpool_limits) else contextlib.nullcontext()
+    with ctx:
+        done, t_fwd, reps = 0, 0.0, 0
+        while t_fwd < budget_s and reps < 64:
+            sl = X[(reps * rows) % shape.M:(reps * rows) % shape.M + rows]
+            t0 = time.perf_counter()
+            O.layer_forward(sl, layer)
+            t_fwd += time.perf_counter() - t0
+            done += sl.shape[0]
+            reps += 1
+        if threadpool_info is not None:
+            used = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        else:
+            used = os.cpu_count()
     flops = layer_flops(done, shape.K, shape.N, shape.rank)
-    return {"value": flops / t_fwd / 1e12, "seconds": t_fwd, "tokens": done, "cores": threads,
-            "prepare_s": t_prep, "reps": reps}
+    return {"value": flops / t_fwd / 1e12, "seconds": t_fwd, "tokens": done, "cores": used,
+            "prepare_s": t_prep, "reps": reps, "layer": layer, "X": X}
 
 
 def run_reference(args, shape, rank, world):
@@ -193,6 +246,7 @@ def run_reference(args, shape, rank, world):
     rows = 256
     res = cpu_oracle_sample(shape, rows, budget_s=max(5.0, min(60.0, 2.0 * args.steps)))
     ms = res["seconds"] / res["reps"] * 1e3
+    res1 = cpu_oracle_sample(shape, 64, budget_s=8.0, threads=1, layer=res["layer"], X=res["X"])
     line = {
         "impl": "reference", "metric": METRIC, "value": res["value"], "unit": "TFLOPS", "n_gpus": args.gpus,
         "steps": res["reps"], "warmup": 0, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -200,7 +254,10 @@ def run_reference(args, shape, rank, world):
         "config": {"workload": workload_name(shape), "M": shape.M, "K": shape.K, "N": shape.N, "rank": shape.rank},
         "cpu_baseline": {"value": res["value"], "unit": "TFLOPS", "cores": res["cores"], "kind": "oracle",
                          "sample": f"{res['reps']} slices of {rows} tokens ({res['tokens']} tokens) of the workload; "
-                                   f"fp64 numpy oracle forward pass, prepare (SVD) excluded ({res['prepare_s']:.1f} s)"},
+                                   f"fp64 numpy oracle forward pass, prepare (SVD) excluded ({res['prepare_s']:.1f} s)",
+                         "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+                         "single_thread": {"value": res1["value"], "unit": "TFLOPS",
+                                           "sample": f"{res1['reps']} slices of 64 tokens, 1 BLAS thread"}},
         "e2e": {"value": res["value"], "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -243,6 +300,35 @@ def time_graphs(stream, graphs):
     return [evs[k].elapsed_time(evs[k + 1]) for k in range(len(graphs))]
 
 
+def time_graphs_rep(stream, graphs, reps):
+    """time_graphs repeated `reps` times (the graphs interleaved); per graph the list of times."""
+    out = [[] for _ in graphs]
+    for _ in range(reps):
+        for lst, t in zip(out, time_graphs(stream, graphs)):
+            lst.append(t)
+    return out
+
+
+def med_best(ms_list, per):
+    """(median, best) of a list of graph times divided by `per` launches each."""
+    v = sorted(x / per for x in ms_list)
+    return statistics.median(v), v[0]
+
+
+def clone_layer(src, dev):
+    """A second copy of a prepared layer's device buffers (so rotating steps do not share weights
+    that would then stay in L2)."""
+    from bit_rank_compensated_b200 import svdq
+
+    L = svdq.Layer(src.N, src.K, src.rank, device=dev, with_bias=src.bias is not None)
+    for name in ("wq", "ws", "inv_lambda", "lam", "L1t", "L2t", "bias"):
+        t = getattr(src, name)
+        if t is not None:
+            getattr(L, name).copy_(t)
+    L.s.w_tensor_scale, L.s.x_tensor_scale = src.s.w_tensor_scale, src.s.x_tensor_scale
+    return L
+
+
 AWQ_WORKLOADS = {"awq_mod": (1, 3072, 18432), "awq_mod_m2": (2, 3072, 18432)}
 
 
@@ -274,10 +360,12 @@ def time_awq(M, K, N, steps, warmup, dev, stream, nb=5):
     g = capture_sequence(steps, launch)
     g.replay()
     torch.cuda.synchronize()
-    (total,) = time_graphs(stream, [g])
+    (tot,) = time_graphs_rep(stream, [g], REPS)
     assert svdq.last_device_error() == 0
-    return total / steps
+    return med_best(tot, steps)[0]
 
+
+REPS = 7  # timed replays of each graph; medians are reported
 
 SUITE = ["qkv", "qkv_qknorm_rope", "awq_mod", "awq_mod_m2", "mlp_up", "mlp_down", "sweep_m256", "sweep_m1024", "sweep_m4096", "sweep_m16384",
          "sweep_r0", "sweep_r16", "sweep_r32", "sweep_r64", "sweep_r128"]
@@ -304,9 +392,10 @@ def time_layer(shape, steps, warmup, dev, stream, unfused=False, nb=3, stage="pl
     Xb, W, b, _ = make_inputs(shape, seed=0)
     X0 = torch.from_numpy(Xb.view(np.int16)).to(dev).view(torch.bfloat16)
     ax = svdq.act_absmax(X0)
-    L = svdq.prepare_weights(torch.from_numpy(W).to(dev), torch.from_numpy(b).to(dev), ax, r)
+    L0 = svdq.prepare_weights(torch.from_numpy(W).to(dev), torch.from_numpy(b).to(dev), ax, r)
+    Ls = [L0] + [clone_layer(L0, dev) for _ in range(nb - 1)]
     Xs = [X0] + [X0.clone() for _ in range(nb - 1)]
-    bufs = [svdq.alloc_activations(M, L, dev) for _ in range(nb)]
+    bufs = [svdq.alloc_activations(M, L0, dev) for _ in range(nb)]
     Ys = [torch.empty(M, N, dtype=torch.bfloat16, device=dev) for _ in range(nb)]
     heads = N // (3 * HEAD_DIM)
     if stage != "plain":
@@ -315,6 +404,7 @@ def time_layer(shape, steps, warmup, dev, stream, unfused=False, nb=3, stage="pl
 
     def k2_part(j):
         xq, xs, la = bufs[j]
+        L = Ls[j]
         if stage == "qknr":
             return lambda st: svdq.gemm_w4a4_lora_up_qk_norm_rope(xq, xs, la, M, L, heads, wq, wk, ropes[j], 1e-6,
                                                                   Ys[j], st)
@@ -328,6 +418,7 @@ def time_layer(shape, steps, warmup, dev, stream, unfused=False, nb=3, stage="pl
     def step_on(j):
         # part 0: K1 (or the whole unfused path), part 1: K2 (None when unfused)
         xq, xs, la = bufs[j]
+        L = Ls[j]
         if unfused:
             return (lambda st: svdq.unfused_forward(Xs[j], L, bufs[j], Ys[j], st)), None
         return (lambda st: svdq.quant_act_lora_down(Xs[j], L, xq, xs, la, st)), k2_part(j)
@@ -344,17 +435,17 @@ def time_layer(shape, steps, warmup, dev, stream, unfused=False, nb=3, stage="pl
     g_steps = capture_sequence(steps, lambda i: step_on(i % nb))
     if unfused:
         g_steps.replay()
-        (total,) = time_graphs(stream, [g_steps])
+        (tot,) = time_graphs_rep(stream, [g_steps], REPS)
         assert svdq.last_device_error() == 0
-        return total / steps, None, None
+        return med_best(tot, steps)[0], None, None
     g_k1 = capture_sequence(steps, lambda i: step_on(i % nb)[:1])
     g_k2 = capture_sequence(steps, lambda i: step_on(i % nb)[1:])
     for g in (g_steps, g_k1, g_k2):  # warm replay
         g.replay()
     torch.cuda.synchronize()
-    total, k1, k2 = time_graphs(stream, [g_steps, g_k1, g_k2])
+    tot, k1, k2 = time_graphs_rep(stream, [g_steps, g_k1, g_k2], REPS)
     assert svdq.last_device_error() == 0
-    return total / steps, k1 / steps, k2 / steps
+    return med_best(tot, steps)[0], med_best(k1, steps)[0], med_best(k2, steps)[0]
 
 
 def run_suite(args):
@@ -431,6 +522,36 @@ def run_suite(args):
     return 0
 
 
+def run_ncu_target(args, shape):
+    """Launch list for ncu: prepare the workload, then `steps` back-to-back plain launches of one
+    kernel (k1, or k2 after one K1), without graphs, so that a capture of consecutive launches
+    (e.g. -k regex:k2_gemm -c 3 --cache-control none) counts the output each launch leaves in L2
+    against the next one. Prints one line; no timing."""
+    import torch
+    from bit_rank_compensated_b200 import svdq
+
+    svdq.load()
+    dev = torch.device("cuda", 0)
+    M, K, N, r = shape.M, shape.K, shape.N, shape.rank
+    Xb, W, b, _ = make_inputs(shape, seed=0)
+    X = torch.from_numpy(Xb.view(np.int16)).to(dev).view(torch.bfloat16)
+    L = svdq.prepare_weights(torch.from_numpy(W).to(dev), torch.from_numpy(b).to(dev), svdq.act_absmax(X), r)
+    xq, xs, la = svdq.alloc_activations(M, L, dev)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream()
+    if args.ncu_kernel == "k2":
+        svdq.quant_act_lora_down(X, L, xq, xs, la, stream)
+    for _ in range(args.steps):
+        if args.ncu_kernel == "k1":
+            svdq.quant_act_lora_down(X, L, xq, xs, la, stream)
+        else:
+            svdq.gemm_w4a4_lora_up(xq, xs, la, M, L, Y, stream)
+    torch.cuda.synchronize()
+    assert svdq.last_device_error() == 0
+    print(json.dumps({"ncu_target": args.ncu_kernel, "workload": shape.name, "launches": args.steps}), flush=True)
+    return 0
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -440,8 +561,12 @@ def main(argv=None):
     ap.add_argument("--workload", default="qkv", choices=sorted(CONFIGS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--soak-s", type=float, default=1.0,
+                    help="seconds of untimed step replays inside the clock-sampling window before the timed region")
     ap.add_argument("--suite", nargs="?", const=",".join(SUITE), default=None,
                     help="time a comma-separated list of workloads (default: all) and print one line each")
+    ap.add_argument("--ncu-kernel", choices=["k1", "k2"], default=None,
+                    help="only launch one kernel `--steps` times back to back (for an ncu capture)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
     if args.suite:
@@ -454,6 +579,8 @@ def main(argv=None):
 
     if args.impl == "reference":
         return run_reference(args, shape, rank, world)
+    if args.ncu_kernel:
+        return run_ncu_target(args, shape)
 
     import torch
 
@@ -479,14 +606,7 @@ def main(argv=None):
     bd = torch.from_numpy(b).to(dev)
     ax = svdq.act_absmax(Xd0)
     layers = [svdq.prepare_weights(Wd, bd, ax, r)]
-    for _ in range(NB - 1):
-        L = svdq.Layer(N, K, r, device=dev)
-        for name in ("wq", "ws", "inv_lambda", "lam", "L1t", "L2t", "bias"):
-            src = getattr(layers[0], name)
-            if src is not None:
-                getattr(L, name).copy_(src)
-        L.s.w_tensor_scale, L.s.x_tensor_scale = layers[0].s.w_tensor_scale, layers[0].s.x_tensor_scale
-        layers.append(L)
+    layers += [clone_layer(layers[0], dev) for _ in range(NB - 1)]
     del Wd
     Xs = [Xd0] + [Xd0.clone() for _ in range(NB - 1)]
     bufs = [svdq.alloc_activations(M, layers[0], dev) for _ in range(NB)]
@@ -495,32 +615,37 @@ def main(argv=None):
                  + Ys[0].numel() * 2 + layers[0].wq.numel() + layers[0].ws.numel())
     stream = torch.cuda.current_stream()
 
-    def step(i):
-        j = i % NB
-        xq, xs, la = bufs[j]
-        svdq.quant_act_lora_down(Xs[j], layers[j], xq, xs, la, stream)
-        svdq.gemm_w4a4_lora_up(xq, xs, la, M, layers[j], Ys[j], stream)
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    assert svdq.last_device_error() == 0
-
     def parts(j):
         xq, xs, la = bufs[j]
         return ((lambda st: svdq.quant_act_lora_down(Xs[j], layers[j], xq, xs, la, st)),
                 (lambda st: svdq.gemm_w4a4_lora_up(xq, xs, la, M, layers[j], Ys[j], st)))
 
+    for i in range(args.warmup):
+        for fn in parts(i % NB):
+            fn(stream)
+    torch.cuda.synchronize()
+    assert svdq.last_device_error() == 0
+
     g_steps = capture_sequence(args.steps, lambda i: parts(i % NB))
     g_k1 = capture_sequence(args.steps, lambda i: parts(i % NB)[:1])
     g_k2 = capture_sequence(args.steps, lambda i: parts(i % NB)[1:])
-    for g in (g_steps, g_k1, g_k2):  # warm replay
+    # K1 over one buffer set only: X (and L1s) stay in L2 between launches (the unflushed figure)
+    g_k1_warm = capture_sequence(args.steps, lambda i: parts(0)[:1])
+    for g in (g_steps, g_k1, g_k2, g_k1_warm):  # warm replay
         g.replay()
     torch.cuda.synchronize()
 
     gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local]) \
         if os.environ.get("CUDA_VISIBLE_DEVICES") else local
     with ClockSampler(gpu_index) as clk:
+        clk.mark_start()
+        # untimed replays first, so that the clock samples of the window see the GPU under this load
+        t_soak = time.time()
+        n_soak = 0
+        while time.time() - t_soak < args.soak_s:
+            g_steps.replay()
+            torch.cuda.synchronize()
+            n_soak += 1
         if dist:
             dist.barrier()
         torch.cuda.synchronize()
@@ -532,11 +657,13 @@ def main(argv=None):
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
+        # per-kernel durations: K back-to-back launches of each kernel alone, same stream, REPS times
+        k1_runs, k2_runs, k1w_runs = time_graphs_rep(stream, [g_k1, g_k2, g_k1_warm], REPS)
+        clk.mark_end()
     total_ms = t_start.elapsed_time(t_end)
-    # per-kernel durations: K back-to-back launches of each kernel alone, same stream
-    k1_total, k2_total = time_graphs(stream, [g_k1, g_k2])
-    k1_avg = k1_total / args.steps
-    k2_avg = k2_total / args.steps
+    k1_avg, k1_best = med_best(k1_runs, args.steps)
+    k2_avg, k2_best = med_best(k2_runs, args.steps)
+    k1w_avg, k1w_best = med_best(k1w_runs, args.steps)
     err = svdq.last_device_error()
 
     total_ms = max_over_ranks(total_ms, dist, dev)
@@ -572,13 +699,19 @@ def main(argv=None):
     fp4_peak = bf16_tf * FP4_OVER_BF16
     k2_tf = k2_flops(M, K, N, r) / (k2_avg * 1e-3) / 1e12
     k1_gbs = k1_bytes(M, K, r) / (k1_avg * 1e-3) / 1e9
-    traffic = k2_traffic(shape.name)
+    k1w_gbs = k1_bytes(M, K, r) / (k1w_avg * 1e-3) / 1e9
+    tr2 = kernel_traffic("k2", shape.name)
+    tr1 = kernel_traffic("k1", shape.name)
     cpu = None
     if not args.no_cpu_baseline and world == 1:
         res = cpu_oracle_sample(shape, 256, budget_s=15.0)
+        res1 = cpu_oracle_sample(shape, 64, budget_s=8.0, threads=1, layer=res["layer"], X=res["X"])
         cpu = {"value": res["value"], "unit": "TFLOPS", "cores": res["cores"], "kind": "oracle",
                "sample": f"{res['reps']} slices of 256 tokens ({res['tokens']} tokens) of the workload; fp64 numpy "
-                         f"oracle forward pass, prepare (SVD) excluded ({res['prepare_s']:.1f} s)"}
+                         f"oracle forward pass, prepare (SVD) excluded ({res['prepare_s']:.1f} s)",
+               "cpu_model": cpu_model(), "nproc": os.cpu_count(),
+               "single_thread": {"value": res1["value"], "unit": "TFLOPS",
+                                 "sample": f"{res1['reps']} slices of 64 tokens ({res1['tokens']} tokens), 1 BLAS thread"}}
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
@@ -587,13 +720,23 @@ def main(argv=None):
                    "l2": f"{NB} rotating buffer sets of {set_bytes / 1e6:.0f} MB (> 126 MB L2 in total)",
                    "parallelism": f"replicas x{world}"},
         "roofline": {"kernel": "svdq_gemm_w4a4_lora_up (K2)", "bound": "tensor", "achieved": k2_tf,
-                     "peak": fp4_peak, "unit": "TFLOP/s", "frac": k2_tf / fp4_peak, "traffic": traffic,
+                     "peak": fp4_peak, "unit": "TFLOP/s", "frac": k2_tf / fp4_peak, "traffic": tr2,
+                     "traffic_over_algorithmic": (tr2 / k2_bytes(M, K, N, r)) if tr2 else None,
+                     "algorithmic_bytes": k2_bytes(M, K, N, r),
                      "peak_source": f"{peak_kind} bf16 {bf16_tf:.0f} TF/s x {FP4_OVER_BF16:.0f} (nvfp4/bf16 nominal)",
-                     "achieved_basis": "2MNK + 2MNr per launch / CUDA-event duration of K back-to-back launches over K"},
+                     "frac_vs_mma_only": k2_tf / MMA_ONLY_FP4_TFLOPS,
+                     "mma_only_peak": MMA_ONLY_FP4_TFLOPS,
+                     "achieved_basis": f"2MNK + 2MNr per launch / median over {REPS} timings of K back-to-back "
+                                       f"launches (CUDA events) / K"},
         "quant_pass": {"kernel": "svdq_quant_act_lora_down (K1)", "bound": "hbm", "achieved": k1_gbs,
                        "peak": hbm_gbs, "unit": "GB/s", "frac": k1_gbs / hbm_gbs, "us": k1_avg * 1e3,
-                       "frac_of_8TBs_datasheet": k1_gbs / 8000.0},
-        "k2": {"us": k2_avg * 1e3, "tflops": k2_tf},
+                       "us_best": k1_best * 1e3, "frac_of_8TBs_datasheet": k1_gbs / 8000.0,
+                       "traffic": tr1, "traffic_over_algorithmic": (tr1 / k1_bytes(M, K, r)) if tr1 else None,
+                       "l2_warm": {"us": k1w_avg * 1e3, "gbs": k1w_gbs, "frac": k1w_gbs / hbm_gbs,
+                                   "note": "K launches over one buffer set (X stays in L2)"}},
+        "k2": {"us": k2_avg * 1e3, "us_best": k2_best * 1e3, "tflops": k2_tf},
+        "timing": {"reps": REPS, "k1_us": [round(t / args.steps * 1e3, 3) for t in k1_runs],
+                   "k2_us": [round(t / args.steps * 1e3, 3) for t in k2_runs], "soak_replays": n_soak},
         "tokens_per_s": world * M * args.steps / (total_ms * 1e-3),
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": int(M * K * 2),

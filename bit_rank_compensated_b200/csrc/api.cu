@@ -5,8 +5,10 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
+#include "common.cuh"
 #include "internal.h"
 #include "svdq.h"
 
@@ -26,6 +28,10 @@ struct DeviceState {
 };
 DeviceState g_dev[kMaxDevices];
 
+// Compute capability that svdq_test_override_capability asks device_check to assume
+// (major * 10 + minor), or -1. It can only make a supported GPU look unsupported.
+std::atomic<int> g_cap_override{-1};
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
                                    const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -43,6 +49,8 @@ void init_encode() {
 // Checks the current device once: compute capability 10.0 ("دعم الأجهزة": unsupported GPUs
 // get a clear error instead of wrong output) and records the SM count and the error word.
 svdq_status device_check(DeviceState **out) {
+  const int ov = g_cap_override.load(std::memory_order_relaxed);
+  if (ov >= 0 && ov != 100) return SVDQ_ERR_UNSUPPORTED_ARCH;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SVDQ_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return SVDQ_ERR_INTERNAL;
@@ -75,6 +83,11 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 
 bool rank_ok(int r) { return r == 0 || r == 16 || r == 32 || r == 64 || r == 128; }
 
+// Tensor scales the quantizers handle exactly: with s in [2^-116, 2^116] every non-zero group
+// scale times s (at least 2^-9 s) is a normal fp32 number whose reciprocal is finite, and 6 s,
+// 448 s and 1 / (6 s) are finite.
+bool scale_ok(float s) { return s >= 0x1p-116f && s <= 0x1p116f; }
+
 svdq_status check_layer(const svdq_layer *L) {
   if (!L) return SVDQ_ERR_INVALID_ARG;
   if (L->N <= 0 || L->K <= 0 || (L->K % 64) != 0 || (L->N % 16) != 0 || !rank_ok(L->rank))
@@ -84,7 +97,7 @@ svdq_status check_layer(const svdq_layer *L) {
   if (!aligned16(L->wq) || !aligned16(L->ws) || !aligned16(L->inv_lambda) || !aligned16(L->bias) ||
       !aligned16(L->L1t) || !aligned16(L->L2t))
     return SVDQ_ERR_MISALIGNED;
-  if (!(L->x_tensor_scale > 0.0f) || !(L->w_tensor_scale > 0.0f)) return SVDQ_ERR_INVALID_ARG;
+  if (!scale_ok(L->x_tensor_scale) || !scale_ok(L->w_tensor_scale)) return SVDQ_ERR_INVALID_ARG;
   return SVDQ_OK;
 }
 
@@ -108,15 +121,17 @@ float alpha_of(const svdq_layer *L) { return L->x_tensor_scale * L->w_tensor_sca
 
 svdq_status run_quant(const uint16_t *X, int M, const svdq_layer *L, uint8_t *xq, uint8_t *xs, uint16_t *la,
                       bool quantize, bool lora, void *stream) {
-  DeviceState *d = nullptr;
-  svdq_status st = device_check(&d);
-  if (st != SVDQ_OK) return st;
-  st = check_layer(L);
+  // argument checks first: they need no device, so a bad call is reported the same way on any
+  // machine
+  svdq_status st = check_layer(L);
   if (st != SVDQ_OK) return st;
   if (!X || M <= 0) return SVDQ_ERR_INVALID_ARG;
   if (quantize && (!xq || !xs)) return SVDQ_ERR_INVALID_ARG;
   if (lora && L->rank > 0 && !la) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(xq) || !aligned16(xs) || !aligned16(la)) return SVDQ_ERR_MISALIGNED;
+  DeviceState *d = nullptr;
+  st = device_check(&d);
+  if (st != SVDQ_OK) return st;
   if (!quantize && (!lora || L->rank == 0)) return SVDQ_OK;
   QuantLaunch q;
   memset(&q, 0, sizeof(q));
@@ -158,16 +173,16 @@ struct QkNormRope {
 
 svdq_status run_gemm(const uint8_t *xq, const uint8_t *xs, const uint16_t *la, int M, const svdq_layer *L,
                      uint16_t *Y, bool fp4, bool add_y, bool lora, void *stream, const QkNormRope *qk = nullptr) {
-  DeviceState *d = nullptr;
-  svdq_status st = device_check(&d);
-  if (st != SVDQ_OK) return st;
-  st = check_layer(L);
+  svdq_status st = check_layer(L);
   if (st != SVDQ_OK) return st;
   if (M <= 0 || !Y) return SVDQ_ERR_INVALID_ARG;
   if (fp4 && (!xq || !xs)) return SVDQ_ERR_INVALID_ARG;
   const int r = lora ? L->rank : 0;
   if (r > 0 && !la) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(xq) || !aligned16(xs) || !aligned16(la) || !aligned16(Y)) return SVDQ_ERR_MISALIGNED;
+  DeviceState *d = nullptr;
+  st = device_check(&d);
+  if (st != SVDQ_OK) return st;
   if (!fp4 && r == 0) return SVDQ_OK;
   GemmLaunch g;
   memset(&g, 0, sizeof(g));
@@ -259,10 +274,10 @@ size_t svdq_act_scale_bytes(int M, int K) {
 }
 
 svdq_status svdq_act_absmax(const uint16_t *X, int M, int K, float *absmax, void *stream) {
+  if (!X || !absmax || M <= 0 || K <= 0) return SVDQ_ERR_INVALID_ARG;
   DeviceState *d = nullptr;
   svdq_status st = device_check(&d);
   if (st != SVDQ_OK) return st;
-  if (!X || !absmax || M <= 0 || K <= 0) return SVDQ_ERR_INVALID_ARG;
   return launch_col_absmax_bf16(X, M, K, absmax, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SVDQ_OK
                                                                                                    : SVDQ_ERR_CUDA;
 }
@@ -282,9 +297,6 @@ size_t svdq_prepare_workspace_bytes(int N, int K, int rank, svdq_status *status)
 
 svdq_status svdq_prepare_weights(const float *W, const float *bias, const float *act_absmax, int N, int K, int rank,
                                  svdq_layer *layer, void *workspace, size_t workspace_bytes, void *stream) {
-  DeviceState *d = nullptr;
-  svdq_status st = device_check(&d);
-  if (st != SVDQ_OK) return st;
   if (!W || !act_absmax || !layer || !workspace) return SVDQ_ERR_INVALID_ARG;
   if (N <= 0 || K <= 0 || K % 64 || N % 16 || !rank_ok(rank)) return SVDQ_ERR_INVALID_ARG;
   if (layer->N != N || layer->K != K || layer->rank != rank) return SVDQ_ERR_INVALID_ARG;
@@ -294,6 +306,9 @@ svdq_status svdq_prepare_weights(const float *W, const float *bias, const float 
       !aligned16(layer->ws) || !aligned16(layer->inv_lambda) || !aligned16(layer->lambda) ||
       !aligned16(layer->L1t) || !aligned16(layer->L2t) || !aligned16(layer->bias) || !aligned16(bias))
     return SVDQ_ERR_MISALIGNED;
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
   PrepArgs p;
   const PrepStatus ps = prepare_plan(N, K, rank, &p.plan);
   if (ps == PREP_NO_SOLVER) return SVDQ_ERR_UNAVAILABLE;
@@ -331,16 +346,84 @@ svdq_status svdq_prepare_weights(const float *W, const float *bias, const float 
   return SVDQ_OK;
 }
 
-svdq_status svdq_smoothing_factors_noalloc(const float *W, const float *act_absmax, int N, int K, float *lambda,
-                                           float *inv_lambda, float *x_tensor_scale, void *stream) {
+svdq_status svdq_prepare_weights_host(const float *W_host, const float *bias_host, const float *act_absmax_host, int N,
+                                      int K, int rank, svdq_layer *layer, float *R_out_host, void *stream) {
+  if (!W_host || !act_absmax_host || !layer) return SVDQ_ERR_INVALID_ARG;
+  if (N <= 0 || K <= 0 || K % 64 || N % 16 || !rank_ok(rank)) return SVDQ_ERR_INVALID_ARG;
+  if (layer->N != N || layer->K != K || layer->rank != rank) return SVDQ_ERR_INVALID_ARG;
+  if (!layer->wq || !layer->ws || !layer->inv_lambda || (rank > 0 && (!layer->L1t || !layer->L2t)))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(layer->wq) || !aligned16(layer->ws) || !aligned16(layer->inv_lambda) || !aligned16(layer->lambda) ||
+      !aligned16(layer->L1t) || !aligned16(layer->L2t) || !aligned16(layer->bias))
+    return SVDQ_ERR_MISALIGNED;
   DeviceState *d = nullptr;
   svdq_status st = device_check(&d);
   if (st != SVDQ_OK) return st;
+  svdq_status ws_st = SVDQ_OK;
+  const size_t ws_bytes = svdq_prepare_workspace_bytes(N, K, rank, &ws_st);
+  if (ws_st != SVDQ_OK) return ws_st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const size_t wbytes = static_cast<size_t>(N) * K * sizeof(float);
+  // one offline allocation: W, the calibration maxima and the workspace, 256-byte aligned pieces
+  const size_t off_ax = (wbytes + 255) & ~size_t(255);
+  const size_t off_ws = off_ax + ((static_cast<size_t>(K) * sizeof(float) + 255) & ~size_t(255));
+  void *buf = nullptr;
+  if (cudaMalloc(&buf, off_ws + ws_bytes) != cudaSuccess) return SVDQ_ERR_CUDA;
+  uint8_t *base = static_cast<uint8_t *>(buf);
+  st = SVDQ_OK;
+  if (cudaMemcpyAsync(base, W_host, wbytes, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      cudaMemcpyAsync(base + off_ax, act_absmax_host, sizeof(float) * K, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+      (bias_host && layer->bias &&
+       cudaMemcpyAsync(layer->bias, bias_host, sizeof(float) * N, cudaMemcpyHostToDevice, s) != cudaSuccess))
+    st = SVDQ_ERR_CUDA;
+  if (st == SVDQ_OK) {
+    PrepArgs p;
+    const PrepStatus ps = prepare_plan(N, K, rank, &p.plan);
+    if (ps != PREP_OK) st = ps == PREP_NO_SOLVER ? SVDQ_ERR_UNAVAILABLE : SVDQ_ERR_CUDA;
+    if (st == SVDQ_OK) {
+      float s_w = 0.0f, s_x = 0.0f;
+      p.W = reinterpret_cast<const float *>(base);
+      p.act_absmax = reinterpret_cast<const float *>(base + off_ax);
+      p.N = N;
+      p.K = K;
+      p.rank = rank;
+      p.workspace = base + off_ws;
+      p.lambda_out = layer->lambda;
+      p.inv_lambda = layer->inv_lambda;
+      p.L1t = layer->L1t;
+      p.L2t = layer->L2t;
+      p.wq = layer->wq;
+      p.wscales = layer->ws;
+      p.wscale_bytes = svdq_weight_scale_bytes(N, K);
+      p.s_w = &s_w;
+      p.s_x = &s_x;
+      p.R_out_host = R_out_host;
+      p.stream = s;
+      const PrepStatus rs = prepare_run(p);
+      if (rs == PREP_SOLVER_FAILED) st = SVDQ_ERR_INTERNAL;
+      else if (rs != PREP_OK) st = SVDQ_ERR_CUDA;
+      if (st == SVDQ_OK) {
+        layer->group = 16;
+        layer->w_tensor_scale = s_w;
+        layer->x_tensor_scale = s_x;
+      }
+    }
+  }
+  if (cudaStreamSynchronize(s) != cudaSuccess) st = SVDQ_ERR_CUDA;
+  if (cudaFree(buf) != cudaSuccess && st == SVDQ_OK) st = SVDQ_ERR_CUDA;
+  return st;
+}
+
+svdq_status svdq_smoothing_factors_noalloc(const float *W, const float *act_absmax, int N, int K, float *lambda,
+                                           float *inv_lambda, float *x_tensor_scale, void *stream) {
   if (!W || !act_absmax || !lambda || !inv_lambda || !x_tensor_scale || N <= 0 || K <= 0 || K % 64 != 0 ||
       K > noalloc_max_k())
     return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(W) || !aligned16(act_absmax) || !aligned16(lambda) || !aligned16(inv_lambda))
     return SVDQ_ERR_MISALIGNED;
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
   return smoothing_noalloc(W, act_absmax, N, K, lambda, inv_lambda, x_tensor_scale,
                            static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? SVDQ_OK
@@ -349,12 +432,12 @@ svdq_status svdq_smoothing_factors_noalloc(const float *W, const float *act_absm
 
 svdq_status svdq_quantize_rows(const float *A, int rows, int K, float s, int row_pad, uint8_t *codes, uint8_t *scales,
                                void *stream) {
+  if (!A || !codes || !scales || rows <= 0 || K <= 0 || K % 64 || !scale_ok(s) || (row_pad != 128 && row_pad != 256))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(A) || !aligned16(codes) || !aligned16(scales)) return SVDQ_ERR_MISALIGNED;
   DeviceState *d = nullptr;
   svdq_status st = device_check(&d);
   if (st != SVDQ_OK) return st;
-  if (!A || !codes || !scales || rows <= 0 || K <= 0 || K % 64 || !(s > 0.0f) || (row_pad != 128 && row_pad != 256))
-    return SVDQ_ERR_INVALID_ARG;
-  if (!aligned16(A) || !aligned16(codes) || !aligned16(scales)) return SVDQ_ERR_MISALIGNED;
   cudaStream_t cs = static_cast<cudaStream_t>(stream);
   const size_t sbytes = round_up(static_cast<size_t>(rows), row_pad) * (K / 16);
   if (cudaMemsetAsync(scales, 0, sbytes, cs) != cudaSuccess) return SVDQ_ERR_CUDA;
@@ -394,13 +477,13 @@ svdq_status svdq_gemm_w4a4_lora_up_qk_norm_rope(const uint8_t *xq, const uint8_t
 
 svdq_status svdq_qk_norm_rope(uint16_t *Y, int M, int heads, int head_dim, const float *norm_q_weight,
                               const float *norm_k_weight, const float *rope, float eps, void *stream) {
-  DeviceState *d = nullptr;
-  svdq_status st = device_check(&d);
-  if (st != SVDQ_OK) return st;
   if (!Y || M <= 0 || heads <= 0) return SVDQ_ERR_INVALID_ARG;
-  st = check_qk_args(3 * heads * head_dim, heads, head_dim, norm_q_weight, norm_k_weight, rope, eps);
+  svdq_status st = check_qk_args(3 * heads * head_dim, heads, head_dim, norm_q_weight, norm_k_weight, rope, eps);
   if (st != SVDQ_OK) return st;
   if (!aligned16(Y)) return SVDQ_ERR_MISALIGNED;
+  DeviceState *d = nullptr;
+  st = device_check(&d);
+  if (st != SVDQ_OK) return st;
   return launch_qk_norm_rope(Y, M, heads, norm_q_weight, norm_k_weight, rope, eps, static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? SVDQ_OK
@@ -409,11 +492,11 @@ svdq_status svdq_qk_norm_rope(uint16_t *Y, int M, int heads, int head_dim, const
 
 svdq_status svdq_awq_quantize_weights(const float *W, int N, int K, uint8_t *wq, uint16_t *scales, uint8_t *zeros,
                                       void *stream) {
+  if (!W || !wq || !scales || !zeros || N <= 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(W) || !aligned16(wq)) return SVDQ_ERR_MISALIGNED;
   DeviceState *d = nullptr;
   svdq_status st = device_check(&d);
   if (st != SVDQ_OK) return st;
-  if (!W || !wq || !scales || !zeros || N <= 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
-  if (!aligned16(W) || !aligned16(wq)) return SVDQ_ERR_MISALIGNED;
   return launch_awq_quantize(W, N, K, wq, scales, zeros, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? SVDQ_OK
              : SVDQ_ERR_CUDA;
@@ -427,11 +510,11 @@ size_t svdq_awq_packed_sz_bytes(int N, int K) { return (N > 0 && K > 0 && K % 64
 
 svdq_status svdq_awq_pack_weights(const uint8_t *wq, const uint16_t *scales, const uint8_t *zeros, int N, int K,
                                   uint8_t *wq_packed, uint8_t *sz_packed, void *stream) {
+  if (!wq || !scales || !zeros || !wq_packed || !sz_packed || N <= 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(wq_packed) || !aligned16(sz_packed)) return SVDQ_ERR_MISALIGNED;
   DeviceState *d = nullptr;
   svdq_status st = device_check(&d);
   if (st != SVDQ_OK) return st;
-  if (!wq || !scales || !zeros || !wq_packed || !sz_packed || N <= 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
-  if (!aligned16(wq_packed) || !aligned16(sz_packed)) return SVDQ_ERR_MISALIGNED;
   return launch_awq_pack(wq, scales, zeros, N, K, wq_packed, sz_packed, static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? SVDQ_OK
@@ -440,15 +523,15 @@ svdq_status svdq_awq_pack_weights(const uint8_t *wq, const uint16_t *scales, con
 
 svdq_status svdq_awq_gemv_w4a16(const uint16_t *X, int M, const uint8_t *wq_packed, const uint8_t *sz_packed,
                                 const float *bias, int N, int K, uint16_t *Y, void *stream) {
-  DeviceState *d = nullptr;
-  svdq_status st = device_check(&d);
-  if (st != SVDQ_OK) return st;
   if (!X || !wq_packed || !sz_packed || !Y || N <= 0 || K <= 0 || K % 64 || M <= 0 || M > awq_max_tokens() ||
       awq_smem_bytes(M, K) > 227u * 1024u)
     return SVDQ_ERR_INVALID_ARG;
   // the kernel walks the tiles with 32-bit indices (times 32 lanes)
   if (static_cast<uint64_t>((N + 15) / 16) * static_cast<uint64_t>(K / 64) >= (1ull << 26)) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(wq_packed) || !aligned16(sz_packed)) return SVDQ_ERR_MISALIGNED;
+  DeviceState *d = nullptr;
+  svdq_status st = device_check(&d);
+  if (st != SVDQ_OK) return st;
   return launch_awq_gemv(X, M, wq_packed, sz_packed, bias, N, K, Y, static_cast<cudaStream_t>(stream)) == cudaSuccess
              ? SVDQ_OK
              : SVDQ_ERR_CUDA;
@@ -465,10 +548,18 @@ svdq_status svdq_linear_forward_host(const uint16_t *X_host, int M, const svdq_l
                                      uint8_t *xq, uint8_t *xs, uint16_t *lora_act, uint16_t *Y_dev, uint16_t *Y_host,
                                      void *stream) {
   if (!X_host || !Y_host || !X_dev || !Y_dev || !layer || M <= 0) return SVDQ_ERR_INVALID_ARG;
+  svdq_status st = check_layer(layer);
+  if (st != SVDQ_OK) return st;
+  if (!xq || !xs || (layer->rank > 0 && !lora_act)) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X_dev) || !aligned16(Y_dev) || !aligned16(xq) || !aligned16(xs) || !aligned16(lora_act))
+    return SVDQ_ERR_MISALIGNED;
+  DeviceState *d = nullptr;
+  st = device_check(&d);
+  if (st != SVDQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const size_t xb = static_cast<size_t>(M) * layer->K * 2, yb = static_cast<size_t>(M) * layer->N * 2;
   if (cudaMemcpyAsync(X_dev, X_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess) return SVDQ_ERR_CUDA;
-  svdq_status st = svdq_linear_forward(X_dev, M, layer, xq, xs, lora_act, Y_dev, stream);
+  st = svdq_linear_forward(X_dev, M, layer, xq, xs, lora_act, Y_dev, stream);
   if (st != SVDQ_OK) return st;
   if (cudaMemcpyAsync(Y_host, Y_dev, yb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return SVDQ_ERR_CUDA;
   return cudaStreamSynchronize(s) == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
@@ -496,21 +587,39 @@ svdq_status svdq_baseline_lora_up(const uint16_t *lora_act, int M, const svdq_la
 }
 
 svdq_status svdq_selftest_wait_timeout(uint32_t limit_us, void *stream) {
+  if (limit_us < 1 || limit_us > 1000000) return SVDQ_ERR_INVALID_ARG;
   DeviceState *d = nullptr;
   svdq_status st = device_check(&d);
   if (st != SVDQ_OK) return st;
-  if (limit_us < 1 || limit_us > 1000000) return SVDQ_ERR_INVALID_ARG;
   return launch_selftest_wait(d->err, static_cast<uint64_t>(limit_us) * 1000ull, static_cast<cudaStream_t>(stream)) ==
                  cudaSuccess
              ? SVDQ_OK
              : SVDQ_ERR_CUDA;
 }
 
+svdq_status svdq_unswizzle_scales(const uint8_t *blocked, int rows, int K, uint8_t *rowmajor) {
+  if (!blocked || !rowmajor || rows <= 0 || K <= 0 || K % 64) return SVDQ_ERR_INVALID_ARG;
+  const uint32_t ng = static_cast<uint32_t>(K / 16);
+  for (uint32_t m = 0; m < static_cast<uint32_t>(rows); ++m)
+    for (uint32_t g = 0; g < ng; ++g) rowmajor[static_cast<size_t>(m) * ng + g] = blocked[scale_offset(m, g, ng)];
+  return SVDQ_OK;
+}
+
+svdq_status svdq_test_override_capability(int major, int minor) {
+  if (major < 0) {
+    g_cap_override.store(-1, std::memory_order_relaxed);
+    return SVDQ_OK;
+  }
+  if (major > 99 || minor < 0 || minor > 9) return SVDQ_ERR_INVALID_ARG;
+  g_cap_override.store(major * 10 + minor, std::memory_order_relaxed);
+  return SVDQ_OK;
+}
+
 svdq_status svdq_last_device_error(void *stream, uint32_t *code) {
+  if (!code) return SVDQ_ERR_INVALID_ARG;
   DeviceState *d = nullptr;
   svdq_status st = device_check(&d);
   if (st != SVDQ_OK) return st;
-  if (!code) return SVDQ_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (cudaStreamSynchronize(s) != cudaSuccess) return SVDQ_ERR_CUDA;
   uint32_t v = 0;

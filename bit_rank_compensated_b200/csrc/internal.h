@@ -107,6 +107,7 @@ struct PrepArgs {
   uint8_t *wq, *wscales;
   size_t wscale_bytes;
   float *s_w, *s_x;  // host outputs
+  float *R_out_host = nullptr;  // host, N x K: the fp32 residual the weight quantizer read (may be null)
   cudaStream_t stream;
 };
 

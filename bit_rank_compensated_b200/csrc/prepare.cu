@@ -522,6 +522,7 @@ PrepStatus prepare_run(const PrepArgs &p) {
   const float s_x = hs[1] > 0.0f ? hs[1] / 2688.0f : 1.0f;
   PCHK(cudaMemsetAsync(p.wscales, 0, p.wscale_bytes, st));
   PCHK(launch_quantize_rows(R, N, K, s_w, p.wq, p.wscales, st));
+  if (p.R_out_host) PCHK(cudaMemcpyAsync(p.R_out_host, R, sizeof(float) * nk, cudaMemcpyDeviceToHost, st));
   PCHK(cudaStreamSynchronize(st));
   *p.s_w = s_w;
   *p.s_x = s_x;

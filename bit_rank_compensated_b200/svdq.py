@@ -30,7 +30,8 @@ EXPORTED = (
     "svdq_baseline_quantize", "svdq_baseline_gemm_w4a4", "svdq_baseline_lora_up", "svdq_last_device_error",
     "svdq_smoothing_factors_noalloc", "svdq_selftest_wait_timeout", "svdq_gemm_w4a4_lora_up_qk_norm_rope",
     "svdq_qk_norm_rope", "svdq_awq_quantize_weights", "svdq_awq_gemv_w4a16", "svdq_awq_pack_weights",
-    "svdq_awq_packed_weight_bytes", "svdq_awq_packed_sz_bytes",
+    "svdq_awq_packed_weight_bytes", "svdq_awq_packed_sz_bytes", "svdq_prepare_weights_host",
+    "svdq_unswizzle_scales", "svdq_test_override_capability",
 )
 
 
@@ -90,6 +91,9 @@ def load() -> ctypes.CDLL:
         "svdq_awq_pack_weights": ([P, P, P, I, I, P, P, P], I),
         "svdq_awq_packed_weight_bytes": ([I, I], S),
         "svdq_awq_packed_sz_bytes": ([I, I], S),
+        "svdq_prepare_weights_host": ([P, P, P, I, I, I, LP, P, P], I),
+        "svdq_unswizzle_scales": ([P, I, I, P], I),
+        "svdq_test_override_capability": ([I, I], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -205,6 +209,46 @@ def prepare_weights(W: torch.Tensor, bias: torch.Tensor | None, act_absmax_: tor
         _stream(stream)))
     del ws
     return L
+
+
+def prepare_weights_host(W, bias, act_absmax_, rank: int, return_residual: bool = False, device="cuda",
+                         stream=None):
+    """svdq_prepare_weights_host: prepare a layer from host (numpy) arrays. With
+    return_residual the fp32 residual R (N x K numpy array) the weight quantizer read comes back too."""
+    import numpy as np
+
+    W = np.ascontiguousarray(W, dtype=np.float32)
+    N, K = W.shape
+    ax = np.ascontiguousarray(act_absmax_, dtype=np.float32)
+    b = None if bias is None else np.ascontiguousarray(bias, dtype=np.float32)
+    L = Layer(N, K, rank, device=device, with_bias=b is not None)
+    R = np.empty((N, K), dtype=np.float32) if return_residual else None
+    _check("svdq_prepare_weights_host", load().svdq_prepare_weights_host(
+        W.ctypes.data_as(ctypes.c_void_p), None if b is None else b.ctypes.data_as(ctypes.c_void_p),
+        ax.ctypes.data_as(ctypes.c_void_p), N, K, rank, ctypes.byref(L.s),
+        None if R is None else R.ctypes.data_as(ctypes.c_void_p), _stream(stream)))
+    return (L, R) if return_residual else L
+
+
+def unswizzle_scales(blocked, rows: int, K: int):
+    """svdq_unswizzle_scales: group scales of `rows` rows from the block layout (host bytes, e.g. a
+    buffer copied back from the device) to a row-major numpy array rows x K/16."""
+    import numpy as np
+
+    buf = np.ascontiguousarray(np.asarray(blocked, dtype=np.uint8).reshape(-1))
+    need = (rows + 127) // 128 * 128 * (K // 16)
+    if buf.size < need:
+        raise ValueError(f"blocked scale buffer holds {buf.size} bytes, {need} needed")
+    out = np.empty((rows, K // 16), dtype=np.uint8)
+    _check("svdq_unswizzle_scales", load().svdq_unswizzle_scales(
+        buf.ctypes.data_as(ctypes.c_void_p), rows, K, out.ctypes.data_as(ctypes.c_void_p)))
+    return out
+
+
+def test_override_capability(major: int, minor: int = 0) -> None:
+    """Test hook: make the library treat the GPU as compute capability major.minor (major < 0
+    removes the override)."""
+    _check("svdq_test_override_capability", load().svdq_test_override_capability(int(major), int(minor)))
 
 
 def smoothing_factors_noalloc(W: torch.Tensor, act_absmax_: torch.Tensor, lam=None, inv_lam=None, s_x=None,

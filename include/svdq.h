@@ -24,8 +24,13 @@
  *     function says otherwise it only enqueues work and returns; results are ready when the
  *     stream reaches that point.
  *   - Device pointers must be 16-byte aligned.
+ *   - Tensor scales (s_w, s_x, the s of svdq_quantize_rows) lie in [2^-116, 2^116]: there every
+ *     non-zero group scale times s is a normal fp32 number, which the quantizers' exact
+ *     division relies on. Others return SVDQ_ERR_INVALID_ARG.
  *   - Shape limits: M >= 1; K % 64 == 0; N % 16 == 0; rank in {0, 16, 32, 64, 128}.
  *     Other values return SVDQ_ERR_INVALID_ARG; misaligned pointers SVDQ_ERR_MISALIGNED.
+ *     Arguments are checked before the device is queried, so these errors are reported the
+ *     same way on any machine.
  *   - The first call on a device checks for compute capability 10.0 and returns
  *     SVDQ_ERR_UNSUPPORTED_ARCH on any other GPU. There is no fallback path.
  *   - Device-side waits are bounded; a kernel that gives up records a code that
@@ -127,6 +132,23 @@ SVDQ_API size_t svdq_prepare_workspace_bytes(int N, int K, int rank, svdq_status
 SVDQ_API svdq_status svdq_prepare_weights(const float *W, const float *bias, const float *act_absmax,
                                  int N, int K, int rank, svdq_layer *layer,
                                  void *workspace, size_t workspace_bytes, void *stream);
+
+/* svdq_prepare_weights from host memory, for offline preparation and for checking the weight
+ * quantizer at full size: the same steps and outputs, plus the residual the quantizer read.
+ *   W_host           host, N x K fp32.
+ *   bias_host        host, N fp32, or NULL. Copied into layer->bias when both are non-NULL.
+ *   act_absmax_host  host, K fp32 calibration maxima a_x.
+ *   layer            as for svdq_prepare_weights (device buffers preallocated by the caller).
+ *   R_out_host       host, N x K fp32, or NULL: receives R = fp32(W_hat - (diag(lambda) L1s L2)^T),
+ *                    the matrix whose NVFP4 codes and scales land in layer->wq / layer->ws (two
+ *                    fp64 routes to the SVD can differ in the last bits of R, so a test of the
+ *                    weight quantizer takes R from here).
+ * This offline entry point allocates and frees its own device memory (a copy of W, the maxima and
+ * the workspace: N K 4 bytes plus svdq_prepare_workspace_bytes) with cudaMalloc / cudaFree.
+ * Synchronous: returns after the work on stream has finished. */
+SVDQ_API svdq_status svdq_prepare_weights_host(const float *W_host, const float *bias_host,
+                                               const float *act_absmax_host, int N, int K, int rank,
+                                               svdq_layer *layer, float *R_out_host, void *stream);
 
 /* NVFP4 quantization of the rows of a fp32 matrix A (rows x K) with tensor scale s
  * ("التحميل الأصلي في الناشرون": nvfp4, group 16). Per 16-element group along K:
@@ -279,14 +301,33 @@ SVDQ_API svdq_status svdq_baseline_lora_up(const uint16_t *lora_act, int M, cons
  *   x_tensor_scale   device, 1 fp32 (out).
  * Its scratch (K column maxima and one running maximum) is a static device array inside the
  * library sized for K <= 65536 (256 KiB, held on every GPU that loads the library until the
- * process exits); larger K returns SVDQ_ERR_INVALID_ARG. It calls no allocating routine. The
- * first call on a device looks up the array's device address (once per device), so make that
- * first call before any stream capture. All calls share the array and the call clears what must
+ * process exits); larger K, K % 64 != 0, N <= 0 or a NULL pointer return SVDQ_ERR_INVALID_ARG.
+ * It calls no allocating routine. The first call on a device looks up the array's device address
+ * (once per device), so make that first call before any stream capture; if that lookup fails,
+ * every later call on that device returns SVDQ_ERR_CUDA for the rest of the process. All calls share the array and the call clears what must
  * start at zero; calls that overlap on the GPU (other streams, other threads) race on it.
  * Asynchronous on stream. */
 SVDQ_API svdq_status svdq_smoothing_factors_noalloc(const float *W, const float *act_absmax, int N, int K,
                                                     float *lambda, float *inv_lambda, float *x_tensor_scale,
                                                     void *stream);
+
+/* Group scales from the block layout (as svdq_quant_act_lora_down, svdq_quantize_rows and
+ * svdq_prepare_weights write them) to row-major order: rowmajor[m * (K / 16) + g] = the e4m3
+ * code of row m, group g, for m < rows. Pure host code, no device needed.
+ *   blocked   host, at least ceil(rows / 128) * 128 * K / 16 bytes (the stored layout; padding
+ *             rows are not read).
+ *   rowmajor  host, rows * K / 16 bytes (out).
+ * Errors: SVDQ_ERR_INVALID_ARG for NULL pointers, rows <= 0, K <= 0 or K % 64 != 0. */
+SVDQ_API svdq_status svdq_unswizzle_scales(const uint8_t *blocked, int rows, int K, uint8_t *rowmajor);
+
+/* Test hook for the architecture check. After svdq_test_override_capability(major, minor) every
+ * entry point that would use the GPU acts as if the device reported compute capability
+ * major.minor: anything other than 10.0 returns SVDQ_ERR_UNSUPPORTED_ARCH before any CUDA call,
+ * so the refusal path can be exercised on any machine; 10.0 falls through to the real check (the
+ * hook can make a B200 look unsupported, never the reverse). major < 0 removes the override.
+ * Argument checks still come first. Returns SVDQ_ERR_INVALID_ARG for major > 99 or minor
+ * outside 0..9. Process-wide; not meant for production use. */
+SVDQ_API svdq_status svdq_test_override_capability(int major, int minor);
 
 /* Failure-path self-test. Launches one CTA whose bounded waits (the same code every kernel of
  * the library uses) wait on an mbarrier that nothing signals; each gives up after limit_us
