@@ -81,6 +81,8 @@ svdq_status device_check(DeviceState **out) {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
+
 bool rank_ok(int r) { return r == 0 || r == 16 || r == 32 || r == 64 || r == 128; }
 
 // Tensor scales the quantizers handle exactly: with s in [2^-116, 2^116] every non-zero group
@@ -171,11 +173,20 @@ struct QkNormRope {
   float eps;
 };
 
+// Output of the fused MLP pair's first GEMM: the down layer's activations.
+struct MlpOut {
+  const svdq_layer *down;
+  uint8_t *xq, *xs;
+  uint16_t *la;  // M x 2 rank_down bf16 ([hi | lo])
+  float *part;   // [ceil(N_up / 256)][M][rank_down] fp32
+};
+
 svdq_status run_gemm(const uint8_t *xq, const uint8_t *xs, const uint16_t *la, int M, const svdq_layer *L,
-                     uint16_t *Y, bool fp4, bool add_y, bool lora, void *stream, const QkNormRope *qk = nullptr) {
+                     uint16_t *Y, bool fp4, bool add_y, bool lora, void *stream, const QkNormRope *qk = nullptr,
+                     bool gelu = false, const MlpOut *mlp = nullptr) {
   svdq_status st = check_layer(L);
   if (st != SVDQ_OK) return st;
-  if (M <= 0 || !Y) return SVDQ_ERR_INVALID_ARG;
+  if (M <= 0 || (!Y && !mlp)) return SVDQ_ERR_INVALID_ARG;
   if (fp4 && (!xq || !xs)) return SVDQ_ERR_INVALID_ARG;
   const int r = lora ? L->rank : 0;
   if (r > 0 && !la) return SVDQ_ERR_INVALID_ARG;
@@ -199,9 +210,10 @@ svdq_status run_gemm(const uint8_t *xq, const uint8_t *xs, const uint16_t *la, i
         !make_map(&g.tm_l2, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, L->L2t, r, N, static_cast<uint64_t>(r) * 2, kc, 128, sw))
       return SVDQ_ERR_CUDA;
   }
-  if (!make_map(&g.tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 64, 128,
-                CU_TENSOR_MAP_SWIZZLE_128B))
+  if (Y && !make_map(&g.tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, static_cast<uint64_t>(N) * 2, 64, 128,
+                     CU_TENSOR_MAP_SWIZZLE_128B))
     return SVDQ_ERR_CUDA;
+  if (!Y) g.tm_y = g.tm_xq;  // the fused MLP pair writes no Y
   if (!fp4) {
     g.tm_xq = g.tm_la;
     g.tm_wq = g.tm_l2;
@@ -232,13 +244,39 @@ svdq_status run_gemm(const uint8_t *xq, const uint8_t *xs, const uint16_t *la, i
                   CU_TENSOR_MAP_SWIZZLE_128B))
       return SVDQ_ERR_CUDA;
   }
+  g.gelu = gelu;
+  if (mlp) {
+    const svdq_layer *D = mlp->down;
+    g.mlp = true;
+    g.il_d = D->inv_lambda;
+    g.sx_d = D->x_tensor_scale;
+    g.rank_d = D->rank;
+    g.mp_scales = static_cast<int>(round_up(static_cast<size_t>(M), 128));
+    g.xq_d = mlp->xq;
+    g.xs_d = mlp->xs;
+    g.part = mlp->part;
+    if (D->rank > 0) {
+      // L1t of the down layer: rank_d rows of N (= its K) bf16; boxes of 32 columns x rank_d / 2 rows
+      if (!make_map(&g.tm_l1d, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D->L1t, N, D->rank, static_cast<uint64_t>(N) * 2, 32,
+                    D->rank / 2, CU_TENSOR_MAP_SWIZZLE_64B))
+        return SVDQ_ERR_CUDA;
+    } else {
+      g.tm_l1d = g.tm_xq;
+    }
+  }
   g.num_sms = d->num_sms;
   g.err = d->err;
   g.stream = static_cast<cudaStream_t>(stream);
-  return launch_gemm(g) == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+  if (launch_gemm(g) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (mlp && mlp->down->rank > 0) {
+    const svdq_layer *D = mlp->down;
+    const float inv_alpha_d = 1.0f / alpha_of(D);
+    if (launch_lora_reduce(mlp->part, gemm_n_tiles(N), M, D->rank, inv_alpha_d, mlp->la,
+                           g.stream) != cudaSuccess)
+      return SVDQ_ERR_CUDA;
+  }
+  return SVDQ_OK;
 }
-
-size_t round_up(size_t a, size_t b) { return (a + b - 1) / b * b; }
 
 }  // namespace
 }  // namespace svdq
@@ -452,6 +490,46 @@ svdq_status svdq_quant_act_lora_down(const uint16_t *X, int M, const svdq_layer 
 svdq_status svdq_gemm_w4a4_lora_up(const uint8_t *xq, const uint8_t *xs, const uint16_t *lora_act, int M,
                                    const svdq_layer *layer, uint16_t *Y, void *stream) {
   return run_gemm(xq, xs, lora_act, M, layer, Y, true, false, true, stream);
+}
+
+size_t svdq_mlp_workspace_bytes(int M, int N_up, int rank_down) {
+  if (M <= 0 || N_up <= 0 || N_up % 64 || !(rank_down == 0 || rank_down == 16 || rank_down == 32 || rank_down == 64))
+    return 0;
+  return static_cast<size_t>(gemm_n_tiles(N_up)) * static_cast<size_t>(M) * static_cast<size_t>(rank_down) * 4u;
+}
+
+svdq_status svdq_gemm_w4a4_lora_up_gelu(const uint8_t *xq, const uint8_t *xs, const uint16_t *lora_act, int M,
+                                        const svdq_layer *layer, uint16_t *H, void *stream) {
+  return run_gemm(xq, xs, lora_act, M, layer, H, true, false, true, stream, nullptr, true);
+}
+
+svdq_status svdq_gemm_w4a4_lora_up_gelu_quant(const uint8_t *xq, const uint8_t *xs, const uint16_t *lora_act, int M,
+                                              const svdq_layer *up, const svdq_layer *down, uint8_t *xq_down,
+                                              uint8_t *xs_down, uint16_t *lora_act_down, void *workspace,
+                                              size_t workspace_bytes, void *stream) {
+  if (!up || !down) return SVDQ_ERR_INVALID_ARG;
+  svdq_status st = check_layer(down);
+  if (st != SVDQ_OK) return st;
+  if (down->K != up->N || down->rank > 64 || M <= 0) return SVDQ_ERR_INVALID_ARG;
+  if (!xq_down || !xs_down) return SVDQ_ERR_INVALID_ARG;
+  if (down->rank > 0 && (!lora_act_down || !workspace || workspace_bytes < svdq_mlp_workspace_bytes(M, up->N, down->rank)))
+    return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(xq_down) || !aligned16(xs_down) || !aligned16(lora_act_down) || !aligned16(workspace))
+    return SVDQ_ERR_MISALIGNED;
+  const MlpOut mo{down, xq_down, xs_down, lora_act_down, static_cast<float *>(workspace)};
+  return run_gemm(xq, xs, lora_act, M, up, nullptr, true, false, true, stream, nullptr, false, &mo);
+}
+
+svdq_status svdq_mlp_forward(const uint16_t *X, int M, const svdq_layer *up, const svdq_layer *down, uint8_t *xq,
+                             uint8_t *xs, uint16_t *lora_act, uint8_t *xq_down, uint8_t *xs_down,
+                             uint16_t *lora_act_down, void *workspace, size_t workspace_bytes, uint16_t *Z,
+                             void *stream) {
+  svdq_status st = svdq_quant_act_lora_down(X, M, up, xq, xs, lora_act, stream);
+  if (st != SVDQ_OK) return st;
+  st = svdq_gemm_w4a4_lora_up_gelu_quant(xq, xs, lora_act, M, up, down, xq_down, xs_down, lora_act_down, workspace,
+                                         workspace_bytes, stream);
+  if (st != SVDQ_OK) return st;
+  return svdq_gemm_w4a4_lora_up(xq_down, xs_down, lora_act_down, M, down, Z, stream);
 }
 
 namespace {

@@ -52,11 +52,26 @@ struct GemmLaunch {
   const float *norm_q, *norm_k;  // [128] each
   int qk_width;
   float eps;
+  bool gelu;  // H = bf16(GELU(alpha acc + bias)) instead of Y (first layer of an unfused MLP pair)
+  // Fused MLP pair: GELU(alpha acc + bias) quantized for the down layer (codes, block scales with
+  // mp_scales rows) plus fp32 partial down-projections [ceil(N / 256)][M][rank_d] against L1t_d.
+  bool mlp;
+  CUtensorMap tm_l1d;  // L1t_d, bf16 [rank_d, N], box 32 x rank_d / 2, 64B swizzle
+  const float *il_d;
+  float sx_d;
+  int rank_d, mp_scales;
+  uint8_t *xq_d, *xs_d;
+  float *part;
   int num_sms;
   uint32_t *err;
   cudaStream_t stream;
 };
 cudaError_t launch_gemm(const GemmLaunch &g);
+// Column tiles of K2 (256 rows of W each): the number of partial-sum slots of the fused MLP pair.
+int gemm_n_tiles(int N);
+// lora_act = [hi | lo] of (sum over n_slots slots of part[slot][m][:], in slot order) * inv_alpha.
+cudaError_t launch_lora_reduce(const float *part, int n_slots, int M, int rank, float inv_alpha, uint16_t *lora_act,
+                               cudaStream_t st);
 
 // Unfused per-head Q/K normalization and rotary embedding of a bf16 Y = [Q | K | V], in place.
 cudaError_t launch_qk_norm_rope(uint16_t *Y, int M, int heads, const float *norm_q, const float *norm_k,

@@ -31,7 +31,8 @@ EXPORTED = (
     "svdq_smoothing_factors_noalloc", "svdq_selftest_wait_timeout", "svdq_gemm_w4a4_lora_up_qk_norm_rope",
     "svdq_qk_norm_rope", "svdq_awq_quantize_weights", "svdq_awq_gemv_w4a16", "svdq_awq_pack_weights",
     "svdq_awq_packed_weight_bytes", "svdq_awq_packed_sz_bytes", "svdq_prepare_weights_host",
-    "svdq_unswizzle_scales", "svdq_test_override_capability",
+    "svdq_unswizzle_scales", "svdq_test_override_capability", "svdq_mlp_workspace_bytes",
+    "svdq_gemm_w4a4_lora_up_gelu_quant", "svdq_gemm_w4a4_lora_up_gelu", "svdq_mlp_forward",
 )
 
 
@@ -94,6 +95,10 @@ def load() -> ctypes.CDLL:
         "svdq_prepare_weights_host": ([P, P, P, I, I, I, LP, P, P], I),
         "svdq_unswizzle_scales": ([P, I, I, P], I),
         "svdq_test_override_capability": ([I, I], I),
+        "svdq_mlp_workspace_bytes": ([I, I, I], S),
+        "svdq_gemm_w4a4_lora_up_gelu_quant": ([P, P, P, I, LP, LP, P, P, P, P, S, P], I),
+        "svdq_gemm_w4a4_lora_up_gelu": ([P, P, P, I, LP, P, P], I),
+        "svdq_mlp_forward": ([P, I, LP, LP, P, P, P, P, P, P, P, S, P, P], I),
     }
     for name, (args, res) in sig.items():
         f = getattr(lib, name)
@@ -362,6 +367,53 @@ def awq_gemv_w4a16(X: torch.Tensor, lin: "AwqLinear", Y=None, stream=None):
     _check("svdq_awq_gemv_w4a16", load().svdq_awq_gemv_w4a16(
         _ptr(X), M, _ptr(lin.wt), _ptr(lin.szt), _ptr(lin.bias), lin.N, K, _ptr(Y), _stream(stream)))
     return Y
+
+
+def mlp_workspace_bytes(M: int, up: Layer, down: Layer) -> int:
+    return load().svdq_mlp_workspace_bytes(M, up.N, down.rank)
+
+
+def alloc_mlp_workspace(M: int, up: Layer, down: Layer, device="cuda"):
+    n = mlp_workspace_bytes(M, up, down)
+    return torch.empty(max(n, 16), dtype=torch.uint8, device=device)
+
+
+def gemm_w4a4_lora_up_gelu_quant(xq, xs, lora_act, M: int, up: Layer, down: Layer, bufs_down=None, workspace=None,
+                                 stream=None):
+    """The fused MLP pair's middle: the down layer's (xq, xs, lora_act) from GELU(up layer output)."""
+    if bufs_down is None:
+        bufs_down = alloc_activations(M, down, xq.device)
+    if workspace is None:
+        workspace = alloc_mlp_workspace(M, up, down, xq.device)
+    xq_d, xs_d, la_d = bufs_down
+    _check("svdq_gemm_w4a4_lora_up_gelu_quant", load().svdq_gemm_w4a4_lora_up_gelu_quant(
+        _ptr(xq), _ptr(xs), _ptr(lora_act), M, ctypes.byref(up.s), ctypes.byref(down.s), _ptr(xq_d), _ptr(xs_d),
+        _ptr(la_d), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return bufs_down
+
+
+def gemm_w4a4_lora_up_gelu(xq, xs, lora_act, M: int, layer: Layer, H=None, stream=None):
+    """H = bf16(GELU(layer output)): the unfused pair's first layer."""
+    if H is None:
+        H = torch.empty(M, layer.N, dtype=torch.bfloat16, device=xq.device)
+    _check("svdq_gemm_w4a4_lora_up_gelu", load().svdq_gemm_w4a4_lora_up_gelu(
+        _ptr(xq), _ptr(xs), _ptr(lora_act), M, ctypes.byref(layer.s), _ptr(H), _stream(stream)))
+    return H
+
+
+def mlp_forward(X, up: Layer, down: Layer, bufs=None, bufs_down=None, workspace=None, Z=None, stream=None):
+    """The fused FLUX feed-forward pair Z = down(GELU(up(X)))."""
+    M = X.shape[0]
+    xq, xs, la = bufs if bufs is not None else alloc_activations(M, up, X.device)
+    xq_d, xs_d, la_d = bufs_down if bufs_down is not None else alloc_activations(M, down, X.device)
+    if workspace is None:
+        workspace = alloc_mlp_workspace(M, up, down, X.device)
+    if Z is None:
+        Z = torch.empty(M, down.N, dtype=torch.bfloat16, device=X.device)
+    _check("svdq_mlp_forward", load().svdq_mlp_forward(
+        _ptr(X), M, ctypes.byref(up.s), ctypes.byref(down.s), _ptr(xq), _ptr(xs), _ptr(la), _ptr(xq_d), _ptr(xs_d),
+        _ptr(la_d), _ptr(workspace), workspace.numel(), _ptr(Z), _stream(stream)))
+    return Z
 
 
 def linear_forward(X: torch.Tensor, layer: Layer, bufs=None, Y=None, stream=None):

@@ -222,6 +222,42 @@ SVDQ_API svdq_status svdq_gemm_w4a4_lora_up_qk_norm_rope(const uint8_t *xq, cons
 SVDQ_API svdq_status svdq_qk_norm_rope(uint16_t *Y, int M, int heads, int head_dim, const float *norm_q_weight,
                                        const float *norm_k_weight, const float *rope, float eps, void *stream);
 
+/* The FLUX feed-forward pair, Linear -> GELU (tanh form) -> Linear, with both linears SVDQuant
+ * layers ("Nunchaku Lite in Diffusers", introduction of Nunchaku Lite: the engine's fused GELU / MLP
+ * kernels). GELU(v) = 0.5 v (1 + tanh(sqrt(2 / pi) (v + 0.044715 v^3))).
+ *
+ * svdq_gemm_w4a4_lora_up_gelu_quant — the fused pair's middle: K2 of the up layer whose output
+ * stage, instead of writing Y, computes h = GELU(alpha acc + bias) in fp32 and produces the down
+ * layer's activations exactly as svdq_quant_act_lora_down would from an unrounded input h:
+ *   xq_down, xs_down  NVFP4 codes / block scales of x_hat = fp32(h inv_lambda_down) with the down
+ *                     layer's s_x (same quantizer, same formats; padding scale rows zero);
+ *   lora_act_down     [hi | lo] of fp32(sum_k h[m, k] L1s_down[k, :]) / alpha_down, the sum formed
+ *                     on the tensor cores from the bf16 pair hi = bf16(h), lo = bf16(h - hi) per
+ *                     256 columns, and the per-tile partials added in tile order (deterministic).
+ * The M x N_up intermediate never reaches memory in 16 bits. Requirements: down->K == up->N,
+ * down->rank in {0, 16, 32, 64}.
+ *   workspace  device, at least svdq_mlp_workspace_bytes(M, up->N, down->rank) bytes (the fp32
+ *              partials; may be NULL at down rank 0). Owned by the caller, contents not kept.
+ * Asynchronous on stream.
+ *
+ * svdq_gemm_w4a4_lora_up_gelu — the unfused pair's first layer: Y = bf16(GELU(alpha acc + bias)),
+ * the bf16 intermediate that svdq_quant_act_lora_down of the down layer then reads back.
+ *
+ * svdq_mlp_forward — the fused pair: svdq_quant_act_lora_down (up), then the fused middle, then
+ * svdq_gemm_w4a4_lora_up (down) writing Z (M x down->N bf16). Buffers as above. Asynchronous. */
+SVDQ_API size_t svdq_mlp_workspace_bytes(int M, int N_up, int rank_down);
+SVDQ_API svdq_status svdq_gemm_w4a4_lora_up_gelu_quant(const uint8_t *xq, const uint8_t *xs,
+                                                       const uint16_t *lora_act, int M, const svdq_layer *up,
+                                                       const svdq_layer *down, uint8_t *xq_down, uint8_t *xs_down,
+                                                       uint16_t *lora_act_down, void *workspace,
+                                                       size_t workspace_bytes, void *stream);
+SVDQ_API svdq_status svdq_gemm_w4a4_lora_up_gelu(const uint8_t *xq, const uint8_t *xs, const uint16_t *lora_act,
+                                                 int M, const svdq_layer *layer, uint16_t *H, void *stream);
+SVDQ_API svdq_status svdq_mlp_forward(const uint16_t *X, int M, const svdq_layer *up, const svdq_layer *down,
+                                      uint8_t *xq, uint8_t *xs, uint16_t *lora_act, uint8_t *xq_down,
+                                      uint8_t *xs_down, uint16_t *lora_act_down, void *workspace,
+                                      size_t workspace_bytes, uint16_t *Z, void *stream);
+
 /* awq_w4a16 — the second kernel family ("Nunchaku Lite in Diffusers": 4-bit weights with 16-bit
  * activations for the adaptive-normalization / modulation projections, memory-bound and
  * precision-sensitive; quantization_config: int4, group_size 64).

@@ -82,6 +82,14 @@ def _calls(lib, layer, X=DEV, M=256, out=DEV):
             P(X), P(X), N, K, P(out), P(out), P(out), None),
         "svdq_prepare_weights": lambda: lib.svdq_prepare_weights(P(X), None, P(X), N, K, layer.rank, L, P(out), 1 << 30,
                                                                  None),
+        "svdq_gemm_w4a4_lora_up_gelu": lambda: lib.svdq_gemm_w4a4_lora_up_gelu(P(out), P(out), P(out), M, L, P(out),
+                                                                               None),
+        "svdq_gemm_w4a4_lora_up_gelu_quant": lambda: lib.svdq_gemm_w4a4_lora_up_gelu_quant(
+            P(out), P(out), P(out), M, L, ctypes.byref(_layer(N=256, K=N, rank=16)), P(out), P(out), P(out), P(out),
+            1 << 30, None),
+        "svdq_mlp_forward": lambda: lib.svdq_mlp_forward(
+            P(X), M, L, ctypes.byref(_layer(N=256, K=N, rank=16)), P(out), P(out), P(out), P(out), P(out), P(out),
+            P(out), 1 << 30, P(out), None),
         "svdq_selftest_wait_timeout": lambda: lib.svdq_selftest_wait_timeout(1000, None),
         "svdq_last_device_error": lambda: lib.svdq_last_device_error(None, ctypes.byref(ctypes.c_uint32(0))),
     }
@@ -164,6 +172,24 @@ def test_tensor_scale_range(lib, unsupported):
                                             None) == UNSUPPORTED
     assert lib.svdq_quantize_rows(_p(DEV), 16, 64, 2.0 ** -117, 128, _p(DEV), _p(DEV), None) == INVALID
     assert lib.svdq_quantize_rows(_p(DEV), 16, 64, float("nan"), 128, _p(DEV), _p(DEV), None) == INVALID
+
+
+def test_mlp_pair_shapes_are_checked_before_the_device(lib, unsupported):
+    up = _layer(N=512, K=512, rank=16)
+    P = _p
+    for down in (_layer(N=256, K=256, rank=16),     # down K != up N
+                 _layer(N=256, K=512, rank=128)):   # down rank above 64
+        assert lib.svdq_gemm_w4a4_lora_up_gelu_quant(P(DEV), P(DEV), P(DEV), 64, ctypes.byref(up), ctypes.byref(down),
+                                                     P(DEV), P(DEV), P(DEV), P(DEV), 1 << 30, None) == INVALID
+    down = _layer(N=256, K=512, rank=32)
+    need = lib.svdq_mlp_workspace_bytes(64, 512, 32)
+    assert need == 2 * 64 * 32 * 4  # two 256-column tiles of fp32 partials
+    assert lib.svdq_gemm_w4a4_lora_up_gelu_quant(P(DEV), P(DEV), P(DEV), 64, ctypes.byref(up), ctypes.byref(down),
+                                                 P(DEV), P(DEV), P(DEV), P(DEV), need - 4, None) == INVALID
+    assert lib.svdq_gemm_w4a4_lora_up_gelu_quant(P(DEV), P(DEV), P(DEV), 64, ctypes.byref(up), ctypes.byref(down),
+                                                 P(DEV), P(DEV), P(DEV), P(DEV), need, None) == UNSUPPORTED
+    assert lib.svdq_mlp_workspace_bytes(64, 500, 32) == 0
+    assert lib.svdq_mlp_workspace_bytes(64, 512, 128) == 0
 
 
 def test_null_layer_is_rejected(lib, unsupported):
