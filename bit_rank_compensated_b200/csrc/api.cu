@@ -610,7 +610,8 @@ svdq_status svdq_awq_gemv_w4a16(const uint16_t *X, int M, const uint8_t *wq_pack
   DeviceState *d = nullptr;
   svdq_status st = device_check(&d);
   if (st != SVDQ_OK) return st;
-  return launch_awq_gemv(X, M, wq_packed, sz_packed, bias, N, K, Y, static_cast<cudaStream_t>(stream)) == cudaSuccess
+  return launch_awq_gemv(X, M, wq_packed, sz_packed, bias, N, K, Y, d->err, static_cast<cudaStream_t>(stream)) ==
+                 cudaSuccess
              ? SVDQ_OK
              : SVDQ_ERR_CUDA;
 }

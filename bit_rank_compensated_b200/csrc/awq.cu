@@ -26,7 +26,6 @@ namespace svdq {
 namespace {
 
 constexpr int kAwqGroup = 64;
-constexpr int kGemvWarps = 8;
 
 // One thread per group of 64: round-to-nearest int4 with a zero point, decided in fp32.
 __global__ void awq_quantize_kernel(const float *W, int N, int K, uint8_t *wq, uint16_t *scales, uint8_t *zeros) {
@@ -124,63 +123,77 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-constexpr int kPf = 8;  // tiles a warp has in flight
+// Streaming tensor-core GEMV. The work is bound by reading the 4-bit weights once, so it is
+// organised around keeping enough bytes in flight: one warp per CTA streams the CTA's tiles with
+// bulk copies (cp.async.bulk) into a ring of shared-memory slots, each slot a run of up to 16
+// consecutive groups of one row block (16 x 512 bytes of codes, 16 x 64 bytes of scales and zero
+// points, contiguous in the packed layout), up to 12 slots (108 KiB) ahead; no registers are held
+// per tile in flight.
+// The 16 consumer warps take one group each of every run (warp w: group 16 j + w of run j of the
+// row block): an m16n8k16 bf16 MMA per k-step with the 16 weight rows of the row block as operand
+// A (each code q turned into the exact bf16 integer 128 + q, one LOP3 per pair) and up to 8 tokens
+// as operand B (the bf16 activations, staged once per CTA in fragment order); the products are
+// exact and summed in fp32, and the scale and zero point enter once per group:
+// acc += s D_G - s (128 + z) sum_G(x). At the end of a row block the 16 warps' sums meet in shared
+// memory and warp 0 adds them in warp order (deterministic) and writes Y. Row blocks are dealt to
+// the CTAs round-robin (persistent grid, one CTA per SM at the benchmarked shapes).
+constexpr int kCW = 16;                               // consumer warps
+constexpr int kRunG = 16;                             // groups per run (slot)
+constexpr uint32_t kSlotBytes = kRunG * (512 + 64);   // 9 KiB
+constexpr int kMaxSlots = 12;
+constexpr uint32_t kRedBytes = kCW * 32 * 4 * 4;      // the warps' partial sums of a row block
 
-// Tensor-core GEMV: warp-wide m16n8k16 bf16 MMAs with the 16 weight rows of a row block as
-// operand A (each code q turned into the exact bf16 integer 128 + q in registers, one LOP3 per
-// pair) and up to 8 tokens as operand B (the bf16 activations, staged once per block in fragment
-// order); the products are exact and summed in fp32, and the scale and zero point are applied per
-// group: acc += s D_G - s (128 + z) sum_G(x). (Summing 128 + q instead of q costs about 2^-23 x
-// 143 / 8 of the group's sum in rounding, ~2e-5 relative.)
-// Work: ks consecutive warps of a block (ks = 1, 2, 4 or 8) share a row block, warp slice
-// j = warp % ks taking groups j gps .. (j + 1) gps - 1 (gps = K/64 / ks); the slices' partial sums
-// meet in shared memory (double-buffered by unit parity, one named barrier per unit) and slice 0
-// adds them in slice order and writes Y. The grid is persistent: a warp group takes row blocks
-// rb0, rb0 + stride, ... and each warp streams its tiles in order, kPf ahead across row blocks.
-__global__ void __launch_bounds__(kGemvWarps * 32) awq_gemv_mma_kernel(const uint16_t *X, int M, const uint8_t *wt,
-                                                                       const uint8_t *szt, const float *bias, int N,
-                                                                       int K, int ks, uint16_t *Y) {
-  extern __shared__ uint32_t smem_w[];
+__global__ void __launch_bounds__((kCW + 1) * 32, 1)
+    awq_gemv_stream_kernel(const uint16_t *X, int M, const uint8_t *wt, const uint8_t *szt, const float *bias, int N,
+                           int K, int nslots, uint16_t *Y, uint32_t *err) {
+  extern __shared__ __align__(16) uint32_t smem_w[];
   const int gpr = K / kAwqGroup;
   uint32_t *xb = smem_w;                                       // gpr x 32 lanes x 8 words (bf16 pairs)
   float *sxg = reinterpret_cast<float *>(smem_w + gpr * 256);  // gpr x 8 tokens
-  float *red = sxg + gpr * 8;                                  // 2 x kGemvWarps x 32 lanes x 4 partial sums
+  float *red = sxg + gpr * 8;                                  // kCW warps x 32 lanes x 4 partial sums
+  uint8_t *ring = reinterpret_cast<uint8_t *>(red) + kRedBytes;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(ring + static_cast<size_t>(nslots) * kSlotBytes);
+  const uint32_t bar_full = smem_u32(bars), bar_empty = bar_full + 8 * nslots;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int row_blocks = (N + 15) / 16;
-  const int slice = warp % ks, gps = gpr / ks, g0 = slice * gps;
-  const int stride = gridDim.x * (kGemvWarps / ks);             // row blocks per round of the grid
-  const int rb0 = blockIdx.x * (kGemvWarps / ks) + warp / ks;
-  const int units = rb0 < row_blocks ? (row_blocks - 1 - rb0) / stride + 1 : 0;
-  const int items = units * gps;
+  const int runs_per_rb = (gpr + kRunG - 1) / kRunG;
+  const int my_rbs = blockIdx.x < row_blocks ? (row_blocks - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
+  const int runs = my_rbs * runs_per_rb;
 
-  // prefetch ring over this warp's tiles: (row block rb0 + i / gps stride, group g0 + i % gps),
-  // walked with a running tile index
-  uint4 cq[kPf];
-  uint2 sz[kPf];
-  uint32_t pf_tile = static_cast<uint32_t>(rb0) * gpr + g0;  // tiles fit 32 bits (N K / 1024 < 2^32)
-  const uint32_t wrap = static_cast<uint32_t>(stride) * gpr - gps;
-  int pf_G = 0, pf_i = 0;
-  const uint4 *wt4 = reinterpret_cast<const uint4 *>(wt) + lane;
-  const uint2 *sz2 = reinterpret_cast<const uint2 *>(szt) + g;
-  auto issue = [&](int slot) {
-    if (pf_i < items) {
-      cq[slot] = __ldg(wt4 + pf_tile * 32);
-      sz[slot] = __ldg(sz2 + pf_tile * 8);
-      ++pf_tile;
-      if (++pf_G == gps) {
-        pf_G = 0;
-        pf_tile += wrap;
-      }
-      ++pf_i;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < nslots; ++i) {
+      mbar_init(bar_full + 8 * i, 1);
+      mbar_init(bar_empty + 8 * i, kCW);
     }
-  };
-#pragma unroll
-  for (int p = 0; p < kPf; ++p) issue(p);
+    fence_mbar_init();
+  }
+  __syncthreads();
 
+  if (warp == kCW) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      for (int c = 0; c < runs; ++c) {
+        const int s = c % nslots;
+        if (c >= nslots && !mbar_wait(bar_empty + 8 * s, ((c / nslots) - 1) & 1, err, KID_AWQ, 1)) break;
+        const int rb = static_cast<int>(blockIdx.x) + (c / runs_per_rb) * static_cast<int>(gridDim.x);
+        const int G0 = (c % runs_per_rb) * kRunG;
+        const int ng = min(kRunG, gpr - G0);
+        const size_t tile0 = static_cast<size_t>(rb) * gpr + G0;
+        const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * kSlotBytes);
+        mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(ng) * (512u + 64u));
+        bulk_load(dst, wt + tile0 * 512, static_cast<uint32_t>(ng) * 512u, bar_full + 8 * s);
+        bulk_load(dst + kRunG * 512u, szt + tile0 * 64, static_cast<uint32_t>(ng) * 64u, bar_full + 8 * s);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------------------------------------ consumers (512 threads)
   // Stage X in fragment order: pair w (k = 2 w) of token m goes to word (G 32 + 4 m + t) 8 + 2 s + u
-  // with k = 64 G + 16 s + 8 u + 2 t. Every thread reads consecutive pairs of the M real tokens
-  // (coalesced); the slots of tokens M .. 7 are zero.
+  // with k = 64 G + 16 s + 8 u + 2 t. Consecutive threads read consecutive pairs of the M real
+  // tokens (coalesced); the slots of tokens M .. 7 are zero.
+  const int ct = threadIdx.x, nct = kCW * 32;
   const int kw = K / 2;
   auto xb_index = [&](int m, int w) {
     const int e = (2 * w) & 63;
@@ -189,15 +202,15 @@ __global__ void __launch_bounds__(kGemvWarps * 32) awq_gemv_mma_kernel(const uin
   for (int m = 0; m < 8; ++m) {
     if (m < M) {
 #pragma unroll 4
-      for (int w = threadIdx.x; w < kw; w += blockDim.x)
+      for (int w = ct; w < kw; w += nct)
         xb[xb_index(m, w)] = __ldg(reinterpret_cast<const uint32_t *>(X + static_cast<size_t>(m) * K) + w);
     } else {
-      for (int w = threadIdx.x; w < kw; w += blockDim.x) xb[xb_index(m, w)] = 0u;
+      for (int w = ct; w < kw; w += nct) xb[xb_index(m, w)] = 0u;
     }
   }
-  __syncthreads();
+  named_bar_sync(1, nct);
   // sums of x over each group, per token, from the staged pairs (lanes 4 m .. 4 m + 3, all words)
-  for (int i = threadIdx.x; i < gpr * 8; i += blockDim.x) {
+  for (int i = ct; i < gpr * 8; i += nct) {
     const int G = i >> 3, m = i & 7;
     float sum = 0.0f;
     if (m < M) {
@@ -212,123 +225,134 @@ __global__ void __launch_bounds__(kGemvWarps * 32) awq_gemv_mma_kernel(const uin
     }
     sxg[i] = sum;
   }
-  __syncthreads();
+  named_bar_sync(1, nct);
 
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  int rb = rb0, G = g0, unit = 0;
-  for (int i0 = 0; i0 < items; i0 += kPf) {
-#pragma unroll
-    for (int p = 0; p < kPf; ++p) {
-      if (i0 + p >= items) break;
-      const uint4 c = cq[p];
-      const uint2 zz = sz[p];
-      issue(p);  // the slot's registers are copied: refill it with the tile kPf ahead
+  bool ok = true;
+  for (int c = 0; c < runs; ++c) {
+    const int s = c % nslots;
+    const int j = c % runs_per_rb;
+    const int G = j * kRunG + warp;
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_parked(bar_full + 8 * s, (c / nslots) & 1, err, KID_AWQ, 2));
+    if (ok && G < gpr) {
+      const uint8_t *slot = ring + static_cast<size_t>(s) * kSlotBytes;
+      const uint4 cq = ld_shared_u32x4(smem_u32(slot + warp * 512 + lane * 16));
+      const uint32_t zz0 = ld_shared_u32(smem_u32(slot + kRunG * 512 + warp * 64 + g * 8));
+      const uint32_t zz1 = ld_shared_u32(smem_u32(slot + kRunG * 512 + warp * 64 + g * 8 + 4));
       const uint4 xa = *reinterpret_cast<const uint4 *>(xb + (G * 32 + lane) * 8);
       const uint4 xc = *reinterpret_cast<const uint4 *>(xb + (G * 32 + lane) * 8 + 4);
       const uint32_t bx[8] = {xa.x, xa.y, xa.z, xa.w, xc.x, xc.y, xc.z, xc.w};
-      const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+      const uint32_t cw[4] = {cq.x, cq.y, cq.z, cq.w};
       float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int st = 0; st < 4; ++st) {
         uint32_t a[4];
-#pragma unroll
         // (128 + q_lo, 128 + q_hi) as a bf16 pair (exact): the 128 joins the zero point below
+#pragma unroll
         for (int r = 0; r < 4; ++r) a[r] = ((cw[st] >> (4 * r)) & 0x000F000Fu) | 0x43004300u;
         mma_bf16_16816(d, a, bx[2 * st], bx[2 * st + 1]);
       }
-      const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(zz.x & 0xFFFFu)));
-      const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(zz.x >> 16)));
+      const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(zz0 & 0xFFFFu)));
+      const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(zz0 >> 16)));
       // D = sum (128 + q) x, so acc += s D - s (128 + z) sum x (s (128 + z) is exact in fp32)
-      const float sz0 = s0 * static_cast<float>(128u + (zz.y & 0xFFu));
-      const float sz1 = s1 * static_cast<float>(128u + ((zz.y >> 8) & 0xFFu));
+      const float sz0 = s0 * static_cast<float>(128u + (zz1 & 0xFFu));
+      const float sz1 = s1 * static_cast<float>(128u + ((zz1 >> 8) & 0xFFu));
       const float2 sx = *reinterpret_cast<const float2 *>(sxg + G * 8 + 2 * t);
       acc[0] = fmaf(-sz0, sx.x, fmaf(s0, d[0], acc[0]));
       acc[1] = fmaf(-sz0, sx.y, fmaf(s0, d[1], acc[1]));
       acc[2] = fmaf(-sz1, sx.x, fmaf(s1, d[2], acc[2]));
       acc[3] = fmaf(-sz1, sx.y, fmaf(s1, d[3], acc[3]));
-      if (++G == g0 + gps) {
-        // this warp's slice of the row block is done: meet the other slices, slice 0 writes
-        float *mine = red + ((unit & 1) * kGemvWarps + warp) * 128 + lane * 4;
-        if (ks > 1) {
-          *reinterpret_cast<float4 *>(mine) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-          asm volatile("bar.sync %0, %1;" ::"r"(1 + warp / ks), "r"(32 * ks) : "memory");
-        }
-        if (slice == 0) {
-          float v[4] = {acc[0], acc[1], acc[2], acc[3]};
-          for (int j = 1; j < ks; ++j) {
-            const float4 o = *reinterpret_cast<const float4 *>(mine + j * 128);
-            v[0] += o.x;
-            v[1] += o.y;
-            v[2] += o.z;
-            v[3] += o.w;
-          }
-          // rows 16 rb + g (v 0, 1) and + 8 (v 2, 3); tokens 2 t, 2 t + 1
-          const int r0 = 16 * rb + g, r1 = r0 + 8, m0 = 2 * t, m1 = m0 + 1;
-          const float b0 = (bias && r0 < N) ? bias[r0] : 0.0f, b1 = (bias && r1 < N) ? bias[r1] : 0.0f;
-          auto put = [&](int m, int r, float x) {
-            if (m < M && r < N) Y[static_cast<size_t>(m) * N + r] = static_cast<uint16_t>(pack_bf16x2(x, 0.0f) & 0xFFFFu);
-          };
-          put(m0, r0, v[0] + b0);
-          put(m1, r0, v[1] + b0);
-          put(m0, r1, v[2] + b1);
-          put(m1, r1, v[3] + b1);
-        }
-        acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
-        G = g0;
-        rb += stride;
-        ++unit;
-      }
     }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(bar_empty + 8 * s);  // also after a failed wait: the producer's waits stay bounded
+    if (j == runs_per_rb - 1) {
+      // the row block is done: the warps' sums meet, warp 0 adds them in warp order and writes Y
+      *reinterpret_cast<float4 *>(red + (warp * 32 + lane) * 4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      named_bar_sync(1, nct);
+      if (warp == 0) {
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int w = 0; w < kCW; ++w) {
+          const float4 o = *reinterpret_cast<const float4 *>(red + (w * 32 + lane) * 4);
+          v[0] += o.x;
+          v[1] += o.y;
+          v[2] += o.z;
+          v[3] += o.w;
+        }
+        // rows 16 rb + g (v 0, 1) and + 8 (v 2, 3); tokens 2 t, 2 t + 1
+        const int rb = static_cast<int>(blockIdx.x) + (c / runs_per_rb) * static_cast<int>(gridDim.x);
+        const int r0 = 16 * rb + g, r1 = r0 + 8, m0 = 2 * t, m1 = m0 + 1;
+        const float b0 = (bias && r0 < N) ? bias[r0] : 0.0f, b1 = (bias && r1 < N) ? bias[r1] : 0.0f;
+        auto put = [&](int m, int r, float x) {
+          if (ok && m < M && r < N) Y[static_cast<size_t>(m) * N + r] = static_cast<uint16_t>(pack_bf16x2(x, 0.0f) & 0xFFFFu);
+        };
+        put(m0, r0, v[0] + b0);
+        put(m1, r0, v[1] + b0);
+        put(m0, r1, v[2] + b1);
+        put(m1, r1, v[3] + b1);
+      }
+      named_bar_sync(1, nct);  // red is free again
+      acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+    }
+  }
+  // After a wait that gave up, the CTA still must not exit with bulk copies in flight into its
+  // shared memory: wait (bounded) for the slots' last phases.
+  if (!ok && warp == 0) {
+    for (int c = runs > nslots ? runs - nslots : 0; c < runs; ++c)
+      mbar_wait(bar_full + 8 * (c % nslots), (c / nslots) & 1, nullptr, KID_AWQ, 3);
   }
 }
 
 }  // namespace
 
 size_t awq_smem_bytes(int M, int K);
+int awq_slots(int K);
 
 namespace {
 
-// Warps per row block: enough (ks = K/64 / groups per warp) that a grid of resident blocks has
-// row blocks x ks warps of work, with ks dividing the groups of a row.
-int pick_ks(int gpr, int row_blocks, int slots) {
-  int ks = 1;
-  while (ks < kGemvWarps && gpr % (2 * ks) == 0 && static_cast<long>(row_blocks) * ks < static_cast<long>(slots) * kGemvWarps * 2)
-    ks *= 2;
-  return ks;
-}
-
-cudaError_t launch_gemv_mma(const uint16_t *X, int M, const uint8_t *wt, const uint8_t *szt, const float *bias, int N,
-                            int K, uint16_t *Y, cudaStream_t st) {
+cudaError_t launch_gemv_stream(const uint16_t *X, int M, const uint8_t *wt, const uint8_t *szt, const float *bias,
+                               int N, int K, uint16_t *Y, uint32_t *err, cudaStream_t st) {
   const size_t smem = awq_smem_bytes(M, K);
+  const int nslots = awq_slots(K);
   static int attr_done[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(awq_gemv_mma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+    cudaError_t e =
+        cudaFuncSetAttribute(awq_gemv_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
   int per_sm = 0, sms = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, awq_gemv_mma_kernel, kGemvWarps * 32, smem) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, awq_gemv_stream_kernel, (kCW + 1) * 32, smem) !=
           cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || per_sm <= 0)
     return cudaErrorLaunchOutOfResources;
-  const int slots = per_sm * sms;  // persistent grid: the blocks resident at once
   const int row_blocks = (N + 15) / 16;
-  const int ks = pick_ks(K / kAwqGroup, row_blocks, slots);
-  const int need = (row_blocks * ks + kGemvWarps - 1) / kGemvWarps;
-  const int blocks = need < slots ? need : slots;
-  awq_gemv_mma_kernel<<<blocks, kGemvWarps * 32, smem, st>>>(X, M, wt, szt, bias, N, K, ks, Y);
+  const int slots = per_sm * sms;
+  const int blocks = row_blocks < slots ? row_blocks : slots;
+  awq_gemv_stream_kernel<<<blocks, (kCW + 1) * 32, smem, st>>>(X, M, wt, szt, bias, N, K, nslots, Y, err);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 int awq_max_tokens() { return 8; }
-// staged activations (K/64 groups x 1 KiB of bf16 pairs), group sums (8 tokens) and the slices'
-// partial sums (2 x 8 warps x 512 bytes); the same for every token count up to 8
+// Shared memory of the GEMV: staged activations (K/64 groups x 1 KiB of bf16 pairs), group sums (8
+// tokens x 4 bytes per group), the warps' partial sums, the ring of weight runs (as many slots as
+// fit, 12 at most, at least 2) and its barriers. The same for every token count up to 8.
+constexpr size_t kSmemLimit = 227 * 1024;
+size_t awq_fixed_smem(int K) { return static_cast<size_t>(K / kAwqGroup) * (1024 + 32) + kRedBytes; }
+int awq_slots(int K) {
+  const size_t fixed = awq_fixed_smem(K);
+  if (fixed >= kSmemLimit) return 0;
+  size_t n = (kSmemLimit - fixed) / (kSlotBytes + 16);
+  return static_cast<int>(n > static_cast<size_t>(kMaxSlots) ? kMaxSlots : n);
+}
+constexpr int kMaxK = 12288;  // the documented limit (at least two slots fit up to it)
 size_t awq_smem_bytes(int, int K) {
-  return static_cast<size_t>(K / kAwqGroup) * (1024 + 32) + 2 * kGemvWarps * 512;
+  const int n = awq_slots(K);
+  if (n < 2 || K > kMaxK) return kSmemLimit + 1;  // too large: the caller rejects the shape
+  return awq_fixed_smem(K) + static_cast<size_t>(n) * (kSlotBytes + 16);
 }
 size_t awq_packed_weight_bytes(int N, int K) { return static_cast<size_t>((N + 15) / 16) * 16 * (K / 2); }
 size_t awq_packed_sz_bytes(int N, int K) { return static_cast<size_t>((N + 15) / 16) * (K / kAwqGroup) * 64; }
@@ -350,8 +374,8 @@ cudaError_t launch_awq_pack(const uint8_t *wq, const uint16_t *scales, const uin
 }
 
 cudaError_t launch_awq_gemv(const uint16_t *X, int M, const uint8_t *wt, const uint8_t *szt, const float *bias, int N,
-                            int K, uint16_t *Y, cudaStream_t st) {
-  return launch_gemv_mma(X, M, wt, szt, bias, N, K, Y, st);
+                            int K, uint16_t *Y, uint32_t *err, cudaStream_t st) {
+  return launch_gemv_stream(X, M, wt, szt, bias, N, K, Y, err, st);
 }
 
 }  // namespace svdq

@@ -13,7 +13,7 @@ namespace svdq {
 // ---------------------------------------------------------------- error word
 // A kernel that gives up on a bounded wait records (kernel << 16) | (site << 8) | 1 into the
 // library's device error word (first error wins) and leaves its loops.
-enum KernelId : uint32_t { KID_QUANT = 1, KID_GEMM = 2, KID_PREP = 3, KID_BASE = 4, KID_SELFTEST = 5 };
+enum KernelId : uint32_t { KID_QUANT = 1, KID_GEMM = 2, KID_PREP = 3, KID_BASE = 4, KID_SELFTEST = 5, KID_AWQ = 6 };
 
 // About two seconds of %globaltimer (ns) before a wait is declared lost.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;

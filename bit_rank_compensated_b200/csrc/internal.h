@@ -87,7 +87,7 @@ cudaError_t launch_awq_quantize(const float *W, int N, int K, uint8_t *wq, uint1
 cudaError_t launch_awq_pack(const uint8_t *wq, const uint16_t *scales, const uint8_t *zeros, int N, int K, uint8_t *wt,
                             uint8_t *szt, cudaStream_t st);
 cudaError_t launch_awq_gemv(const uint16_t *X, int M, const uint8_t *wt, const uint8_t *szt, const float *bias, int N,
-                            int K, uint16_t *Y, cudaStream_t st);
+                            int K, uint16_t *Y, uint32_t *err, cudaStream_t st);
 
 // Failure-path self-test (selftest.cu): bounded waits on an mbarrier nobody signals.
 cudaError_t launch_selftest_wait(uint32_t *err, uint64_t limit_ns, cudaStream_t st);

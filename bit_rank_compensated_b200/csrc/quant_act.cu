@@ -301,6 +301,12 @@ __global__ void __launch_bounds__(QCfg<RANK, QUANT>::THREADS, 1)
     // the slots in rank order (deterministic) once its own writes and the remote bytes are in.
     // The stage memory of every CTA must be idle first: a split cluster barrier, arrived at as
     // soon as this CTA's quantizer warps and MMAs are done with it.
+    // Failure path: if the wait for the peers' bytes (bar_recv) gives up after its time limit (a
+    // peer CTA stalled), the owner records the error and exits without a final cluster barrier
+    // (a barrier.cluster wait cannot be bounded); a peer that resumes later could then still store
+    // into the exited CTA's shared memory. The recorded error marks every output of the launch as
+    // invalid (svdq_last_device_error); on the normal path every byte has landed before the owner
+    // reads the slots, so no store is in flight when a CTA exits.
     constexpr uint32_t RS = C::RED_STRIDE;
     const uint32_t slot_bytes = static_cast<uint32_t>(rows_per) * RS * 4u;
     uint8_t *red = smem + C::RED_OFF;

@@ -192,6 +192,17 @@ def test_mlp_pair_shapes_are_checked_before_the_device(lib, unsupported):
     assert lib.svdq_mlp_workspace_bytes(64, 512, 128) == 0
 
 
+def test_awq_gemv_size_limits(lib, unsupported):
+    # K up to 12288 (staged activations beside a ring of at least two weight runs), 1..8 tokens
+    P = _p
+    call = lambda M, K: lib.svdq_awq_gemv_w4a16(P(DEV), M, P(DEV), P(DEV), None, 64, K, P(DEV), None)  # noqa: E731
+    assert call(1, 12288) == UNSUPPORTED
+    assert call(8, 3072) == UNSUPPORTED
+    assert call(1, 12352) == INVALID
+    assert call(9, 3072) == INVALID
+    assert call(0, 3072) == INVALID
+
+
 def test_null_layer_is_rejected(lib, unsupported):
     assert lib.svdq_quant_act_lora_down(_p(DEV), 16, None, _p(DEV), _p(DEV), _p(DEV), None) == INVALID
     assert lib.svdq_gemm_w4a4_lora_up(_p(DEV), _p(DEV), _p(DEV), 16, None, _p(DEV), None) == INVALID
