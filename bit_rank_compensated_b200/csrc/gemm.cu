@@ -244,7 +244,7 @@ constexpr uint32_t SF_GROUP_WARPS = 4;
 constexpr uint32_t EPI_WARPS = 8;
 constexpr uint32_t FULL_COUNT = 1 + 2 * SF_GROUP_WARPS;
 constexpr uint32_t ACCEMPTY_COUNT = 2 * EPI_WARPS;
-constexpr int N_BARS = 4 * STAGES + 2 + 3;  // + rope_full, rope_empty (QKNR) or hbox_full, hbox_empty, l1d_full (MLP)
+constexpr int N_BARS = 4 * STAGES + 2 + 4;  // + rope_full, rope_empty (QKNR) or hfull, hempty, l1dfull, l1dfree (MLP)
 static_assert(STAGE_BYTES % 1024 == 0, "stages keep the 1 KiB alignment of 128B-swizzled tiles");
 static_assert(SF_COL0 + STAGES * SF_COLS <= TMEM_COLS, "scale slots exceed the tensor memory");
 static_assert(SMEM_QKNR <= 232448, "shared memory per CTA");
@@ -351,9 +351,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   // MLP: hfull (even CTA: both CTAs' eight output warps wrote the pass's hi / lo rows), hempty (the
   // pass's down-projection MMAs are done; both CTAs), l1dfull (even CTA: the tile's L1s boxes landed
   // in both CTAs)
+  // l1dfree (both CTAs: the MMAs that read the tile's L1s boxes are done; one phase per tile, so
+  // the odd CTA's loader, which runs ahead of the passes, never waits on a phase two behind)
   const uint32_t bar_hfull = bar_sf + 8 * 2 * STAGES;
   const uint32_t bar_hempty = bar_hfull + 8;
   const uint32_t bar_l1dfull = bar_hempty + 8;
+  const uint32_t bar_l1dfree = bar_l1dfull + 8;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(bars + N_BARS);
 
   const int warp = threadIdx.x >> 5;
@@ -385,6 +388,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(bar_hfull, 2 * EPI_WARPS);
       mbar_init(bar_hempty, 1);
       mbar_init(bar_l1dfull, 1);
+      mbar_init(bar_l1dfree, 1);
     }
     fence_mbar_init();
   }
@@ -918,7 +922,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       // ------------------------------------------------------------ down-projection (MLP)
       // Per tile: both CTAs load their half of the down layer's L1s for the tile's 256 columns
       // (eight boxes of 32 columns x rank_d / 2 rows, 64B swizzle; counted on the even CTA's
-      // l1dfull), once the MMAs that read the previous tile's boxes are done. In the even CTA the
+      // l1dfull), once the MMAs that read the previous tile's boxes are done (l1dfree, committed
+      // after each tile's fourth pass; a wait on hempty, four phases a tile, could return early in
+      // the odd CTA, whose loader runs ahead: tests/test_mlp_down_protocol.py models both). In the even CTA the
       // warp then issues, per pass of 32 columns, the pair MMAs  D += hi L1s + lo L1s  (M = 256 across
       // the pair, N = rank_d, K = 16 each; both halves' boxes) and commits them to hempty in both
       // CTAs. D sits in columns LA_COL0.. of tensor memory; the first MMA of a tile starts it afresh.
@@ -936,7 +942,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int t = pid; t < tiles && ok; t += npairs, ++tcount) {
           const int nt = t / a.Mt;
           if (tcount > 0) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar_hempty, (4 * tcount - 1) & 1, a.err, KID_GEMM, 14));
+            ok = __all_sync(0xffffffffu, mbar_wait(bar_l1dfree, (tcount - 1) & 1, a.err, KID_GEMM, 14));
             if (!ok) break;
           }
           if (elect_one()) {
@@ -967,12 +973,13 @@ __global__ void __launch_bounds__(THREADS, 1)
                 }
               }
               tc_commit_pair_mc(bar_hempty, 0x3);
+              if (p == 3) tc_commit_pair_mc(bar_l1dfree, 0x3);
             }
             __syncwarp();
           }
         }
         // the last commit has arrived (in this CTA) before the CTA can exit
-        if (ok && tcount > 0) mbar_wait(bar_hempty, (4 * tcount - 1) & 1, a.err, KID_GEMM, 17);
+        if (ok && tcount > 0) mbar_wait(bar_l1dfree, (tcount - 1) & 1, a.err, KID_GEMM, 17);
       }
     } else if ((warp >= 2 && warp < EPI_WARP0) || warp == 16 || warp == 17) {
       // ------------------------------------------------------------ scale-factor writers
