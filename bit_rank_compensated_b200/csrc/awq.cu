@@ -123,95 +123,95 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Streaming tensor-core GEMV. The work is bound by reading the 4-bit weights once, so it is
-// organised around keeping enough bytes in flight: one warp per CTA streams the CTA's tiles with
-// bulk copies (cp.async.bulk) into a ring of shared-memory slots, each slot a run of up to 16
-// consecutive groups of one row block (16 x 512 bytes of codes, 16 x 64 bytes of scales and zero
-// points, contiguous in the packed layout), up to 12 slots (108 KiB) ahead; no registers are held
-// per tile in flight.
-// The 16 consumer warps take one group each of every run (warp w: group 16 j + w of run j of the
-// row block): an m16n8k16 bf16 MMA per k-step with the 16 weight rows of the row block as operand
-// A (each code q turned into the exact bf16 integer 128 + q, one LOP3 per pair) and up to 8 tokens
-// as operand B (the bf16 activations, staged once per CTA in fragment order); the products are
-// exact and summed in fp32, and the scale and zero point enter once per group:
-// acc += s D_G - s (128 + z) sum_G(x). At the end of a row block the 16 warps' sums meet in shared
-// memory and warp 0 adds them in warp order (deterministic) and writes Y. Row blocks are dealt to
-// the CTAs round-robin (persistent grid, one CTA per SM at the benchmarked shapes).
-constexpr int kCW = 16;                               // consumer warps
-constexpr int kRunG = 16;                             // groups per run (slot)
-constexpr uint32_t kSlotBytes = kRunG * (512 + 64);   // 9 KiB
-constexpr int kMaxSlots = 12;
-constexpr uint32_t kRedBytes = kCW * 32 * 4 * 4;      // the warps' partial sums of a row block
+// Tensor-core GEMV, bound by reading the 4-bit weights once. What keeps it at the memory's
+// rate is the number of bytes in flight per SM: every lane streams its own share of the tiles
+// into shared memory with cp.async (16 bytes of codes per lane per tile, plus the tile's 64 bytes
+// of scales and zero points from four lanes), up to 16 tiles ahead per warp, with no register held
+// per tile in flight (one CTA of 16 warps per SM: ~147 KiB in flight). Each lane's 16 bytes of a
+// tile are exactly its operand-A registers, so a warp only waits for its own copies.
+// Per tile: an m16n8k16 bf16 MMA per k-step with the 16 weight rows of the row block as operand A
+// (each code q turned into the exact bf16 integer 128 + q in registers, one LOP3 per pair) and up
+// to 8 tokens as operand B (the bf16 activations, staged once per CTA in fragment order); the
+// products are exact and summed in fp32, and the scale and zero point are applied per group:
+// acc += s D_G - s (128 + z) sum_G(x). (Summing 128 + q instead of q costs about 2^-23 x 143 / 8 of
+// the group's sum in rounding, ~2e-5 relative.)
+// Work: ks consecutive warps of a CTA (ks = 1, 2, 4 or 8) share a row block, warp slice
+// j = warp % ks taking groups j gps .. (j + 1) gps - 1 (gps = K/64 / ks); the slices' partial sums
+// meet in shared memory (double-buffered by unit parity, one named barrier per unit) and slice 0
+// adds them in slice order and writes Y. The grid is persistent: a warp group takes row blocks
+// rb0, rb0 + stride, ... and each warp streams its tiles in order, across row blocks.
+constexpr int kMaxWarps = 16;
+constexpr uint32_t kTileSlot = 576; // 512 bytes of codes + 64 of scales and zero points
 
-__global__ void __launch_bounds__((kCW + 1) * 32, 1)
-    awq_gemv_stream_kernel(const uint16_t *X, int M, const uint8_t *wt, const uint8_t *szt, const float *bias, int N,
-                           int K, int nslots, uint16_t *Y, uint32_t *err) {
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+template <int DEPTH>
+__global__ void __launch_bounds__(kMaxWarps * 32) awq_gemv_mma_kernel(const uint16_t *X, int M, const uint8_t *wt,
+                                                                      const uint8_t *szt, const float *bias, int N,
+                                                                      int K, int ks, uint16_t *Y) {
   extern __shared__ __align__(16) uint32_t smem_w[];
+  const int nwarps = blockDim.x >> 5;
   const int gpr = K / kAwqGroup;
   uint32_t *xb = smem_w;                                       // gpr x 32 lanes x 8 words (bf16 pairs)
   float *sxg = reinterpret_cast<float *>(smem_w + gpr * 256);  // gpr x 8 tokens
-  float *red = sxg + gpr * 8;                                  // kCW warps x 32 lanes x 4 partial sums
-  uint8_t *ring = reinterpret_cast<uint8_t *>(red) + kRedBytes;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(ring + static_cast<size_t>(nslots) * kSlotBytes);
-  const uint32_t bar_full = smem_u32(bars), bar_empty = bar_full + 8 * nslots;
+  float *red = sxg + gpr * 8;                                  // 2 x nwarps x 32 lanes x 4 partial sums
+  uint8_t *rings = reinterpret_cast<uint8_t *>(red + 2 * nwarps * 128);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int row_blocks = (N + 15) / 16;
-  const int runs_per_rb = (gpr + kRunG - 1) / kRunG;
-  const int my_rbs = blockIdx.x < row_blocks ? (row_blocks - 1 - static_cast<int>(blockIdx.x)) / gridDim.x + 1 : 0;
-  const int runs = my_rbs * runs_per_rb;
+  const int slice = warp % ks, gps = gpr / ks, g0 = slice * gps;
+  const int stride = gridDim.x * (nwarps / ks);  // row blocks per round of the grid
+  const int rb0 = blockIdx.x * (nwarps / ks) + warp / ks;
+  const int units = rb0 < row_blocks ? (row_blocks - 1 - rb0) / stride + 1 : 0;
+  const int items = units * gps;
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < nslots; ++i) {
-      mbar_init(bar_full + 8 * i, 1);
-      mbar_init(bar_empty + 8 * i, kCW);
-    }
-    fence_mbar_init();
-  }
-  __syncthreads();
-
-  if (warp == kCW) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      for (int c = 0; c < runs; ++c) {
-        const int s = c % nslots;
-        if (c >= nslots && !mbar_wait(bar_empty + 8 * s, ((c / nslots) - 1) & 1, err, KID_AWQ, 1)) break;
-        const int rb = static_cast<int>(blockIdx.x) + (c / runs_per_rb) * static_cast<int>(gridDim.x);
-        const int G0 = (c % runs_per_rb) * kRunG;
-        const int ng = min(kRunG, gpr - G0);
-        const size_t tile0 = static_cast<size_t>(rb) * gpr + G0;
-        const uint32_t dst = smem_u32(ring + static_cast<size_t>(s) * kSlotBytes);
-        mbar_arrive_expect_tx(bar_full + 8 * s, static_cast<uint32_t>(ng) * (512u + 64u));
-        bulk_load(dst, wt + tile0 * 512, static_cast<uint32_t>(ng) * 512u, bar_full + 8 * s);
-        bulk_load(dst + kRunG * 512u, szt + tile0 * 64, static_cast<uint32_t>(ng) * 64u, bar_full + 8 * s);
+  // this warp's ring: tile (row block rb0 + i / gps stride, group g0 + i % gps) goes to slot i % DEPTH
+  const uint32_t ring = smem_u32(rings) + static_cast<uint32_t>(warp) * DEPTH * kTileSlot;
+  uint32_t pf_tile = static_cast<uint32_t>(rb0) * gpr + g0;  // tiles fit 32 bits (N K / 1024 < 2^32)
+  const uint32_t wrap = static_cast<uint32_t>(stride) * gpr - gps;
+  int pf_G = 0, pf_i = 0;
+  auto issue = [&](int slot) {
+    if (pf_i < items) {
+      const uint32_t dst = ring + static_cast<uint32_t>(slot) * kTileSlot;
+      cp_async16(dst + lane * 16, wt + static_cast<size_t>(pf_tile) * 512 + lane * 16);
+      if (lane < 4) cp_async16(dst + 512 + lane * 16, szt + static_cast<size_t>(pf_tile) * 64 + lane * 16);
+      ++pf_tile;
+      if (++pf_G == gps) {
+        pf_G = 0;
+        pf_tile += wrap;
       }
+      ++pf_i;
     }
-    return;
-  }
+    cp_async_commit();  // one group per tile (empty past the end), so wait_group counts tiles
+  };
+#pragma unroll
+  for (int p = 0; p < DEPTH; ++p) issue(p);
 
-  // ------------------------------------------------------------ consumers (512 threads)
   // Stage X in fragment order: pair w (k = 2 w) of token m goes to word (G 32 + 4 m + t) 8 + 2 s + u
-  // with k = 64 G + 16 s + 8 u + 2 t. Consecutive threads read consecutive pairs of the M real
-  // tokens (coalesced); the slots of tokens M .. 7 are zero.
-  const int ct = threadIdx.x, nct = kCW * 32;
+  // with k = 64 G + 16 s + 8 u + 2 t. Every thread reads consecutive pairs of the M real tokens
+  // (coalesced). Lane L's operand-B registers belong to token L / 4, so the lanes of tokens M .. 7
+  // take zeros in registers and their slots are never written or read.
   const int kw = K / 2;
   auto xb_index = [&](int m, int w) {
     const int e = (2 * w) & 63;
     return (((2 * w) >> 6) * 32 + 4 * m + ((e & 7) >> 1)) * 8 + 2 * (e >> 4) + ((e >> 3) & 1);
   };
-  for (int m = 0; m < 8; ++m) {
-    if (m < M) {
+  for (int m = 0; m < M; ++m) {
 #pragma unroll 4
-      for (int w = ct; w < kw; w += nct)
-        xb[xb_index(m, w)] = __ldg(reinterpret_cast<const uint32_t *>(X + static_cast<size_t>(m) * K) + w);
-    } else {
-      for (int w = ct; w < kw; w += nct) xb[xb_index(m, w)] = 0u;
-    }
+    for (int w = threadIdx.x; w < kw; w += blockDim.x)
+      xb[xb_index(m, w)] = __ldg(reinterpret_cast<const uint32_t *>(X + static_cast<size_t>(m) * K) + w);
   }
-  named_bar_sync(1, nct);
+  __syncthreads();
   // sums of x over each group, per token, from the staged pairs (lanes 4 m .. 4 m + 3, all words)
-  for (int i = ct; i < gpr * 8; i += nct) {
-    const int G = i >> 3, m = i & 7;
+  for (int i = threadIdx.x; i < gpr * 8; i += blockDim.x) {
+    const int G = i >> 3, m = i & 7;  // tokens M .. 7: zero sums
     float sum = 0.0f;
     if (m < M) {
       const uint4 *w4 = reinterpret_cast<const uint4 *>(xb + (G * 32 + 4 * m) * 8);
@@ -225,135 +225,169 @@ __global__ void __launch_bounds__((kCW + 1) * 32, 1)
     }
     sxg[i] = sum;
   }
-  named_bar_sync(1, nct);
+  __syncthreads();
 
   float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  bool ok = true;
-  for (int c = 0; c < runs; ++c) {
-    const int s = c % nslots;
-    const int j = c % runs_per_rb;
-    const int G = j * kRunG + warp;
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait_parked(bar_full + 8 * s, (c / nslots) & 1, err, KID_AWQ, 2));
-    if (ok && G < gpr) {
-      const uint8_t *slot = ring + static_cast<size_t>(s) * kSlotBytes;
-      const uint4 cq = ld_shared_u32x4(smem_u32(slot + warp * 512 + lane * 16));
-      const uint32_t zz0 = ld_shared_u32(smem_u32(slot + kRunG * 512 + warp * 64 + g * 8));
-      const uint32_t zz1 = ld_shared_u32(smem_u32(slot + kRunG * 512 + warp * 64 + g * 8 + 4));
-      const uint4 xa = *reinterpret_cast<const uint4 *>(xb + (G * 32 + lane) * 8);
-      const uint4 xc = *reinterpret_cast<const uint4 *>(xb + (G * 32 + lane) * 8 + 4);
-      const uint32_t bx[8] = {xa.x, xa.y, xa.z, xa.w, xc.x, xc.y, xc.z, xc.w};
-      const uint32_t cw[4] = {cq.x, cq.y, cq.z, cq.w};
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int st = 0; st < 4; ++st) {
-        uint32_t a[4];
-        // (128 + q_lo, 128 + q_hi) as a bf16 pair (exact): the 128 joins the zero point below
-#pragma unroll
-        for (int r = 0; r < 4; ++r) a[r] = ((cw[st] >> (4 * r)) & 0x000F000Fu) | 0x43004300u;
-        mma_bf16_16816(d, a, bx[2 * st], bx[2 * st + 1]);
-      }
-      const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(zz0 & 0xFFFFu)));
-      const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(zz0 >> 16)));
-      // D = sum (128 + q) x, so acc += s D - s (128 + z) sum x (s (128 + z) is exact in fp32)
-      const float sz0 = s0 * static_cast<float>(128u + (zz1 & 0xFFu));
-      const float sz1 = s1 * static_cast<float>(128u + ((zz1 >> 8) & 0xFFu));
-      const float2 sx = *reinterpret_cast<const float2 *>(sxg + G * 8 + 2 * t);
-      acc[0] = fmaf(-sz0, sx.x, fmaf(s0, d[0], acc[0]));
-      acc[1] = fmaf(-sz0, sx.y, fmaf(s0, d[1], acc[1]));
-      acc[2] = fmaf(-sz1, sx.x, fmaf(s1, d[2], acc[2]));
-      acc[3] = fmaf(-sz1, sx.y, fmaf(s1, d[3], acc[3]));
-    }
+  int rb = rb0, G = g0, unit = 0;
+  for (int i = 0; i < items; ++i) {
+    const int slot = i % DEPTH;
+    // this lane's copies of tile i are complete (one group per tile, DEPTH - 1 younger ones may
+    // still be in flight); the warp then sees every lane's (the scale bytes come from lanes 0..3)
+    cp_async_wait<DEPTH - 1>();
     __syncwarp();
-    if (lane == 0) mbar_arrive(bar_empty + 8 * s);  // also after a failed wait: the producer's waits stay bounded
-    if (j == runs_per_rb - 1) {
-      // the row block is done: the warps' sums meet, warp 0 adds them in warp order and writes Y
-      *reinterpret_cast<float4 *>(red + (warp * 32 + lane) * 4) = make_float4(acc[0], acc[1], acc[2], acc[3]);
-      named_bar_sync(1, nct);
-      if (warp == 0) {
-        float v[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int w = 0; w < kCW; ++w) {
-          const float4 o = *reinterpret_cast<const float4 *>(red + (w * 32 + lane) * 4);
+    const uint32_t sl = ring + static_cast<uint32_t>(slot) * kTileSlot;
+    const uint4 c = ld_shared_u32x4(sl + lane * 16);
+    const uint32_t zz0 = ld_shared_u32(sl + 512 + g * 8);
+    const uint32_t zz1 = ld_shared_u32(sl + 512 + g * 8 + 4);
+    __syncwarp();  // every lane has read the slot before it is refilled
+    issue(slot);   // the tile DEPTH ahead
+    uint4 xa = make_uint4(0u, 0u, 0u, 0u), xc = xa;
+    if (g < M) {
+      xa = *reinterpret_cast<const uint4 *>(xb + (G * 32 + lane) * 8);
+      xc = *reinterpret_cast<const uint4 *>(xb + (G * 32 + lane) * 8 + 4);
+    }
+    const uint32_t bx[8] = {xa.x, xa.y, xa.z, xa.w, xc.x, xc.y, xc.z, xc.w};
+    const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int st = 0; st < 4; ++st) {
+      uint32_t a[4];
+      // (128 + q_lo, 128 + q_hi) as a bf16 pair (exact): the 128 joins the zero point below
+#pragma unroll
+      for (int r = 0; r < 4; ++r) a[r] = ((cw[st] >> (4 * r)) & 0x000F000Fu) | 0x43004300u;
+      mma_bf16_16816(d, a, bx[2 * st], bx[2 * st + 1]);
+    }
+    const float s0 = __half2float(__ushort_as_half(static_cast<uint16_t>(zz0 & 0xFFFFu)));
+    const float s1 = __half2float(__ushort_as_half(static_cast<uint16_t>(zz0 >> 16)));
+    // D = sum (128 + q) x, so acc += s D - s (128 + z) sum x (s (128 + z) is exact in fp32)
+    const float sz0 = s0 * static_cast<float>(128u + (zz1 & 0xFFu));
+    const float sz1 = s1 * static_cast<float>(128u + ((zz1 >> 8) & 0xFFu));
+    const float2 sx = *reinterpret_cast<const float2 *>(sxg + G * 8 + 2 * t);
+    acc[0] = fmaf(-sz0, sx.x, fmaf(s0, d[0], acc[0]));
+    acc[1] = fmaf(-sz0, sx.y, fmaf(s0, d[1], acc[1]));
+    acc[2] = fmaf(-sz1, sx.x, fmaf(s1, d[2], acc[2]));
+    acc[3] = fmaf(-sz1, sx.y, fmaf(s1, d[3], acc[3]));
+    if (++G == g0 + gps) {
+      // this warp's slice of the row block is done: meet the other slices, slice 0 writes
+      float *mine = red + ((unit & 1) * nwarps + warp) * 128 + lane * 4;
+      if (ks > 1) {
+        *reinterpret_cast<float4 *>(mine) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+        asm volatile("bar.sync %0, %1;" ::"r"(1 + warp / ks), "r"(32 * ks) : "memory");
+      }
+      if (slice == 0) {
+        float v[4] = {acc[0], acc[1], acc[2], acc[3]};
+        for (int j = 1; j < ks; ++j) {
+          const float4 o = *reinterpret_cast<const float4 *>(mine + j * 128);
           v[0] += o.x;
           v[1] += o.y;
           v[2] += o.z;
           v[3] += o.w;
         }
         // rows 16 rb + g (v 0, 1) and + 8 (v 2, 3); tokens 2 t, 2 t + 1
-        const int rb = static_cast<int>(blockIdx.x) + (c / runs_per_rb) * static_cast<int>(gridDim.x);
         const int r0 = 16 * rb + g, r1 = r0 + 8, m0 = 2 * t, m1 = m0 + 1;
         const float b0 = (bias && r0 < N) ? bias[r0] : 0.0f, b1 = (bias && r1 < N) ? bias[r1] : 0.0f;
         auto put = [&](int m, int r, float x) {
-          if (ok && m < M && r < N) Y[static_cast<size_t>(m) * N + r] = static_cast<uint16_t>(pack_bf16x2(x, 0.0f) & 0xFFFFu);
+          if (m < M && r < N) Y[static_cast<size_t>(m) * N + r] = static_cast<uint16_t>(pack_bf16x2(x, 0.0f) & 0xFFFFu);
         };
         put(m0, r0, v[0] + b0);
         put(m1, r0, v[1] + b0);
         put(m0, r1, v[2] + b1);
         put(m1, r1, v[3] + b1);
       }
-      named_bar_sync(1, nct);  // red is free again
       acc[0] = acc[1] = acc[2] = acc[3] = 0.0f;
+      G = g0;
+      rb += stride;
+      ++unit;
     }
   }
-  // After a wait that gave up, the CTA still must not exit with bulk copies in flight into its
-  // shared memory: wait (bounded) for the slots' last phases.
-  if (!ok && warp == 0) {
-    for (int c = runs > nslots ? runs - nslots : 0; c < runs; ++c)
-      mbar_wait(bar_full + 8 * (c % nslots), (c / nslots) & 1, nullptr, KID_AWQ, 3);
-  }
+  cp_async_wait<0>();  // no copy in flight when the CTA exits
 }
 
 }  // namespace
 
-size_t awq_smem_bytes(int M, int K);
-int awq_slots(int K);
+// Launch shape of the GEMV for K: warps per CTA (16, or 8 where 16 warps' rings do not fit beside
+// the staged activations) and tiles in flight per warp (DEPTH: 16, 8, 4 or 2); 0 when K is too
+// large for two tiles per warp.
+constexpr size_t kSmemLimit = 227 * 1024;
+size_t awq_fixed_smem(int K, int warps) {
+  return static_cast<size_t>(K / kAwqGroup) * (1024 + 32) + 2u * warps * 512u;
+}
+void awq_shape(int K, int *warps, int *depth) {
+  *warps = 0;
+  *depth = 0;
+  for (int w : {16, 8}) {
+    for (int d : {16, 8, 4, 2}) {
+      if (awq_fixed_smem(K, w) + static_cast<size_t>(w) * d * kTileSlot <= kSmemLimit) {
+        *warps = w;
+        *depth = d;
+        return;
+      }
+    }
+  }
+}
+constexpr int kMaxK = 12288;  // the documented limit (8 warps with 4 tiles in flight each fit up to it)
+size_t awq_smem_bytes(int, int K) {
+  int w, d;
+  awq_shape(K, &w, &d);
+  if (w == 0 || K > kMaxK) return kSmemLimit + 1;  // too large: the caller rejects the shape
+  return awq_fixed_smem(K, w) + static_cast<size_t>(w) * d * kTileSlot;
+}
 
 namespace {
 
-cudaError_t launch_gemv_stream(const uint16_t *X, int M, const uint8_t *wt, const uint8_t *szt, const float *bias,
-                               int N, int K, uint16_t *Y, uint32_t *err, cudaStream_t st) {
+// Warps per row block: enough (ks = K/64 / groups per warp) that a grid of resident blocks has
+// row blocks x ks warps of work, with ks dividing the groups of a row.
+int pick_ks(int gpr, int row_blocks, int slots, int warps) {
+  int ks = 1;
+  while (ks < warps && ks < 8 && gpr % (2 * ks) == 0 &&
+         static_cast<long>(row_blocks) * ks < static_cast<long>(slots) * warps * 2)
+    ks *= 2;
+  return ks;
+}
+
+template <int DEPTH>
+cudaError_t launch_gemv_depth(const uint16_t *X, int M, const uint8_t *wt, const uint8_t *szt, const float *bias,
+                              int N, int K, uint16_t *Y, int warps, cudaStream_t st) {
   const size_t smem = awq_smem_bytes(M, K);
-  const int nslots = awq_slots(K);
   static int attr_done[64] = {0};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_done[dev]) {
     cudaError_t e =
-        cudaFuncSetAttribute(awq_gemv_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
+        cudaFuncSetAttribute(awq_gemv_mma_kernel<DEPTH>, cudaFuncAttributeMaxDynamicSharedMemorySize, 227 * 1024);
     if (e != cudaSuccess) return e;
     attr_done[dev] = 1;
   }
   int per_sm = 0, sms = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, awq_gemv_stream_kernel, (kCW + 1) * 32, smem) !=
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, awq_gemv_mma_kernel<DEPTH>, warps * 32, smem) !=
           cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || per_sm <= 0)
     return cudaErrorLaunchOutOfResources;
+  const int slots = per_sm * sms;  // persistent grid: the blocks resident at once
   const int row_blocks = (N + 15) / 16;
-  const int slots = per_sm * sms;
-  const int blocks = row_blocks < slots ? row_blocks : slots;
-  awq_gemv_stream_kernel<<<blocks, (kCW + 1) * 32, smem, st>>>(X, M, wt, szt, bias, N, K, nslots, Y, err);
+  const int ks = pick_ks(K / kAwqGroup, row_blocks, slots, warps);
+  const int need = (row_blocks * ks + warps - 1) / warps;
+  const int blocks = need < slots ? need : slots;
+  awq_gemv_mma_kernel<DEPTH><<<blocks, warps * 32, smem, st>>>(X, M, wt, szt, bias, N, K, ks, Y);
   return cudaGetLastError();
+}
+
+cudaError_t launch_gemv(const uint16_t *X, int M, const uint8_t *wt, const uint8_t *szt, const float *bias, int N,
+                        int K, uint16_t *Y, cudaStream_t st) {
+  int warps, depth;
+  awq_shape(K, &warps, &depth);
+  switch (depth) {
+    case 16: return launch_gemv_depth<16>(X, M, wt, szt, bias, N, K, Y, warps, st);
+    case 8: return launch_gemv_depth<8>(X, M, wt, szt, bias, N, K, Y, warps, st);
+    case 4: return launch_gemv_depth<4>(X, M, wt, szt, bias, N, K, Y, warps, st);
+    case 2: return launch_gemv_depth<2>(X, M, wt, szt, bias, N, K, Y, warps, st);
+  }
+  return cudaErrorInvalidValue;
 }
 
 }  // namespace
 
 int awq_max_tokens() { return 8; }
-// Shared memory of the GEMV: staged activations (K/64 groups x 1 KiB of bf16 pairs), group sums (8
-// tokens x 4 bytes per group), the warps' partial sums, the ring of weight runs (as many slots as
-// fit, 12 at most, at least 2) and its barriers. The same for every token count up to 8.
-constexpr size_t kSmemLimit = 227 * 1024;
-size_t awq_fixed_smem(int K) { return static_cast<size_t>(K / kAwqGroup) * (1024 + 32) + kRedBytes; }
-int awq_slots(int K) {
-  const size_t fixed = awq_fixed_smem(K);
-  if (fixed >= kSmemLimit) return 0;
-  size_t n = (kSmemLimit - fixed) / (kSlotBytes + 16);
-  return static_cast<int>(n > static_cast<size_t>(kMaxSlots) ? kMaxSlots : n);
-}
-constexpr int kMaxK = 12288;  // the documented limit (at least two slots fit up to it)
-size_t awq_smem_bytes(int, int K) {
-  const int n = awq_slots(K);
-  if (n < 2 || K > kMaxK) return kSmemLimit + 1;  // too large: the caller rejects the shape
-  return awq_fixed_smem(K) + static_cast<size_t>(n) * (kSlotBytes + 16);
-}
 size_t awq_packed_weight_bytes(int N, int K) { return static_cast<size_t>((N + 15) / 16) * 16 * (K / 2); }
 size_t awq_packed_sz_bytes(int N, int K) { return static_cast<size_t>((N + 15) / 16) * (K / kAwqGroup) * 64; }
 
@@ -374,8 +408,8 @@ cudaError_t launch_awq_pack(const uint8_t *wq, const uint16_t *scales, const uin
 }
 
 cudaError_t launch_awq_gemv(const uint16_t *X, int M, const uint8_t *wt, const uint8_t *szt, const float *bias, int N,
-                            int K, uint16_t *Y, uint32_t *err, cudaStream_t st) {
-  return launch_gemv_stream(X, M, wt, szt, bias, N, K, Y, err, st);
+                            int K, uint16_t *Y, uint32_t *, cudaStream_t st) {
+  return launch_gemv(X, M, wt, szt, bias, N, K, Y, st);
 }
 
 }  // namespace svdq

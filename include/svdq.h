@@ -281,8 +281,8 @@ SVDQ_API svdq_status svdq_mlp_forward(const uint16_t *X, int M, const svdq_layer
  *   the tensor cores sum exact products (128 + q) x in fp32 per group of 64, and the scale and
  *   zero point are applied per group in fp32: s (D - (128 + z) sum x). X device M x K bf16 (16-byte aligned); wq_packed, sz_packed from
  *   svdq_awq_pack_weights; bias device N fp32 or NULL; Y device M x N bf16. K <= 12288 (the
- *   staged activations take K/64 KiB of shared memory beside a ring of at least two 9 KiB weight
- *   runs) and ceil(N/16) * K/64 < 2^26 tiles; otherwise SVDQ_ERR_INVALID_ARG.
+ *   staged activations take K/64 KiB of shared memory beside the warps' rings of weight tiles in
+ *   flight) and ceil(N/16) * K/64 < 2^26 tiles; otherwise SVDQ_ERR_INVALID_ARG.
  *   Asynchronous on stream. */
 SVDQ_API svdq_status svdq_awq_quantize_weights(const float *W, int N, int K, uint8_t *wq, uint16_t *scales,
                                                uint8_t *zeros, void *stream);
