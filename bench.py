@@ -608,21 +608,57 @@ def run_suite(args):
 
 def run_ncu_target(args, shape):
     """Launch list for ncu: prepare the workload, then `steps` back-to-back plain launches of one
-    kernel (k1, or k2 after one K1), without graphs, so that a capture of consecutive launches
-    (e.g. -k regex:k2_gemm -c 3 --cache-control none) counts the output each launch leaves in L2
-    against the next one. Prints one line; no timing."""
+    kernel (k1, or k2 after one K1; mlp: the fused MLP pair's middle kernel on the FLUX feed-forward
+    shapes; awq: the awq_w4a16 GEMV on the double-block modulation shape), without graphs, so that
+    a capture of consecutive launches (e.g. -k regex:k2_gemm -c 3 --cache-control none) counts the
+    output each launch leaves in L2 against the next one. Prints one line; no timing."""
     import torch
     from bit_rank_compensated_b200 import svdq
 
     svdq.load()
     dev = torch.device("cuda", 0)
+    stream = torch.cuda.current_stream()
+    if args.ncu_kernel == "awq":
+        from synth import make_modulation_inputs
+
+        M, K, N = AWQ_WORKLOADS["awq_mod"]
+        Xb, W, b = make_modulation_inputs(M, K, N)
+        lin = svdq.AwqLinear.from_float(torch.from_numpy(W).to(dev), torch.from_numpy(b).to(dev))
+        X = torch.from_numpy(Xb.view(np.int16)).to(dev).view(torch.bfloat16)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        for _ in range(args.steps):
+            svdq.awq_gemv_w4a16(X, lin, Y, stream)
+        torch.cuda.synchronize()
+        assert svdq.last_device_error() == 0
+        print(json.dumps({"ncu_target": "awq", "launches": args.steps}), flush=True)
+        return 0
+    if args.ncu_kernel == "mlp":
+        up_s, down_s = CONFIGS["mlp_up"], CONFIGS["mlp_down"]
+        M = up_s.M
+        Xb, Wu, bu, _ = make_inputs(up_s, seed=0)
+        _, Wd, bd, _ = make_inputs(down_s, seed=0)
+        X = torch.from_numpy(Xb.view(np.int16)).to(dev).view(torch.bfloat16)
+        up = svdq.prepare_weights(torch.from_numpy(Wu).to(dev), torch.from_numpy(bu).to(dev), svdq.act_absmax(X),
+                                  up_s.rank)
+        xq, xs, la = svdq.quant_act_lora_down(X, up)
+        H = svdq.gemm_w4a4_lora_up_gelu(xq, xs, la, M, up)
+        down = svdq.prepare_weights(torch.from_numpy(Wd).to(dev), torch.from_numpy(bd).to(dev), svdq.act_absmax(H),
+                                    down_s.rank)
+        del H
+        bufs = svdq.alloc_activations(M, down, dev)
+        ws = svdq.alloc_mlp_workspace(M, up, down, dev)
+        for _ in range(args.steps):
+            svdq.gemm_w4a4_lora_up_gelu_quant(xq, xs, la, M, up, down, bufs, ws, stream)
+        torch.cuda.synchronize()
+        assert svdq.last_device_error() == 0
+        print(json.dumps({"ncu_target": "mlp", "launches": args.steps}), flush=True)
+        return 0
     M, K, N, r = shape.M, shape.K, shape.N, shape.rank
     Xb, W, b, _ = make_inputs(shape, seed=0)
     X = torch.from_numpy(Xb.view(np.int16)).to(dev).view(torch.bfloat16)
     L = svdq.prepare_weights(torch.from_numpy(W).to(dev), torch.from_numpy(b).to(dev), svdq.act_absmax(X), r)
     xq, xs, la = svdq.alloc_activations(M, L, dev)
     Y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    stream = torch.cuda.current_stream()
     if args.ncu_kernel == "k2":
         svdq.quant_act_lora_down(X, L, xq, xs, la, stream)
     for _ in range(args.steps):
@@ -649,7 +685,7 @@ def main(argv=None):
                     help="seconds of untimed step replays inside the clock-sampling window before the timed region")
     ap.add_argument("--suite", nargs="?", const=",".join(SUITE), default=None,
                     help="time a comma-separated list of workloads (default: all) and print one line each")
-    ap.add_argument("--ncu-kernel", choices=["k1", "k2"], default=None,
+    ap.add_argument("--ncu-kernel", choices=["k1", "k2", "mlp", "awq"], default=None,
                     help="only launch one kernel `--steps` times back to back (for an ncu capture)")
     args = ap.parse_args(argv)
     args.warmup = max(args.warmup, 3)
