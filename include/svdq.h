@@ -272,7 +272,8 @@ SVDQ_API svdq_status svdq_mlp_forward(const uint16_t *X, int M, const svdq_layer
  *
  * svdq_awq_pack_weights: rearranges wq, scales and zeros (as above) into the layout the GEMV
  *   streams: per 16 rows x 64 columns a 512-byte tile of codes in tensor-core operand order and
- *   64 bytes of scales and zero points (rows padded to a multiple of 16 with zeros).
+ *   64 bytes of scales and zero points (fp16 s and fp16 128 + z per row; rows padded to a multiple
+ *   of 16 with zeros).
  *   wq_packed  device, svdq_awq_packed_weight_bytes(N, K) bytes, 16-byte aligned.
  *   sz_packed  device, svdq_awq_packed_sz_bytes(N, K) bytes, 16-byte aligned.
  *   Done once per layer. Asynchronous on stream.
@@ -283,7 +284,12 @@ SVDQ_API svdq_status svdq_mlp_forward(const uint16_t *X, int M, const svdq_layer
  *   svdq_awq_pack_weights; bias device N fp32 or NULL; Y device M x N bf16. K <= 12288 (the
  *   staged activations take K/64 KiB of shared memory beside the warps' rings of weight tiles in
  *   flight) and ceil(N/16) * K/64 < 2^26 tiles; otherwise SVDQ_ERR_INVALID_ARG.
- *   Asynchronous on stream. */
+ *   Asynchronous on stream, launched as a programmatic dependent launch: it may start under the
+ *   tail of the previous kernel of the stream and read wq_packed / sz_packed before that kernel
+ *   has finished (X, bias and Y only after), so those two buffers must not be written by a kernel
+ *   that triggers its dependents early (griddepcontrol.launch_dependents) right before this call;
+ *   svdq_awq_pack_weights and ordinary kernels do not. A lost wait inside the kernel (about two
+ *   seconds) sets the library's device error word. */
 SVDQ_API svdq_status svdq_awq_quantize_weights(const float *W, int N, int K, uint8_t *wq, uint16_t *scales,
                                                uint8_t *zeros, void *stream);
 SVDQ_API size_t svdq_awq_packed_weight_bytes(int N, int K);

@@ -8,15 +8,16 @@ def tile_layout(q, s, z):
     """The GEMV's tile layout written out from its definition (rows padded to 16): word st of
     lane L = 4 g + t of tile (rb, G), nibble j = 4 h + i, holds
     q[16 rb + g + 8 (i & 1)][64 G + 16 st + 2 t + 8 (i >> 1) + h]; the tile's 64 side bytes hold,
-    for each g, {s[row g], s[row g + 8]} as fp16, {z[row g], z[row g + 8]}, two zero bytes."""
+    for each g, {s[row g], s[row g + 8], 128 + z[row g], 128 + z[row g + 8]} as fp16."""
     N, K = q.shape
     Np = (N + 15) // 16 * 16
     qp = np.zeros((Np, K), np.uint32)
     qp[:N] = q
     sp = np.zeros((Np, K // 64), np.float16)
     sp[:N] = s.astype(np.float16)
-    zp = np.zeros((Np, K // 64), np.uint8)
-    zp[:N] = z
+    zp = np.zeros((Np, K // 64), np.float16)  # 128 + z (rows past N: z = 0)
+    zp[:] = 128
+    zp[:N] = 128 + z.astype(np.float64)
     wt = np.zeros((Np // 16, K // 64, 32, 4), np.uint32)
     szt = np.zeros((Np // 16, K // 64, 8, 8), np.uint8)
     for L in range(32):
@@ -31,8 +32,8 @@ def tile_layout(q, s, z):
         r0 = np.arange(Np // 16) * 16 + g
         szt[:, :, g, 0:2] = sp[r0].view(np.uint8).reshape(Np // 16, K // 64, 2)
         szt[:, :, g, 2:4] = sp[r0 + 8].view(np.uint8).reshape(Np // 16, K // 64, 2)
-        szt[:, :, g, 4] = zp[r0]
-        szt[:, :, g, 5] = zp[r0 + 8]
+        szt[:, :, g, 4:6] = zp[r0].view(np.uint8).reshape(Np // 16, K // 64, 2)
+        szt[:, :, g, 6:8] = zp[r0 + 8].view(np.uint8).reshape(Np // 16, K // 64, 2)
     return wt.reshape(-1).view(np.uint8), szt.reshape(-1)
 
 
@@ -60,7 +61,7 @@ def emulate_gemv(X, q, s, z):
     bytes into A registers i = 0..3 with halves (128 + nibble i, 128 + nibble i + 4); the MMA's
     fragments place register i at rows g + 8 (i & 1), columns 2 t + 8 (i >> 1) + (0, 1), and B
     registers b0 / b1 at columns (rows of B) 2 t + (0, 1) / 2 t + 8 + (0, 1), token g; then
-    acc += s D - s (128 + z) sum_G(x). Returns Y (M x N) without bias."""
+    acc += s (D - (128 + z) sum_G(x)). Returns Y (M x N) without bias."""
     M, K = X.shape
     N = q.shape[0]
     wt, szt = tile_layout(q, s, z)
@@ -88,11 +89,10 @@ def emulate_gemv(X, q, s, z):
                     B[2 * t + 8:2 * t + 10, g] = b[2 * st + 1]
                 D += A @ B
             for g in range(8):
-                sv = side[rb, G, g].view(np.float16).astype(np.float64)[:2]
-                zv = side[rb, G, g, 4:6].astype(np.float64)
+                sv = side[rb, G, g].view(np.float16).astype(np.float64)
                 sx = np.array([xb[G, 4 * m:4 * m + 4].sum() for m in range(8)])
                 for h in range(2):
                     r = g + 8 * h
-                    acc[r] += sv[h] * D[r] - sv[h] * (128 + zv[h]) * sx
+                    acc[r] += sv[h] * (D[r] - sv[2 + h] * sx)
         Y[:, 16 * rb:16 * rb + 16] = acc.T
     return Y[:M, :N]
