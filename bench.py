@@ -576,7 +576,14 @@ def run_suite(args):
                 "k1": {"us": k1_ms * 1e3, "gbs": k1_bytes(M, K, r) / (k1_ms * 1e-3) / 1e9,
                        "frac_hbm": k1_bytes(M, K, r) / (k1_ms * 1e-3) / 1e9 / hbm_gbs},
                 "k2": {"us": k2_ms * 1e3, "tflops": k2_flops(M, K, N, r) / (k2_ms * 1e-3) / 1e12,
-                       "frac_fp4": k2_flops(M, K, N, r) / (k2_ms * 1e-3) / 1e12 / fp4_peak},
+                       "frac_fp4": k2_flops(M, K, N, r) / (k2_ms * 1e-3) / 1e12 / fp4_peak,
+                       "gbs": k2_bytes(M, K, N, r) / (k2_ms * 1e-3) / 1e9,
+                       "frac_hbm": k2_bytes(M, K, N, r) / (k2_ms * 1e-3) / 1e9 / hbm_gbs,
+                       # the binding roof: the larger of the tensor time and the HBM time of the algorithmic work
+                       "binding": "tensor" if k2_flops(M, K, N, r) / (fp4_peak * 1e12) >= k2_bytes(M, K, N, r) / (hbm_gbs * 1e9)
+                       else "hbm",
+                       "frac_binding": max(k2_flops(M, K, N, r) / (fp4_peak * 1e12),
+                                           k2_bytes(M, K, N, r) / (hbm_gbs * 1e9)) / (k2_ms * 1e-3)},
                 "tokens_per_s": M / (step_ms * 1e-3), "peaks": peak_kind}
         if not qknr:
             plain_k2[shape.name] = k2_ms
