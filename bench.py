@@ -110,6 +110,38 @@ def kernel_traffic(kernel: str, workload: str):
     return None
 
 
+def host_link_times(Xh, Xd, Yh, Yd, dev, reps=5):
+    """Median ms of one step's host-to-device copy of X, device-to-host copy of Y, and both
+    together on two streams (pinned host buffers)."""
+    import torch
+
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def timed(fn):
+        out = []
+        for _ in range(reps):
+            torch.cuda.synchronize()
+            t0 = time.perf_counter()
+            fn()
+            torch.cuda.synchronize()
+            out.append((time.perf_counter() - t0) * 1e3)
+        return statistics.median(out)
+
+    def h2d():
+        with torch.cuda.stream(s_in):
+            Xd.copy_(Xh, non_blocking=True)
+
+    def d2h():
+        with torch.cuda.stream(s_out):
+            Yh.copy_(Yd, non_blocking=True)
+
+    h2d_ms = timed(h2d)
+    d2h_ms = timed(d2h)
+    both_ms = timed(lambda: (h2d(), d2h()))
+    return {"h2d_ms": h2d_ms, "d2h_ms": d2h_ms, "both_ms": both_ms,
+            "h2d_gbs": Xh.numel() * 2 / (h2d_ms * 1e-3) / 1e9, "d2h_gbs": Yh.numel() * 2 / (d2h_ms * 1e-3) / 1e9}
+
+
 def read_sustained_bf16():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -820,6 +852,9 @@ def main(argv=None):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1)
     e2e_ms = max_over_ranks(e2e_ms, dist, dev)
+    # the host link alone: one step's copy in and copy out (pinned), each direction timed alone and
+    # both at once on two streams; with the copies overlapped the step cannot beat the slower one
+    link = host_link_times(Xh, Xs[0], Yh, Ys[0], dev)
     if dist:
         dist.barrier()
         dist.destroy_process_group()
@@ -888,7 +923,11 @@ def main(argv=None):
         "tokens_per_s": world * M * args.steps / (total_ms * 1e-3),
         "cpu_baseline": cpu,
         "e2e": {"value": e2e_value, "unit": "TFLOPS", "h2d_bytes_per_step": int(M * K * 2),
-                "d2h_bytes_per_step": int(M * N * 2), "api": "svdq_linear_forward_host"},
+                "d2h_bytes_per_step": int(M * N * 2), "api": "svdq_linear_forward_host",
+                "ms_per_step": e2e_ms / e2e_steps,
+                # the copies alone (host clock, synchronised): the step's floor is both directions at once
+                "link": {k: round(v, 4) for k, v in link.items()},
+                "frac_of_link_floor": link["both_ms"] / (e2e_ms / e2e_steps)},
         "gpu_launches": 2 * args.steps,
         "clocks": clk.summary(),
         "clocks_burst": clk_b.summary(),

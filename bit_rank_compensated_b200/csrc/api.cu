@@ -48,6 +48,19 @@ void init_encode() {
 
 // Checks the current device once: compute capability 10.0 ("دعم الأجهزة": unsupported GPUs
 // get a clear error instead of wrong output) and records the SM count and the error word.
+// Copy streams and events of svdq_linear_forward_host's pipelined path, per device, created on
+// first use (a mutex serialises the calls that share them).
+constexpr int kHostChunks = 8;
+struct HostPipe {
+  std::once_flag once;
+  bool ok = false;
+  std::mutex mu;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t start = nullptr, end = nullptr;
+  cudaEvent_t in_done[kHostChunks] = {}, fwd_done[kHostChunks] = {};
+};
+HostPipe g_pipe[kMaxDevices];
+
 svdq_status device_check(DeviceState **out) {
   const int ov = g_cap_override.load(std::memory_order_relaxed);
   if (ov >= 0 && ov != 100) return SVDQ_ERR_UNSUPPORTED_ARCH;
@@ -120,6 +133,21 @@ CUtensorMapSwizzle swizzle_for_row_bytes(uint32_t b) {
 }
 
 float alpha_of(const svdq_layer *L) { return L->x_tensor_scale * L->w_tensor_scale; }
+
+HostPipe *host_pipe(DeviceState *d) {
+  HostPipe &p = g_pipe[d - g_dev];
+  std::call_once(p.once, [&]() {
+    bool ok = cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking) == cudaSuccess &&
+              cudaEventCreateWithFlags(&p.start, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventCreateWithFlags(&p.end, cudaEventDisableTiming) == cudaSuccess;
+    for (int i = 0; ok && i < kHostChunks; ++i)
+      ok = cudaEventCreateWithFlags(&p.in_done[i], cudaEventDisableTiming) == cudaSuccess &&
+           cudaEventCreateWithFlags(&p.fwd_done[i], cudaEventDisableTiming) == cudaSuccess;
+    p.ok = ok;
+  });
+  return p.ok ? &p : nullptr;
+}
 
 svdq_status run_quant(const uint16_t *X, int M, const svdq_layer *L, uint8_t *xq, uint8_t *xs, uint16_t *la,
                       bool quantize, bool lora, void *stream) {
@@ -636,11 +664,54 @@ svdq_status svdq_linear_forward_host(const uint16_t *X_host, int M, const svdq_l
   st = device_check(&d);
   if (st != SVDQ_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const size_t xb = static_cast<size_t>(M) * layer->K * 2, yb = static_cast<size_t>(M) * layer->N * 2;
-  if (cudaMemcpyAsync(X_dev, X_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess) return SVDQ_ERR_CUDA;
-  st = svdq_linear_forward(X_dev, M, layer, xq, xs, lora_act, Y_dev, stream);
-  if (st != SVDQ_OK) return st;
-  if (cudaMemcpyAsync(Y_host, Y_dev, yb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return SVDQ_ERR_CUDA;
+  const int K = layer->K, N = layer->N, r = layer->rank;
+  // Row chunks (multiples of 256 rows: whole K2 tiles and whole 128-row scale blocks, so each
+  // chunk's kernels write exactly the bytes the whole-M call would): the copy in of chunk i + 1
+  // and the copy out of chunk i - 1 run on their own streams while chunk i's kernels run on
+  // `stream`; the two copy directions use separate copy engines of the full-duplex link.
+  const int chunk = static_cast<int>(round_up(static_cast<size_t>((M + kHostChunks - 1) / kHostChunks), 256));
+  const int n_chunks = (M + chunk - 1) / chunk;
+  HostPipe *hp = n_chunks > 1 ? host_pipe(d) : nullptr;
+  if (!hp) {
+    const size_t xb = static_cast<size_t>(M) * K * 2, yb = static_cast<size_t>(M) * N * 2;
+    if (cudaMemcpyAsync(X_dev, X_host, xb, cudaMemcpyHostToDevice, s) != cudaSuccess) return SVDQ_ERR_CUDA;
+    st = svdq_linear_forward(X_dev, M, layer, xq, xs, lora_act, Y_dev, stream);
+    if (st != SVDQ_OK) return st;
+    if (cudaMemcpyAsync(Y_host, Y_dev, yb, cudaMemcpyDeviceToHost, s) != cudaSuccess) return SVDQ_ERR_CUDA;
+    return cudaStreamSynchronize(s) == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
+  }
+  std::lock_guard<std::mutex> lock(hp->mu);
+  auto fail = [&]() {
+    cudaStreamSynchronize(hp->in);
+    cudaStreamSynchronize(hp->out);
+    cudaStreamSynchronize(s);
+    return SVDQ_ERR_CUDA;
+  };
+  // the copies wait for the work already enqueued on `stream` (which may still use the buffers)
+  if (cudaEventRecord(hp->start, s) != cudaSuccess || cudaStreamWaitEvent(hp->in, hp->start, 0) != cudaSuccess ||
+      cudaStreamWaitEvent(hp->out, hp->start, 0) != cudaSuccess)
+    return fail();
+  for (int i = 0; i < n_chunks; ++i) {
+    const int r0 = i * chunk, mc = M - r0 < chunk ? M - r0 : chunk;
+    const size_t x0 = static_cast<size_t>(r0) * K, y0 = static_cast<size_t>(r0) * N;
+    if (cudaMemcpyAsync(X_dev + x0, X_host + x0, static_cast<size_t>(mc) * K * 2, cudaMemcpyHostToDevice, hp->in) !=
+            cudaSuccess ||
+        cudaEventRecord(hp->in_done[i], hp->in) != cudaSuccess || cudaStreamWaitEvent(s, hp->in_done[i], 0) != cudaSuccess)
+      return fail();
+    st = svdq_linear_forward(X_dev + x0, mc, layer, xq + x0 / 2, xs + static_cast<size_t>(r0) * (K / 16),
+                             r > 0 ? lora_act + static_cast<size_t>(r0) * 2 * r : lora_act, Y_dev + y0, stream);
+    if (st != SVDQ_OK) {
+      fail();
+      return st;
+    }
+    if (cudaEventRecord(hp->fwd_done[i], s) != cudaSuccess || cudaStreamWaitEvent(hp->out, hp->fwd_done[i], 0) != cudaSuccess ||
+        cudaMemcpyAsync(Y_host + y0, Y_dev + y0, static_cast<size_t>(mc) * N * 2, cudaMemcpyDeviceToHost, hp->out) !=
+            cudaSuccess)
+      return fail();
+  }
+  // `stream` is ordered after the last copy out
+  if (cudaEventRecord(hp->end, hp->out) != cudaSuccess || cudaStreamWaitEvent(s, hp->end, 0) != cudaSuccess)
+    return fail();
   return cudaStreamSynchronize(s) == cudaSuccess ? SVDQ_OK : SVDQ_ERR_CUDA;
 }
 

@@ -305,9 +305,14 @@ SVDQ_API svdq_status svdq_linear_forward(const uint16_t *X, int M, const svdq_la
                                 uint16_t *Y, void *stream);
 
 /* The forward pass from and to host memory: copies X_host (M x K bf16) to X_dev, runs
- * svdq_linear_forward, copies Y_dev (M x N bf16) back to Y_host, all enqueued on stream
- * (pinned host buffers make the copies asynchronous). Synchronous: returns after the
- * stream has finished. */
+ * svdq_linear_forward, copies Y_dev (M x N bf16) back to Y_host. For M > 256 it runs in row
+ * chunks of a multiple of 256 rows (up to 8): the kernels of a chunk run on stream while the next
+ * chunk is copied in and the previous one copied out on two streams of the library's own (one per
+ * copy direction, created on first use and ordered after the work already on stream), so the
+ * copies of both directions overlap each other and the kernels; the result is the whole-M call's,
+ * bit for bit. Pinned host buffers make the copies asynchronous (pageable ones work, without the
+ * overlap). Synchronous: returns after the last copy out; concurrent calls on one device take
+ * turns. */
 SVDQ_API svdq_status svdq_linear_forward_host(const uint16_t *X_host, int M, const svdq_layer *layer,
                                      uint16_t *X_dev, uint8_t *xq, uint8_t *xs,
                                      uint16_t *lora_act, uint16_t *Y_dev, uint16_t *Y_host,

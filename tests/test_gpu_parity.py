@@ -220,6 +220,30 @@ def test_forward_host_buffers(lib):
     assert rel_err_floor(bf16_tensor_to_np(Yh).reshape(Y_ref.shape), Y_ref) <= Y_TOL
 
 
+@pytest.mark.parametrize("M,rank", [(300, 32), (1100, 16), (1024, 0), (1, 32)])
+def test_forward_host_buffers_chunked(lib, M, rank):
+    # the host-buffer path runs in row chunks of multiples of 256 rows (copies overlapping the
+    # kernels of the neighbouring chunks): the output must be the whole-M device call's, bit for
+    # bit, from pinned and from pageable host buffers
+    Xb, X, W, b = _problem(_shape(M, 768, 512, rank), seed=M)
+    layer_o = O.prepare(W, b, O.calibration_absmax(X), rank)
+    Ld = to_device_layer(layer_o)
+    Xd0 = x_to_device(Xb)
+    Y_dev = lib.linear_forward(Xd0, Ld)
+    torch.cuda.synchronize()
+    want = Y_dev.view(torch.int16).cpu().numpy()
+    for pinned in (True, False):
+        Xh = torch.from_numpy(Xb.view(np.int16)).view(torch.bfloat16)
+        Yh = torch.empty(M, Ld.N, dtype=torch.bfloat16)
+        if pinned:
+            Xh, Yh = Xh.pin_memory(), Yh.pin_memory()
+        Xd = torch.empty(M, Ld.K, dtype=torch.bfloat16, device="cuda")
+        Yd = torch.empty(M, Ld.N, dtype=torch.bfloat16, device="cuda")
+        lib.linear_forward_host(Xh, Ld, Xd, lib.alloc_activations(M, Ld), Yd, Yh)
+        np.testing.assert_array_equal(Yh.view(torch.int16).numpy(), want)
+    assert lib.last_device_error() == 0
+
+
 # ------------------------------------------------------------------ prepare
 def _bits(t):
     return t.view(torch.int16).cpu().numpy().view(np.uint16)
