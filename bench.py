@@ -93,21 +93,29 @@ def k2_bytes(M, K, N, r):
 
 def kernel_traffic(kernel: str, workload: str):
     """DRAM bytes per launch of `kernel` ("k1" or "k2") from the committed ncu capture of
-    consecutive launches (profiles/<kernel>_traffic.json), if it was taken on the current source
-    of that kernel (the file records its sha1) and this workload; otherwise None."""
-    import hashlib
-
+    consecutive launches (profiles/<kernel>_traffic.json), if it was taken on the current sources
+    of that kernel (the file records the sha1 of kernel_sources_sha1) and this workload; otherwise
+    None."""
     tr_path = os.path.join(ROOT, "profiles", f"{kernel}_traffic.json")
-    src = os.path.join(ROOT, "bit_rank_compensated_b200", "csrc", {"k1": "quant_act.cu", "k2": "gemm.cu"}[kernel])
-    if not (os.path.exists(tr_path) and os.path.exists(src)):
+    if not os.path.exists(tr_path):
         return None
     with open(tr_path) as f:
         tr = json.load(f)
-    with open(src, "rb") as f:
-        sha = hashlib.sha1(f.read()).hexdigest()
-    if tr.get("workload") == workload and tr.get("source_sha1") == sha:
+    if tr.get("workload") == workload and tr.get("source_sha1") == kernel_sources_sha1(kernel):
         return tr.get("bytes_per_launch")
     return None
+
+
+def kernel_sources_sha1(kernel: str) -> str:
+    """sha1 over the kernel's source file and the device headers it includes, in that order."""
+    import hashlib
+
+    csrc = os.path.join(ROOT, "bit_rank_compensated_b200", "csrc")
+    h = hashlib.sha1()
+    for name in ({"k1": "quant_act.cu", "k2": "gemm.cu"}[kernel], "common.cuh", "nvfp4.cuh"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
 
 
 def host_link_times(Xh, Xd, Yh, Yd, dev, reps=5):

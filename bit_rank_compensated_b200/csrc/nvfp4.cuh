@@ -52,13 +52,17 @@ __device__ __forceinline__ f2 mul2(f2 a, f2 b) {
 constexpr float kBracketLo = 1.0f - 9.5367431640625e-07f;  // 1 - 2^-20
 constexpr float kBracketHi = 1.0f + 9.5367431640625e-07f;  // 1 + 2^-20
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
 __device__ __forceinline__ float absmax16(const float *v) {
-  float m[8];
+  float m[6];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m[i] = fmaxf(fabsf(v[i]), fabsf(v[i + 8]));
-#pragma unroll
-  for (int i = 0; i < 4; ++i) m[i] = fmaxf(m[i], m[i + 4]);
-  return fmaxf(fmaxf(m[0], m[2]), fmaxf(m[1], m[3]));
+  for (int i = 0; i < 5; ++i) m[i] = max3(fabsf(v[3 * i]), fabsf(v[3 * i + 1]), fabsf(v[3 * i + 2]));
+  m[5] = fabsf(v[15]);
+  return fmaxf(max3(m[0], m[1], m[2]), max3(m[3], m[4], m[5]));
 }
 
 // e4m3 code of the correctly rounded quotient fp32(amax / d). Kept out of line: it is needed only
