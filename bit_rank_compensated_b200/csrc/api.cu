@@ -632,7 +632,7 @@ svdq_status svdq_awq_gemv_w4a16(const uint16_t *X, int M, const uint8_t *wq_pack
   if (!X || !wq_packed || !sz_packed || !Y || N <= 0 || K <= 0 || K % 64 || M <= 0 || M > awq_max_tokens() ||
       awq_smem_bytes(M, K) > 227u * 1024u)
     return SVDQ_ERR_INVALID_ARG;
-  // the kernel walks the tiles with 32-bit indices (times 32 lanes)
+  // the documented tile limit (the pack kernel runs 32 threads per tile, a grid of < 2^31 threads)
   if (static_cast<uint64_t>((N + 15) / 16) * static_cast<uint64_t>(K / 64) >= (1ull << 26)) return SVDQ_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(wq_packed) || !aligned16(sz_packed)) return SVDQ_ERR_MISALIGNED;
   DeviceState *d = nullptr;

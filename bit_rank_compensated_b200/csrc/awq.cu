@@ -125,13 +125,11 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// Tensor-core GEMV, bound by reading the 4-bit weights once. What keeps it at the memory's
-// rate is the number of bytes in flight per SM: every warp streams its own tiles into a ring of
-// shared-memory slots with bulk copies (the copy engine, one copy of a step's codes and one of its
-// side bytes, completing on the slot's mbarrier), up to 16 tiles ahead, with no register held per
-// tile in flight (one CTA of 16 warps per SM: ~147 KiB in flight; per-lane 16-byte copies tracked
-// by the load path capped the stream near 2.4 TB/s). Each lane's 16 bytes of a tile are exactly
-// its operand-A registers.
+// Tensor-core GEMV, bound by reading the 4-bit weights once. Every warp streams its own tiles
+// into a ring of shared-memory slots with bulk copies (the copy engine: one copy of a step's codes
+// and one of its side bytes, completing on the slot's mbarrier), up to 16 tiles ahead, with no
+// register held per tile in flight (one CTA of 16 warps per SM: ~147 KiB in flight; the loop finds
+// every step already landed). Each lane's 16 bytes of a tile are exactly its operand-A registers.
 // Per tile: an m16n8k16 bf16 MMA per k-step with the 16 weight rows of the row block as operand A
 // (each code q turned into the exact bf16 integer 128 + q in registers, one LOP3 per pair) and up
 // to 8 tokens as operand B (the bf16 activations, staged once per CTA in fragment order, zeros in
@@ -152,9 +150,9 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 constexpr int kMaxWarps = 16;
 constexpr uint32_t kTileSlot = 576; // 512 bytes of codes + 64 of scales and zero points
 
-// Shared-memory loads of the main loop with the state space explicit (a generic load of a shared
-// address is tracked like a global one); volatile keeps them after the cp.async wait, with no
-// memory clobber so that the compiler may still schedule the other loads around them.
+// Shared-memory loads of the main loop with the state space explicit; volatile keeps them after the
+// slot's mbarrier wait, with no memory clobber so that the compiler may still schedule the other
+// loads around them.
 constexpr int kMaxSlots = 16;  // mbarriers reserved per warp
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
   uint4 v;
