@@ -238,6 +238,25 @@ class ClockSampler:
         return out
 
 
+def clock_snapshot(gpu_index: int = 0):
+    """One nvidia-smi reading of the SM clock and the active throttle reasons, taken right after a
+    workload's timed region (the clock state it ran in); None where nvidia-smi is missing."""
+    try:
+        out = subprocess.run(["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={ClockSampler.Q}",
+                              "--format=csv,noheader,nounits"], capture_output=True, text=True, timeout=10).stdout
+    except (FileNotFoundError, subprocess.TimeoutExpired):
+        return None
+    f = [x.strip() for x in out.strip().split(",")]
+    if len(f) < 10:
+        return None
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    try:
+        return {"sm_mhz": float(f[2]), "sm_max_mhz": float(f[3]),
+                "reasons": [n for n, v in zip(names, f[6:10]) if v.lower() == "active"]}
+    except ValueError:
+        return None
+
+
 def cpu_model() -> str:
     try:
         with open("/proc/cpuinfo") as f:
@@ -585,7 +604,7 @@ def run_suite(args):
                 "mlp_pair": {"fused_us": f_ms * 1e3, "unfused_us": u_ms * 1e3, "unfused_over_fused": u_ms / f_ms,
                              "fused_middle_us": mid_ms * 1e3,
                              "intermediate_bytes_saved": 2 * 2 * us.M * us.N},
-                "peaks": peak_kind}), flush=True)
+                "clocks_after": clock_snapshot(), "peaks": peak_kind}), flush=True)
             torch.cuda.empty_cache()
             continue
         if name in AWQ_WORKLOADS:
@@ -600,7 +619,7 @@ def run_suite(args):
                            "M": M, "K": K, "N": N},
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm_gbs, "unit": "GB/s", "frac": gbs / hbm_gbs,
                              "bytes_per_launch": awq_bytes(M, K, N)},
-                "peaks": peak_kind}), flush=True)
+                "clocks_after": clock_snapshot(), "peaks": peak_kind}), flush=True)
             torch.cuda.empty_cache()
             continue
         qknr = name.endswith("_qknorm_rope")
@@ -624,7 +643,7 @@ def run_suite(args):
                        else "hbm",
                        "frac_binding": max(k2_flops(M, K, N, r) / (fp4_peak * 1e12),
                                            k2_bytes(M, K, N, r) / (hbm_gbs * 1e9)) / (k2_ms * 1e-3)},
-                "tokens_per_s": M / (step_ms * 1e-3), "peaks": peak_kind}
+                "tokens_per_s": M / (step_ms * 1e-3), "clocks_after": clock_snapshot(), "peaks": peak_kind}
         if not qknr:
             plain_k2[shape.name] = k2_ms
         else:
