@@ -74,8 +74,12 @@ def _oracle_linear(lib, M, N, K, seed, with_bias=True):
 
 # K = 128 and 256 give 2 and 4 groups per row, so 2 and 4 warps share a row block (the other
 # shapes use 1 or 8)
+# The launch shape (warps, tiles in flight, warps per row block, groups per step) depends on K and
+# N; these cover every compiled (ring slots, groups per step) pair: (4,4) (2,4) (8,2) (2,2) (4,2)
+# (16,1) (8,1) (4,1) (2,1), and odd group counts per slice.
 @pytest.mark.parametrize("M,N,K", [(1, 18432, 3072), (2, 9216, 3072), (3, 333, 576), (5, 64, 1024), (8, 130, 6144),
-                                   (1, 1, 64), (7, 4100, 12288), (1, 1000, 128), (2, 1000, 256)])
+                                   (1, 1, 64), (7, 4100, 12288), (1, 1000, 128), (2, 1000, 256), (1, 24000, 4224),
+                                   (1, 96, 4160), (1, 500, 10560), (2, 300, 11840)])
 def test_gemv_matches_oracle(lib, M, N, K):
     Xb, lin, Y_ref = _oracle_linear(lib, M, N, K, seed=M, with_bias=M != 5)
     Y = lib.awq_gemv_w4a16(x_to_device(Xb), lin)
