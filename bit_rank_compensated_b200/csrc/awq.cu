@@ -246,8 +246,8 @@ __global__ void __launch_bounds__(kMaxWarps * 32, 1) awq_gemv_mma_kernel(const u
   };
   // Prologue. The launch may overlap the tail of the previous kernel of the stream (programmatic
   // dependent launch): the first step of the ring is requested before the dependency wait, since
-  // the packed weights are a layer's constants (the caller may not write them in the kernel just
-  // before this one); the activations, which that kernel may produce, only after it. They are
+  // the packed weights are a layer's constants, complete before that kernel began (the interface
+  // requires it); the activations, which that kernel may produce, only after the wait. They are
   // requested before the rest of the ring: ~150 KiB of weight copies per SM queued ahead of them
   // in the memory system delayed them by about 3 us.
   issue();

@@ -347,12 +347,15 @@ def awq_pack_weights(wq, scales, zeros, stream=None):
 
 
 class AwqLinear:
-    """A packed awq_w4a16 weight (N x K) with its bias, ready for awq_gemv_w4a16."""
+    """A packed awq_w4a16 weight (N x K) with its bias, ready for awq_gemv_w4a16. Built at load
+    time: the constructor waits for the packing to finish, since the GEMV may read the packed
+    weights before the kernel just before it on its stream has finished."""
 
     def __init__(self, wq, scales, zeros, bias=None, stream=None):
         self.N, self.K = wq.shape[0], 2 * wq.shape[1]
         self.wt, self.szt = awq_pack_weights(wq, scales, zeros, stream)
         self.bias = bias
+        (stream if stream is not None else torch.cuda.current_stream(wq.device)).synchronize()
 
     @classmethod
     def from_float(cls, W: torch.Tensor, bias=None, stream=None):

@@ -285,11 +285,11 @@ SVDQ_API svdq_status svdq_mlp_forward(const uint16_t *X, int M, const svdq_layer
  *   staged activations take K/64 KiB of shared memory beside the warps' rings of weight tiles in
  *   flight) and ceil(N/16) * K/64 < 2^26 tiles; otherwise SVDQ_ERR_INVALID_ARG.
  *   Asynchronous on stream, launched as a programmatic dependent launch: it may start under the
- *   tail of the previous kernel of the stream and read wq_packed / sz_packed before that kernel
- *   has finished (X, bias and Y only after), so those two buffers must not be written by a kernel
- *   that triggers its dependents early (griddepcontrol.launch_dependents) right before this call;
- *   svdq_awq_pack_weights and ordinary kernels do not. A lost wait inside the kernel (about two
- *   seconds) sets the library's device error word. */
+ *   tail of the previous kernel of the stream and read wq_packed / sz_packed before waiting for
+ *   that kernel (X, bias and Y only after the wait), so the packed weights must be complete before
+ *   the kernel launched just before this call on the stream begins: pack them at load time, or
+ *   put an event or a synchronization between svdq_awq_pack_weights and the first GEMV. A lost
+ *   wait inside the kernel (about two seconds) sets the library's device error word. */
 SVDQ_API svdq_status svdq_awq_quantize_weights(const float *W, int N, int K, uint8_t *wq, uint16_t *scales,
                                                uint8_t *zeros, void *stream);
 SVDQ_API size_t svdq_awq_packed_weight_bytes(int N, int K);
