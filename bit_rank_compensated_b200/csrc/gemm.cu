@@ -784,9 +784,9 @@ __global__ void __launch_bounds__(THREADS, 1)
           const int wrow0 = nt * BN + static_cast<int>(crank) * BNH;  // this CTA's rows of W
           for (int j = 0; j < total; ++j, ++it) {
             const int s = it % ST;
-            // spin rather than park: a parked thread wakes measurably later, and this round trip
-            // (slot released -> loads issued -> stage full) is the kernel's critical path
-            if (it >= ST && !mbar_wait(bar_empty + 8 * s, ((it / ST) - 1) & 1, a.err, KID_GEMM, 1)) {
+            // parked rather than spinning: the spinning loop's instructions cost the MMA warp
+            // issue slots and the SM power, and under the power cap the step ran faster parked
+            if (it >= ST && !mbar_wait_parked(bar_empty + 8 * s, ((it / ST) - 1) & 1, a.err, KID_GEMM, 1)) {
               ok = false;
               break;
             }
@@ -997,8 +997,9 @@ __global__ void __launch_bounds__(THREADS, 1)
       for (int step = h; step < nsteps; step += 2) {
         const int s = step % ST;
         const int j = step % total;
-        // sffull of this step: its scale blocks are in shared memory and slot s is free
-        if (!__all_sync(0xffffffffu, mbar_wait(bar_sf + 8 * (2 * s + h), (step / SF_PERIOD) & 1, a.err, KID_GEMM, 6)))
+        // sffull of this step: its scale blocks are in shared memory and slot s is free (parked,
+        // as the producer's wait)
+        if (!__all_sync(0xffffffffu, mbar_wait_parked(bar_sf + 8 * (2 * s + h), (step / SF_PERIOD) & 1, a.err, KID_GEMM, 6)))
           break;
         if (FP4 && j >= N_LORA) {
           const int kt = j - N_LORA;
