@@ -89,3 +89,36 @@ def test_binding_argument_counts_match_the_header(lib):
                 assert t in (ctypes.c_int, ctypes.c_uint32), (name, p, t)
             elif re.match(r"(const\s+)?float\b", p):
                 assert t is ctypes.c_float, (name, p, t)
+
+
+def _declared_returns():
+    """{name: return type} parsed from include/svdq.h."""
+    src = open(os.path.join(ROOT, "include", "svdq.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return {m.group(2): " ".join(m.group(1).split())
+            for m in re.finditer(r"SVDQ_API\s+([^;(]*?)\b(svdq_\w+)\s*\(", src, flags=re.S)}
+
+
+def test_binding_types_match_the_header(lib):
+    # every parameter and return type is bound with a ctypes type of the same width: size_t as
+    # c_size_t (a 32-bit binding would truncate workspace sizes), enums and int as c_int
+    import ctypes
+
+    scalar = {"int": (ctypes.c_int,), "uint32_t": (ctypes.c_uint32, ctypes.c_int), "float": (ctypes.c_float,),
+              "size_t": (ctypes.c_size_t,), "svdq_status": (ctypes.c_int,)}
+    for name, params in _declared_params().items():
+        f = getattr(lib, name)
+        for p, t in zip(params, f.argtypes):
+            if "*" in p:
+                continue  # pointers: checked by the count test
+            base = re.sub(r"^const\s+", "", p).split()[0]
+            assert base in scalar, (name, p)
+            assert t in scalar[base], (name, p, t)
+    for name, ret in _declared_returns().items():
+        f = getattr(lib, name)
+        if ret.endswith("*"):
+            assert f.restype is ctypes.c_char_p, (name, ret, f.restype)
+        else:
+            base = re.sub(r"^const\s+", "", ret).split()[-1]
+            assert base in scalar, (name, ret)
+            assert f.restype in scalar[base], (name, ret, f.restype)
