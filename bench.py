@@ -21,7 +21,8 @@ same stream. The e2e number goes through the host-buffer entry point call by cal
 Metric: layer TFLOPS = (2MNK + 2MNr + 2MKr) / step time, summed over ranks (weak scaling:
 every rank runs its own replica on its own batch, no collective on the data path).
 Rank 0 prints one JSON line. ``--impl reference`` times the fp64 CPU oracle instead (the
-only reference implementation of this method available here) on a bounded row sample.
+only reference implementation of this method available here): W untimed warm-up steps, then K
+timed steps, each step one bounded slice of the workload's tokens.
 
 ``--suite`` also covers the fused QKV layer with the Q/K normalization + rotary output stage
 (``qkv_qknorm_rope``: against the plain K2 and against plain K2 + the separate step) and the
@@ -269,10 +270,11 @@ def cpu_model() -> str:
 
 
 def cpu_oracle_sample(shape, rows: int, seed: int = 0, budget_s: float = 20.0, threads: int | None = None,
-                      layer=None, X=None):
+                      layer=None, X=None, steps: int | None = None, warmup: int = 0):
     """Times the fp64 oracle's forward pass (quantize + down-projection + dequantized GEMM +
-    up-projection) on `rows`-token slices of the workload for about budget_s seconds; the SVD
-    prepare is timed apart. threads: BLAS thread limit (None: numpy's default pool)."""
+    up-projection) on `rows`-token slices of the workload: for about budget_s seconds, or, with
+    `steps`, for exactly that many slices after `warmup` untimed ones; the SVD prepare is timed
+    apart. threads: BLAS thread limit (None: numpy's default pool)."""
     from oracle import svdq_oracle as O
     from synth import bf16_bits_to_f32
 
@@ -291,8 +293,10 @@ def cpu_oracle_sample(shape, rows: int, seed: int = 0, budget_s: float = 20.0, t
 
     ctx = threadpool_limits(threads) if (threads and threadpool_limits) else contextlib.nullcontext()
     with ctx:
+        for w in range(warmup):
+            O.layer_forward(X[(w * rows) % shape.M:(w * rows) % shape.M + rows], layer)
         done, t_fwd, reps = 0, 0.0, 0
-        while t_fwd < budget_s and reps < 64:
+        while (reps < steps) if steps is not None else (t_fwd < budget_s and reps < 64):
             sl = X[(reps * rows) % shape.M:(reps * rows) % shape.M + rows]
             t0 = time.perf_counter()
             O.layer_forward(sl, layer)
@@ -308,21 +312,31 @@ def cpu_oracle_sample(shape, rows: int, seed: int = 0, budget_s: float = 20.0, t
             "prepare_s": t_prep, "reps": reps, "layer": layer, "X": X}
 
 
+def reference_rows(steps: int) -> int:
+    """Tokens per step of the reference arm: 256, halved while K steps would exceed 16384 tokens
+    (about a minute of the fp64 oracle on the host cores), at least 16."""
+    rows = 256
+    while rows > 16 and steps * rows > 16384:
+        rows //= 2
+    return rows
+
+
 def run_reference(args, shape, rank, world):
     if rank != 0:
         return 0
-    rows = 256
-    res = cpu_oracle_sample(shape, rows, budget_s=max(5.0, min(60.0, 2.0 * args.steps)))
+    rows = reference_rows(args.steps)
+    res = cpu_oracle_sample(shape, rows, steps=args.steps, warmup=args.warmup)
     ms = res["seconds"] / res["reps"] * 1e3
     res1 = cpu_oracle_sample(shape, 64, budget_s=8.0, threads=1, layer=res["layer"], X=res["X"])
     line = {
         "impl": "reference", "metric": METRIC, "value": res["value"], "unit": "TFLOPS", "n_gpus": args.gpus,
-        "steps": res["reps"], "warmup": 0, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "steps": res["reps"], "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": workload_name(shape), "M": shape.M, "K": shape.K, "N": shape.N, "rank": shape.rank},
         "cpu_baseline": {"value": res["value"], "unit": "TFLOPS", "cores": res["cores"], "kind": "oracle",
-                         "sample": f"{res['reps']} slices of {rows} tokens ({res['tokens']} tokens) of the workload; "
-                                   f"fp64 numpy oracle forward pass, prepare (SVD) excluded ({res['prepare_s']:.1f} s)",
+                         "sample": f"{res['reps']} timed steps of {rows} tokens ({res['tokens']} tokens) of the "
+                                   f"workload after {args.warmup} untimed ones; fp64 numpy oracle forward pass, "
+                                   f"prepare (SVD) excluded ({res['prepare_s']:.1f} s)",
                          "cpu_model": cpu_model(), "nproc": os.cpu_count(),
                          "single_thread": {"value": res1["value"], "unit": "TFLOPS",
                                            "sample": f"{res1['reps']} slices of 64 tokens, 1 BLAS thread"}},
