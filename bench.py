@@ -312,19 +312,16 @@ def cpu_oracle_sample(shape, rows: int, seed: int = 0, budget_s: float = 20.0, t
             "prepare_s": t_prep, "reps": reps, "layer": layer, "X": X}
 
 
-def reference_rows(steps: int) -> int:
-    """Tokens per step of the reference arm: 256, halved while K steps would exceed 16384 tokens
-    (about a minute of the fp64 oracle on the host cores), at least 16."""
-    rows = 256
-    while rows > 16 and steps * rows > 16384:
-        rows //= 2
-    return rows
+# Tokens per step of the reference arm. A step of the oracle costs about the same for any slice
+# up to a few hundred tokens (each call first dequantizes the whole weight), so smaller slices
+# would not shorten the run, only lower the measured rate.
+REFERENCE_ROWS = 256
 
 
 def run_reference(args, shape, rank, world):
     if rank != 0:
         return 0
-    rows = reference_rows(args.steps)
+    rows = min(REFERENCE_ROWS, shape.M)
     res = cpu_oracle_sample(shape, rows, steps=args.steps, warmup=args.warmup)
     ms = res["seconds"] / res["reps"] * 1e3
     res1 = cpu_oracle_sample(shape, 64, budget_s=8.0, threads=1, layer=res["layer"], X=res["X"])
